@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Benchmark of the MSA decode step (indexer -> max-pool -> top-16 -> sparse
+attention) on B200, one process per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Multi-GPU: launch with torch.distributed.run (one rank per GPU); the path
+shards by sequence, so every rank decodes its own batch of the workload with
+no data-path collective (weak scaling); the only collectives are the timing
+barrier and the max-over-ranks of the measured time.
+
+Prints one JSON line (rank 0).  `value` is whole-job decode queries/s (query
+tokens of all ranks per second), device-timed with CUDA events; `roofline`
+describes the kernel with the largest time share; `e2e` repeats the step
+through the Python binding with host (pinned) query buffers copied in and the
+output copied out inside the timed region; `cpu_baseline` times the float64
+oracle on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MSA decode queries/s and achieved HBM GB/s (% of B200 peak) at 128K ctx"
+DEFAULT_WORKLOAD = "ctx128k_b64_t8"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ ranks --
+def rank_info():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Every rank decodes its own batch: same shapes, its own seed."""
+    return 7919 * rank
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- peaks --
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_sha(files) -> str:
+    h = hashlib.sha1()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+KERNEL_SOURCES = {
+    "indexer": ["block_sparse_attention_decode_b200/csrc/msa_indexer.cu",
+                "block_sparse_attention_decode_b200/csrc/msa_device.cuh"],
+    "attention": ["block_sparse_attention_decode_b200/csrc/msa_attn.cu",
+                  "block_sparse_attention_decode_b200/csrc/msa_device.cuh"],
+    "topk": ["block_sparse_attention_decode_b200/csrc/msa_topk.cu"],
+}
+
+
+def dram_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel, {})
+    if d.get("workload") != workload or d.get("source_sha") != source_sha(KERNEL_SOURCES[kernel]):
+        return None
+    return d.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks --
+def smi_index(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ byte model --
+def algorithmic_bytes(w, sel):
+    """Bytes the traffic model of the method implies for one step: the full
+    index-key scan, the selected K/V only (each distinct block of a (sequence,
+    group) once, over the union of its query tokens' selections, counting only
+    the visible tokens of a partial block), the queries and the output."""
+    import torch
+    lens = w.seq_lens.long()
+    idx_per_tok = 128 if w.idx_fp8 else 72
+    idx_bytes = int(lens.sum().item()) * idx_per_tok
+    B, T = w.batch, w.q_tokens
+    s = sel.long()                                        # [B][T][4][16]
+    mp = w.max_pages
+    mark = torch.zeros(B, 4, mp + 1, dtype=torch.bool, device=s.device)
+    flat = torch.where(s >= 0, s, torch.full_like(s, mp))  # -1 -> dummy column
+    mark.scatter_(2, flat.permute(0, 2, 1, 3).reshape(B, 4, T * 16), True)
+    mark = mark[:, :, :mp]
+    blk = torch.arange(mp, device=s.device)
+    valid_tok = (lens.view(B, 1) - blk.view(1, mp) * 128).clamp(0, 128)   # tokens in block
+    kv_tokens = int((mark.to(torch.int64) * valid_tok.view(B, 1, mp)).sum().item())
+    kv_bytes = kv_tokens * 144
+    q_bytes = B * T * (64 * 128 + 4 * 128)
+    out_bytes = B * T * 64 * 128 * 2
+    return {"index_scan": idx_bytes, "kv_selected": kv_bytes, "queries": q_bytes,
+            "output": out_bytes, "total": idx_bytes + kv_bytes + q_bytes + out_bytes,
+            "kv_tokens": kv_tokens}
+
+
+# --------------------------------------------------------- CPU baseline --
+def cpu_sample_workload(name: str, seed_offset: int = 0):
+    """One sequence with the shapes of `name` (its full context, all of its
+    query tokens), generated on the host: a bounded sample of the workload."""
+    from block_sparse_attention_decode_b200 import synth
+    kw = dict(synth.WORKLOADS[name])
+    if kw["seq_lens"] is None:
+        kw["seq_lens"] = synth.ragged_lengths(kw["batch"], 2048, 262144, kw["seed"])
+    L = max(kw["seq_lens"])
+    kw.update(batch=1, seq_lens=[L], seed=kw["seed"] + 100 + seed_offset)
+    if kw.get("plant_every"):
+        kw["plant_every"] = kw["plant_every"]
+    return synth.make_workload(name + "_cpu_sample", device="cpu", **kw)
+
+
+def oracle_step(w, tokens, threads):
+    import numpy as np
+    import oracle
+    oracle.set_threads(threads)
+    n = lambda t: None if t is None else t.numpy()
+    c = oracle.Cache(idx_data=n(w.idx_data), idx_scale=n(w.idx_scale), k_data=n(w.k_data),
+                     k_scale=n(w.k_scale), v_data=n(w.v_data), v_scale=n(w.v_scale),
+                     s_idx=w.s_idx, s_k=w.s_k, s_v=w.s_v, page_table=n(w.page_table),
+                     max_pages=w.max_pages, seq_lens=n(w.seq_lens), q_tokens=w.q_tokens)
+    rows = [(0, t) for t in tokens]
+    t0 = time.perf_counter()
+    oracle.decode(c, np.ascontiguousarray(n(w.qi)), w.s_qi, np.ascontiguousarray(n(w.q)), w.s_q,
+                  w.softmax_scale, rows)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(name: str, budget_s: float = 20.0):
+    w = cpu_sample_workload(name)
+    threads = max(1, min(os.cpu_count() or 1, w.q_tokens))
+    tokens = list(range(w.q_tokens))
+    dt = oracle_step(w, tokens, threads)
+    reps = 1
+    while dt * (reps + 1) / reps < budget_s and reps < 3:
+        dt += oracle_step(w, tokens, threads)
+        reps += 1
+    qps = reps * len(tokens) / dt
+    return {"value": qps, "unit": "queries/s", "cores": threads, "kind": "oracle",
+            "sample": "%d x (1 sequence of %d tokens, its %d query tokens: full index scan, "
+                      "top-16, attention) of %s, float64 C oracle" % (reps, int(w.seq_lens[0]),
+                                                                    w.q_tokens, name)}
+
+
+# ------------------------------------------------------------- GPU arm ----
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import block_sparse_attention_decode_b200 as msa
+    from block_sparse_attention_decode_b200 import build as msa_build
+    from block_sparse_attention_decode_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    if rank == 0 or not os.path.exists(msa.LIB_PATH):
+        msa_build.build()
+    barrier(world)
+    msa.load()
+    name = args.workload
+    kw = dict(synth.WORKLOADS[name])
+    if kw["seq_lens"] is None:
+        kw["seq_lens"] = synth.ragged_lengths(kw["batch"], 2048, 262144, kw["seed"])
+    kw["seed"] += rank_seed_offset(rank)
+    w = synth.make_workload(name, device="cuda", **kw)
+    cache, seqs = msa.cache_of(w), msa.seqs_of(w)
+    ws = msa.alloc_workspace(seqs)
+    B, T = w.batch, w.q_tokens
+    out = torch.empty(B, T, 64, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(B, T, 4, 16, dtype=torch.int32, device="cuda")
+    bscores = torch.empty(B, T, 4, w.max_pages, dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")   # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step():
+        msa.msa_decode(cache, seqs, w.qi, w.s_qi, w.q, w.s_q, w.softmax_scale, out, sel, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, detail = msa.msa_get_last_error(ws)
+    if st != msa.MSA_OK:
+        raise RuntimeError("device error %d (%d) during warm-up" % (st, detail))
+
+    # ---- timed region: K steps, L2 flushed before each (outside the events)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(smi_index(local_rank)) as clk:
+        t_wall = time.perf_counter()
+        for e0, e1 in evs:
+            flush.fill_(1)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    barrier(world)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    ms_max = max_over_ranks(ms, world)
+    clocks = clk.summary()
+
+    # ---- per-kernel times (the same kernels through the stage entry points)
+    names = ("indexer", "topk", "attention")
+    per = {k: 0.0 for k in names}
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(stream)
+        msa.msa_indexer_score(cache, seqs, w.qi, w.s_qi, None, bscores, ws, stream)
+        e[1].record(stream)
+        msa.msa_block_maxpool_topk(bscores, False, seqs, sel, ws, stream)
+        e[2].record(stream)
+        msa.msa_sparse_attn_decode(cache, seqs, w.q, w.s_q, sel, w.softmax_scale, out, ws, stream)
+        e[3].record(stream)
+        torch.cuda.synchronize()
+        for i, k in enumerate(names):
+            per[k] += e[i].elapsed_time(e[i + 1]) / args.steps
+    st, detail = msa.msa_get_last_error(ws)
+    if st != msa.MSA_OK:
+        raise RuntimeError("device error %d (%d) during timing" % (st, detail))
+
+    bytes_ = algorithmic_bytes(w, sel)
+    kernel_bytes = {"indexer": bytes_["index_scan"] + B * T * 512 + B * T * 4 * w.max_pages * 4,
+                    "topk": B * T * 4 * w.max_pages * 4 + B * T * 4 * 16 * 4,
+                    "attention": bytes_["kv_selected"] + B * T * 64 * 128 * 3 + B * T * 4 * 16 * 4}
+    dom = max(names, key=lambda k: per[k])
+    peak, peak_src = measured_peaks()
+    achieved = kernel_bytes[dom] / (per[dom] * 1e-3) / 1e9
+    traffic = dram_traffic(dom, name)
+
+    # ---- end to end through the binding: host queries in, output out
+    h_qi = w.qi.cpu().pin_memory()
+    h_q = w.q.cpu().pin_memory()
+    h_lens = w.seq_lens.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_qi, d_q, d_lens = torch.empty_like(w.qi), torch.empty_like(w.q), torch.empty_like(w.seq_lens)
+    seqs_e2e = msa.Seqs(d_lens, T, w.max_pages, w.page_table)
+
+    def e2e_step():
+        d_qi.copy_(h_qi, non_blocking=True)
+        d_q.copy_(h_q, non_blocking=True)
+        d_lens.copy_(h_lens, non_blocking=True)
+        msa.msa_decode(cache, seqs_e2e, d_qi, w.s_qi, d_q, w.s_q, w.softmax_scale, out, None, ws,
+                       stream)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    for e0, e1 in ev2:
+        flush.fill_(1)
+        e0.record(stream)
+        e2e_step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / args.steps, world)
+    h2d = h_qi.numel() + h_q.numel() + h_lens.numel() * 4
+    d2h = h_out.numel() * 2
+
+    result = None
+    if rank == 0:
+        q_total = B * T * world
+        value = q_total / (ms_max * 1e-3)
+        gbs = bytes_["total"] / (ms * 1e-3) / 1e9
+        result = {
+            "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3", "data": "synthetic",
+            "config": {"workload": name, "batch_per_gpu": B, "context": int(w.seq_lens.max()),
+                       "q_tokens": T, "index_keys": "fp8" if w.idx_fp8 else "nvfp4",
+                       "kv_cache": "nvfp4, 128-token pages" + (", shuffled page table"
+                                                                 if w.page_table is not None else ""),
+                       "global_batch": B * world, "parallelism": "dp%d" % world,
+                       "l2": "256 MiB written before each timed step (outside the events); "
+                             "inputs %.1f GB > 126 MB L2" % (
+                                 (w.idx_data.numel() + 2 * (w.k_data.numel() + w.k_scale.numel())
+                                  + (w.idx_scale.numel() if w.idx_scale is not None else 0)) / 1e9)},
+            "hbm": {"algorithmic_bytes_per_step": bytes_["total"], "achieved_gbs": gbs,
+                    "frac_of_measured": gbs / peak, "frac_of_spec_8000": gbs / SPEC_HBM_GBS,
+                    "peak_source": peak_src, "bytes": bytes_},
+            "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": kernel_bytes[dom],
+                         "peak_source": peak_src},
+            "kernel_ms": per,
+            "gpu_launches": 3 * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"]},
+            "e2e": {"value": q_total / (ms_e2e * 1e-3), "unit": "queries/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+            "wall_s_timed_region": t_wall,
+        }
+    return result
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local_rank = rank_info()
+
+    if args.impl == "reference":
+        # The reference arm is the float64 oracle on the host cores, rank 0 only.
+        if rank != 0:
+            return 0
+        w = cpu_sample_workload(args.workload)
+        threads = max(1, min(os.cpu_count() or 1, w.q_tokens))
+        tokens = list(range(w.q_tokens))
+        for _ in range(args.warmup):
+            oracle_step(w, tokens[:1], threads)
+        t = sum(oracle_step(w, tokens, threads) for _ in range(args.steps))
+        qps = args.steps * len(tokens) / t
+        sample = ("per step: 1 sequence of %d tokens (shapes of %s), its %d query tokens through "
+                  "the float64 C oracle (full index scan, top-16, attention)"
+                  % (int(w.seq_lens[0]), args.workload, len(tokens)))
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample": sample},
+            "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            res["cpu_baseline"] = cpu_baseline(args.workload)
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

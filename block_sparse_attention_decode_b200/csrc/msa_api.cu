@@ -1,0 +1,264 @@
+// msa_api.cu -- the C ABI declared in include/msa.h: argument checks, the
+// workspace layout, the work planner and the kernel launches.
+#include <cmath>
+#include <cstring>
+
+#include "msa.h"
+#include "msa_internal.h"
+
+using namespace msa;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 148; }
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return sms;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool good_scale(float s) { return std::isfinite(s) && s > 0.f; }
+
+// Workspace layout (byte offsets).
+struct Layout {
+  size_t flags, bscores, sel, counters, partials, total;
+  int splits;
+};
+
+bool seqs_ok(const msa_seqs* s) {
+  if (!s || !s->seq_lens) return false;
+  if (!aligned16(s->seq_lens) || (s->page_table && !aligned16(s->page_table))) return false;
+  if (s->batch < 1 || s->batch > MSA_MAX_BATCH || s->q_tokens < 1 || s->max_pages < 1) return false;
+  if ((long long)s->max_pages * MSA_BLOCK_TOKENS < s->q_tokens) return false;
+  if ((long long)s->max_pages * MSA_BLOCK_TOKENS > 0x7FFFFFFFLL) return false;
+  const long long rows = (long long)s->batch * s->q_tokens * MSA_KV_HEADS;
+  return rows <= 0x7FFFFFFFLL / MSA_TOPK;
+}
+
+Layout layout_for(const msa_seqs* s, int sms) {
+  Layout L{};
+  const long long rows = (long long)s->batch * s->q_tokens * kG;
+  L.splits = attn_splits(rows, sms);
+  size_t off = 0;
+  L.flags = off;    off += align_up(sizeof(Flags));
+  L.bscores = off;  off += align_up((size_t)rows * s->max_pages * sizeof(float));
+  L.sel = off;      off += align_up((size_t)rows * kTopk * sizeof(int32_t));
+  L.counters = off; off += align_up((size_t)rows * sizeof(int));
+  L.partials = off;
+  if (L.splits > 1) off += align_up((size_t)rows * L.splits * kPartialFloats * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+msa_status check_cache(const msa_cache* c, bool need_index, bool need_kv) {
+  if (!c) return MSA_ERR_INVALID_ARG;
+  if (c->num_pages < 1) return MSA_ERR_INVALID_ARG;
+  if (need_index) {
+    if (c->idx_dtype != MSA_IDX_NVFP4 && c->idx_dtype != MSA_IDX_FP8) return MSA_ERR_INVALID_ARG;
+    if (!c->idx_data || !aligned16(c->idx_data)) return MSA_ERR_INVALID_ARG;
+    if (c->idx_dtype == MSA_IDX_NVFP4 && (!c->idx_scale || !aligned16(c->idx_scale)))
+      return MSA_ERR_INVALID_ARG;
+    if (!good_scale(c->s_idx)) return MSA_ERR_INVALID_ARG;
+  }
+  if (need_kv) {
+    const uint8_t* p[4] = {c->k_data, c->k_scale, c->v_data, c->v_scale};
+    for (const uint8_t* x : p)
+      if (!x || !aligned16(x)) return MSA_ERR_INVALID_ARG;
+    if (!good_scale(c->s_k) || !good_scale(c->s_v)) return MSA_ERR_INVALID_ARG;
+  }
+  return MSA_OK;
+}
+
+msa_status check_ws(const msa_seqs* s, void* ws, size_t ws_bytes, Layout* L) {
+  *L = layout_for(s, device_sms());
+  if (!ws || !aligned16(ws) || ws_bytes < L->total) return MSA_ERR_WORKSPACE;
+  return MSA_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off); }
+
+msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi, float s_qi,
+                       float* token_scores, float* block_scores, void* ws, const Layout& L,
+                       cudaStream_t st) {
+  IdxArgs a{};
+  a.idx_data = c->idx_data;
+  a.idx_scale = c->idx_scale;
+  a.page_table = s->page_table;
+  a.seq_lens = s->seq_lens;
+  a.qi = qi;
+  a.token_scores = token_scores;
+  a.block_scores = block_scores;
+  a.flags = at<Flags>(ws, L.flags);
+  a.score_scale = s_qi * c->s_idx;
+  a.B = s->batch;
+  a.T = s->q_tokens;
+  a.max_pages = s->max_pages;
+  a.num_pages = c->num_pages;
+  return cuda_status(launch_indexer(a, c->idx_dtype == MSA_IDX_FP8, device_sms(), st));
+}
+
+msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, float s_q,
+                    const int32_t* sel, float softmax_scale, uint16_t* out, void* ws,
+                    const Layout& L, cudaStream_t st) {
+  const long long rows = (long long)s->batch * s->q_tokens * kG;
+  if (L.splits > 1) {
+    cudaError_t e = cudaMemsetAsync(at<int>(ws, L.counters), 0, (size_t)rows * sizeof(int), st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+  }
+  AttnArgs a{};
+  a.k_data = c->k_data;
+  a.k_scale = c->k_scale;
+  a.v_data = c->v_data;
+  a.v_scale = c->v_scale;
+  a.page_table = s->page_table;
+  a.seq_lens = s->seq_lens;
+  a.q = q;
+  a.sel = sel;
+  a.out = out;
+  a.partials = at<float>(ws, L.partials);
+  a.counters = at<int>(ws, L.counters);
+  a.flags = at<Flags>(ws, L.flags);
+  a.logit_scale_log2 = (float)((double)softmax_scale * s_q * c->s_k * 1.4426950408889634);
+  a.out_scale = c->s_v;
+  a.B = s->batch;
+  a.T = s->q_tokens;
+  a.max_pages = s->max_pages;
+  a.num_pages = c->num_pages;
+  a.splits = L.splits;
+  return cuda_status(launch_attn(a, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t msa_workspace_size(const msa_seqs* seqs) {
+  if (!seqs_ok(seqs)) return 0;
+  return layout_for(seqs, device_sms()).total;
+}
+
+msa_status msa_workspace_init(void* ws, size_t ws_bytes, msa_stream_t stream) {
+  if (!ws || ws_bytes < sizeof(Flags)) return MSA_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, align_up(sizeof(Flags)) <= ws_bytes ? align_up(sizeof(Flags)) : ws_bytes,
+                                     (cudaStream_t)stream));
+}
+
+msa_status msa_indexer_score(const msa_cache* cache, const msa_seqs* seqs, const uint8_t* qi,
+                             float s_qi, float* token_scores, float* block_scores, void* ws,
+                             size_t ws_bytes, msa_stream_t stream) {
+  if (!seqs_ok(seqs)) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_cache(cache, true, false);
+  if (st != MSA_OK) return st;
+  if (!qi || !aligned16(qi) || !block_scores || !aligned16(block_scores) || !good_scale(s_qi))
+    return MSA_ERR_INVALID_ARG;
+  if (token_scores && !aligned16(token_scores)) return MSA_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  return run_indexer(cache, seqs, qi, s_qi, token_scores, block_scores, ws, L,
+                     (cudaStream_t)stream);
+}
+
+msa_status msa_block_maxpool_topk(const float* scores, int32_t is_token_level, const msa_seqs* seqs,
+                                  int32_t* sel, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  if (!seqs_ok(seqs)) return MSA_ERR_INVALID_ARG;
+  if (!scores || !aligned16(scores) || !sel || !aligned16(sel)) return MSA_ERR_INVALID_ARG;
+  if (is_token_level != 0 && is_token_level != 1) return MSA_ERR_INVALID_ARG;
+  Layout L;
+  msa_status st = check_ws(seqs, ws, ws_bytes, &L);
+  if (st != MSA_OK) return st;
+  const cudaStream_t s = (cudaStream_t)stream;
+  const float* bs = scores;
+  if (is_token_level) {
+    float* dst = at<float>(ws, L.bscores);
+    st = cuda_status(launch_maxpool(scores, seqs->seq_lens, seqs->batch, seqs->q_tokens,
+                                    seqs->max_pages, dst, at<Flags>(ws, L.flags), s));
+    if (st != MSA_OK) return st;
+    bs = dst;
+  }
+  return cuda_status(launch_topk(bs, seqs->seq_lens, seqs->batch, seqs->q_tokens, seqs->max_pages,
+                                 sel, at<Flags>(ws, L.flags), s));
+}
+
+msa_status msa_sparse_attn_decode(const msa_cache* cache, const msa_seqs* seqs, const uint8_t* q,
+                                  float s_q, const int32_t* sel, float softmax_scale,
+                                  uint16_t* out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  if (!seqs_ok(seqs)) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_cache(cache, false, true);
+  if (st != MSA_OK) return st;
+  if (!q || !aligned16(q) || !sel || !aligned16(sel) || !out || !aligned16(out))
+    return MSA_ERR_INVALID_ARG;
+  if (!good_scale(s_q) || !good_scale(softmax_scale)) return MSA_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  return run_attn(cache, seqs, q, s_q, sel, softmax_scale, out, ws, L, (cudaStream_t)stream);
+}
+
+msa_status msa_decode(const msa_cache* cache, const msa_seqs* seqs, const uint8_t* qi, float s_qi,
+                      const uint8_t* q, float s_q, float softmax_scale, uint16_t* out,
+                      int32_t* sel_out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  if (!seqs_ok(seqs)) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_cache(cache, true, true);
+  if (st != MSA_OK) return st;
+  if (!qi || !aligned16(qi) || !q || !aligned16(q) || !out || !aligned16(out))
+    return MSA_ERR_INVALID_ARG;
+  if (sel_out && !aligned16(sel_out)) return MSA_ERR_INVALID_ARG;
+  if (!good_scale(s_qi) || !good_scale(s_q) || !good_scale(softmax_scale))
+    return MSA_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  const cudaStream_t s = (cudaStream_t)stream;
+  float* bs = at<float>(ws, L.bscores);
+  int32_t* sel = sel_out ? sel_out : at<int32_t>(ws, L.sel);
+  if ((st = run_indexer(cache, seqs, qi, s_qi, nullptr, bs, ws, L, s)) != MSA_OK) return st;
+  st = cuda_status(launch_topk(bs, seqs->seq_lens, seqs->batch, seqs->q_tokens, seqs->max_pages,
+                               sel, at<Flags>(ws, L.flags), s));
+  if (st != MSA_OK) return st;
+  return run_attn(cache, seqs, q, s_q, sel, softmax_scale, out, ws, L, s);
+}
+
+msa_status msa_get_last_error(void* ws, msa_stream_t stream, int32_t* detail) {
+  if (!ws) return MSA_ERR_WORKSPACE;
+  const cudaStream_t s = (cudaStream_t)stream;
+  Flags h{};
+  if (cudaMemcpyAsync(&h, ws, sizeof(Flags), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (detail) *detail = h.detail;
+  if (h.code != 0) {
+    const Flags zero{};
+    if (cudaMemcpyAsync(ws, &zero, sizeof(Flags), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return MSA_ERR_CUDA;
+  }
+  return (msa_status)h.code;
+}
+
+msa_status msa_debug_nvfp4_table(uint8_t* out, msa_stream_t stream) {
+  if (!out || !aligned16(out)) return MSA_ERR_INVALID_ARG;
+  return cuda_status(launch_nvfp4_table(out, (cudaStream_t)stream));
+}
+
+const char* msa_status_string(msa_status status) {
+  switch (status) {
+    case MSA_OK: return "ok";
+    case MSA_ERR_INVALID_ARG: return "invalid argument";
+    case MSA_ERR_UNSUPPORTED: return "unsupported request";
+    case MSA_ERR_CUDA: return "CUDA runtime error";
+    case MSA_ERR_DEVICE_BOUNDS: return "device bounds check failed (page id, block id or length)";
+    case MSA_ERR_TIMEOUT: return "device wait timed out";
+    case MSA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

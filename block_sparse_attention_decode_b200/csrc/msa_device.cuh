@@ -1,0 +1,181 @@
+// msa_device.cuh -- device helpers shared by the MSA kernels (sm_100a).
+//
+// NVFP4 -> E4M3 decode.  [post, "NVIDIA Blackwell optimized MSA kernels"]
+// (post = vLLM 為 MiniMax-M3.1-Flash 提供 Day-0 支援, hot.atechcom.net) feeds
+// an FP8 MMA, so each E2M1 code times its E4M3 block scale is rounded back to
+// E4M3.  The toolkit here (CUDA 12.9) has no e2m1 x e4m3 scale-multiply
+// instruction, so the rounding is tabulated: for each of the 256 scale bytes
+// the 8 E2M1 magnitudes times the scale, rounded by the CUDA fp8 conversion
+// (round-to-nearest-even, satfinite), make one 8-byte row of a 2 KB shared
+// table (the table-lookup idea of [post, "AMD GPU support", "NVFP4 MSA
+// kernel"], rebuilt for PTX `prmt`).  Four codes then decode with one byte
+// permute for the magnitudes and one for the signs.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+namespace msa {
+
+constexpr int kBlock = 128;      // tokens per block / page
+constexpr int kDim = 128;        // head dim
+constexpr int kG = 4;            // KV heads = GQA groups
+constexpr int kHpg = 16;         // query heads per group
+constexpr int kHq = kG * kHpg;   // query heads
+constexpr int kTopk = 16;        // selected blocks
+constexpr int kRowCodes = 64;    // bytes of NVFP4 codes per 128-vector
+constexpr int kRowScales = 8;    // E4M3 scale bytes per 128-vector
+constexpr int kPageCodes = kBlock * kRowCodes;    // 8192
+constexpr int kPageScales = kBlock * kRowScales;  // 1024
+
+// Workspace header: device error flags (first 256 bytes of the workspace).
+struct Flags {
+  int code;     // first msa_status recorded on the device (0 = none)
+  int detail;   // the offending value
+};
+
+__device__ __forceinline__ void report(Flags* f, int code, int detail) {
+  if (atomicCAS(&f->code, 0, code) == 0) atomicExch(&f->detail, detail);
+}
+
+// ----------------------------------------------------------- NVFP4 table --
+// lut[s] = {E4M3(m*e4m3(s)) for m = 0..3 in .x, m = 4..7 in .y}, m indexing
+// the E2M1 magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6} (OCP MX v1.0).
+__device__ __forceinline__ void build_nvfp4_lut(uint2* lut, int tid, int nthreads) {
+  const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+  for (int i = tid; i < 512; i += nthreads) {
+    const int s = i >> 1, half = i & 1;
+    __nv_fp8_e4m3 sc;
+    sc.__x = (__nv_fp8_storage_t)s;
+    const float scale = float(sc);
+    uint32_t word = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      // the product of a 2-bit and a 4-bit significand is exact in fp32
+      const float prod = mag[4 * half + k] * scale;
+      const uint32_t b = __nv_cvt_float_to_fp8(prod, __NV_SATFINITE, __NV_E4M3);
+      word |= (b & 0xFFu) << (8 * k);
+    }
+    if (half) lut[s].y = word; else lut[s].x = word;
+  }
+}
+
+// Decode 8 codes (one 32-bit word: element n in nibble n) with table row r.
+// o0 = elements 0..3, o1 = elements 4..7 (E4M3 bytes, element order kept).
+__device__ __forceinline__ void dq8(uint32_t w, uint2 r, uint32_t& o0, uint32_t& o1) {
+  const uint32_t mag = w & 0x77777777u;
+  const uint32_t sgn = (w >> 3) & 0x11111111u;
+  o0 = __byte_perm(r.x, r.y, mag) ^ __byte_perm(0x00008000u, 0u, sgn);
+  o1 = __byte_perm(r.x, r.y, mag >> 16) ^ __byte_perm(0x00008000u, 0u, sgn >> 16);
+}
+
+// Decode 32 consecutive elements (16 code bytes, 2 scale bytes) into 8 words:
+// out[m] = elements 4m..4m+3.
+__device__ __forceinline__ void dq32(const uint2* lut, uint4 c, uint32_t sc2, uint32_t (&out)[8]) {
+  const uint2 r0 = lut[sc2 & 0xFFu];
+  const uint2 r1 = lut[(sc2 >> 8) & 0xFFu];
+  dq8(c.x, r0, out[0], out[1]);
+  dq8(c.y, r0, out[2], out[3]);
+  dq8(c.z, r1, out[4], out[5]);
+  dq8(c.w, r1, out[6], out[7]);
+}
+
+// ------------------------------------------------------------ FP8 MMA -----
+// D(16x8 f32) += A(16x32 e4m3, row) * B(32x8 e4m3, col).
+//   a0:(row g, k 4t..4t+3) a1:(row g+8, same k) a2:(row g, k 16+4t..) a3:(row g+8, ..)
+//   b0:(k 4t..4t+3, col g)  b1:(k 16+4t.., col g)
+//   d0:(row g, col 2t) d1:(row g, col 2t+1) d2:(row g+8, col 2t) d3:(row g+8, col 2t+1)
+// with g = lane/4, t = lane%4.
+__device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two fp32 -> packed E4M3x2 (lo in the low byte), RNE, satfinite.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  return pack_e4m3x2(a, b) | (pack_e4m3x2(c, d) << 16);
+}
+
+// -------------------------------------------- mbarrier + bulk async copy --
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// One bulk copy global -> shared (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Bounded wait on an mbarrier phase.  Returns false after the iteration limit
+// (each try_wait itself suspends for a bounded, hardware-defined time).
+constexpr uint32_t kSpinLimit = 1u << 20;
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n"
+        "selp.b32 %0, 1, 0, P;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+__device__ __forceinline__ uint32_t lds16(const void* p) {
+  return *reinterpret_cast<const uint16_t*>(p);
+}
+
+// Order-preserving map float -> uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_float(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(u);
+}
+
+}  // namespace msa

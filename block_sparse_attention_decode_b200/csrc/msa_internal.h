@@ -1,0 +1,68 @@
+// msa_internal.h -- kernel argument blocks and launchers shared between the
+// C-ABI layer (msa_api.cu) and the kernel files.  Not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "msa_device.cuh"
+
+namespace msa {
+
+constexpr int kIdxConsumers = 4;
+constexpr int kIdxThreads = (kIdxConsumers + 1) * 32;
+constexpr int kIdxStages = 8;
+
+struct IdxArgs {
+  const uint8_t* idx_data;     // NVFP4 codes [P][128][64] or FP8 keys [P][128][128]
+  const uint8_t* idx_scale;    // [P][128][8] (NVFP4 only)
+  const int32_t* page_table;   // [B][max_pages] or null
+  const int32_t* seq_lens;     // [B]
+  const uint8_t* qi;           // [B][T][4][128] E4M3
+  float* token_scores;         // [B][T][4][max_pages*128] or null
+  float* block_scores;         // [B][T][4][max_pages]
+  Flags* flags;
+  float score_scale;           // s_qi * s_idx
+  int B, T, max_pages, num_pages;
+};
+
+size_t indexer_smem_bytes(bool fp8idx, int batch);
+int indexer_ntiles(int T);
+cudaError_t launch_indexer(const IdxArgs& a, bool fp8idx, int num_sms, cudaStream_t st);
+
+// Top-k over block scores of every (b, t, g) row.
+cudaError_t launch_topk(const float* block_scores, const int32_t* seq_lens, int B, int T,
+                        int max_pages, int32_t* sel, Flags* flags, cudaStream_t st);
+// Max-pool token scores [B][T][4][max_pages*128] into block scores.
+cudaError_t launch_maxpool(const float* token_scores, const int32_t* seq_lens, int B, int T,
+                           int max_pages, float* block_scores, Flags* flags, cudaStream_t st);
+
+constexpr int kAttConsumers = 4;
+constexpr int kAttThreads = (kAttConsumers + 1) * 32;
+constexpr int kAttStages = 4;
+constexpr int kPartialFloats = kHpg * kDim + 2 * kHpg;   // O[16][128], m[16], l[16]
+
+struct AttnArgs {
+  const uint8_t *k_data, *k_scale, *v_data, *v_scale;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const uint8_t* q;            // [B][T][64][128] E4M3
+  const int32_t* sel;          // [B][T][4][16]
+  uint16_t* out;               // [B][T][64][128] bf16
+  float* partials;             // [units][splits][kPartialFloats]
+  int* counters;               // [units]
+  Flags* flags;
+  float logit_scale_log2;      // softmax_scale * s_q * s_k * log2(e)
+  float out_scale;             // s_v
+  int B, T, max_pages, num_pages, splits;
+};
+
+size_t attn_smem_bytes();
+int attn_splits(long long units, int num_sms);
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
+
+// The kernels' NVFP4 -> E4M3 table for all (scale, code) pairs.
+cudaError_t launch_nvfp4_table(uint8_t* out, cudaStream_t st);
+
+}  // namespace msa
