@@ -137,7 +137,10 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which: str):
+        setattr(self, which, time.time())
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -150,7 +153,10 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0, t1 = getattr(self, "start", 0.0), getattr(self, "stop", float("inf"))
+        for ts, ln in self.lines:
+            if not (t0 <= ts <= t1 + 0.15):
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -259,6 +265,9 @@ def run_gpu(args, rank, world, local_rank):
     kw = dict(synth.WORKLOADS[name])
     if kw["seq_lens"] is None:
         kw["seq_lens"] = synth.ragged_lengths(kw["batch"], 2048, 262144, kw["seed"])
+    if args.batch:
+        kw["seq_lens"] = (list(kw["seq_lens"]) * args.batch)[: args.batch]
+        kw["batch"] = args.batch
     kw["seed"] += rank_seed_offset(rank)
     w = synth.make_workload(name, device="cuda", **kw)
     cache, seqs = msa.cache_of(w), msa.seqs_of(w)
@@ -273,6 +282,7 @@ def run_gpu(args, rank, world, local_rank):
     def step():
         msa.msa_decode(cache, seqs, w.qi, w.s_qi, w.q, w.s_q, w.softmax_scale, out, sel, ws, stream)
 
+    clk = ClockSampler(smi_index(local_rank)).__enter__()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -285,19 +295,18 @@ def run_gpu(args, rank, world, local_rank):
            for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(smi_index(local_rank)) as clk:
-        t_wall = time.perf_counter()
-        for e0, e1 in evs:
-            flush.fill_(1)
-            e0.record(stream)
-            step()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        t_wall = time.perf_counter() - t_wall
+    clk.mark("start")
+    t_wall = time.perf_counter()
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
     barrier(world)
     ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
     ms_max = max_over_ranks(ms, world)
-    clocks = clk.summary()
 
     # ---- per-kernel times (the same kernels through the stage entry points)
     names = ("indexer", "topk", "attention")
@@ -356,6 +365,9 @@ def run_gpu(args, rank, world, local_rank):
         e2e_step()
         e1.record(stream)
     torch.cuda.synchronize()
+    clk.mark("stop")
+    clk.__exit__(None, None, None)
+    clocks = clk.summary()
     ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / args.steps, world)
     h2d = h_qi.numel() + h_q.numel() + h_lens.numel() * 4
     d2h = h_out.numel() * 2
@@ -370,7 +382,7 @@ def run_gpu(args, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8_e4m3", "data": "synthetic",
-            "config": {"workload": name, "batch_per_gpu": B, "context": int(w.seq_lens.max()),
+            "config": {"workload": name if not args.batch else "%s (batch %d)" % (name, B), "batch_per_gpu": B, "context": int(w.seq_lens.max()),
                        "q_tokens": T, "index_keys": "fp8" if w.idx_fp8 else "nvfp4",
                        "kv_cache": "nvfp4, 128-token pages" + (", shuffled page table"
                                                                  if w.page_table is not None else ""),
@@ -400,9 +412,11 @@ def run_gpu(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -1,5 +1,6 @@
 // msa_api.cu -- the C ABI declared in include/msa.h: argument checks, the
 // workspace layout, the work planner and the kernel launches.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -139,6 +140,30 @@ msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, flo
 }
 
 }  // namespace
+
+namespace msa {
+
+int ctas_per_sm(const void* kernel, int threads, size_t smem, int tmem_cols) {
+  int dev = 0, smem_sm = 0, regs_sm = 0, max_threads = 0;
+  cudaFuncAttributes fa{};
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaFuncGetAttributes(&fa, kernel) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&max_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
+  const int warps = (threads + 31) / 32;
+  const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;      // allocation granularity
+  int n = regs_warp > 0 ? regs_sm / (regs_warp * warps) : 1;
+  const size_t per_cta_smem = smem + fa.sharedSizeBytes + 1024;      // 1 KB reserved per CTA
+  n = std::min<long long>(n, (long long)(smem_sm / per_cta_smem));
+  n = std::min(n, max_threads / (warps * 32));
+  if (tmem_cols > 0) n = std::min(n, 512 / tmem_cols);
+  return n < 1 ? 1 : n;
+}
+
+}  // namespace msa
 
 extern "C" {
 

@@ -42,11 +42,14 @@ int attn_splits(long long units, int num_sms) {
   return s;
 }
 
-// key (within a warp's 32) held as S column n of n-tile j:
-//   pi(j, n) = 4*(n/2) + 2*(j%2) + n%2 + 16*(j/2)
-// so thread tig holds keys 4tig..4tig+3 (n-tiles 0,1) and 16+4tig..+3 (2,3).
+// Key (within a warp's 32) held as S column n of n-tile j:
+//   pi(j, n) = 4*(2j + n%2) + n/2.
+// Thread tig then holds the keys congruent to tig mod 4, which is exactly the
+// set its P A-fragment needs when the V^T word of key quad q holds keys
+// q, q+8, q+16, q+24; and each K or V load instruction of the warp covers 8
+// consecutive rows of the stage (bank-conflict free).
 __device__ __forceinline__ int key_of(int j, int n) {
-  return 4 * (n >> 1) + 2 * (j & 1) + (n & 1) + 16 * (j >> 1);
+  return 4 * (2 * j + (n & 1)) + (n >> 1);
 }
 
 // 4x4 byte transpose: x[r] byte e -> y[e] byte r.
@@ -185,13 +188,13 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(AttnArgs a) {
                    kw[2 * st], kw[2 * st + 1]);
       }
 
-      // ---- V^T tile: lane (kq, dc) decodes keys 4kq..4kq+3, dims 32dc..32dc+31
+      // ---- V^T tile: lane (kq, dc) decodes keys kq + 8r (r = 0..3), dims 32dc..32dc+31
       {
         const int kq = lane >> 2, dc = lane & 3;
         uint32_t vw[4][8];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const int kk = 32 * warp + 4 * kq + r;
+          const int kk = 32 * warp + kq + 8 * r;
           dq32(lut, lds128(vc + kk * kRowCodes + 16 * dc), lds16(vs + kk * kRowScales + 2 * dc), vw[r]);
         }
 #pragma unroll
@@ -243,22 +246,29 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(AttnArgs a) {
       }
 #pragma unroll
       for (int r = 0; r < 2; ++r) l_run[r] = l_run[r] * alpha[r] + ps[r];
+      if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        o[nt][0] *= alpha[0]; o[nt][1] *= alpha[0];
-        o[nt][2] *= alpha[1]; o[nt][3] *= alpha[1];
+        for (int nt = 0; nt < 16; ++nt) {
+          o[nt][0] *= alpha[0]; o[nt][1] *= alpha[0];
+          o[nt][2] *= alpha[1]; o[nt][3] *= alpha[1];
+        }
       }
-      // ---- P fragments (E4M3): logical k 4tig+i <-> key 4tig+i, 16+4tig+i <-> key 16+4tig+i
-      const uint32_t pa0 = pack_e4m3x4(sacc[0][0], sacc[0][1], sacc[1][0], sacc[1][1]);
-      const uint32_t pa1 = pack_e4m3x4(sacc[0][2], sacc[0][3], sacc[1][2], sacc[1][3]);
-      const uint32_t pa2 = pack_e4m3x4(sacc[2][0], sacc[2][1], sacc[3][0], sacc[3][1]);
-      const uint32_t pa3 = pack_e4m3x4(sacc[2][2], sacc[2][3], sacc[3][2], sacc[3][3]);
-      // ---- O += P V
+      // ---- P fragments: logical k 4tig+e <-> key tig+8e (S n-tile e, column
+      // 2tig), logical 16+4tig+e <-> key tig+4+8e (n-tile e, column 2tig+1).
+      // P = Ph + Pl, both E4M3, so the FP8 MMA sees P to ~8 significant bits
+      // (one E4M3 term alone moves the weights of a few-key softmax by ~3%).
+      uint32_t ph0, pl0, ph1, pl1, ph2, pl2, ph3, pl3;
+      split_e4m3x4(sacc[0][0], sacc[1][0], sacc[2][0], sacc[3][0], ph0, pl0);
+      split_e4m3x4(sacc[0][2], sacc[1][2], sacc[2][2], sacc[3][2], ph1, pl1);
+      split_e4m3x4(sacc[0][1], sacc[1][1], sacc[2][1], sacc[3][1], ph2, pl2);
+      split_e4m3x4(sacc[0][3], sacc[1][3], sacc[2][3], sacc[3][3], ph3, pl3);
+      // ---- O += Ph V + Pl V
 #pragma unroll
       for (int nt = 0; nt < 16; ++nt) {
         const int d = 8 * nt + gid;
         const uint2 bb = *reinterpret_cast<const uint2*>(vt + vt_index(d, tig));
-        mma_e4m3(o[nt], pa0, pa1, pa2, pa3, bb.x, bb.y);
+        mma_e4m3(o[nt], ph0, ph1, ph2, ph3, bb.x, bb.y);
+        mma_e4m3(o[nt], pl0, pl1, pl2, pl3, bb.x, bb.y);
       }
       __syncwarp();   // V^T tile reused by the next block
     }

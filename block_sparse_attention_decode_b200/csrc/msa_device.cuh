@@ -43,7 +43,6 @@ __device__ __forceinline__ void report(Flags* f, int code, int detail) {
 // lut[s] = {E4M3(m*e4m3(s)) for m = 0..3 in .x, m = 4..7 in .y}, m indexing
 // the E2M1 magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6} (OCP MX v1.0).
 __device__ __forceinline__ void build_nvfp4_lut(uint2* lut, int tid, int nthreads) {
-  const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
   for (int i = tid; i < 512; i += nthreads) {
     const int s = i >> 1, half = i & 1;
     __nv_fp8_e4m3 sc;
@@ -53,7 +52,10 @@ __device__ __forceinline__ void build_nvfp4_lut(uint2* lut, int tid, int nthread
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       // the product of a 2-bit and a 4-bit significand is exact in fp32
-      const float prod = mag[4 * half + k] * scale;
+      const int m = 4 * half + k;                       // E2M1 magnitude code
+      const float mag = (m < 2) ? 0.5f * (float)m
+                                : (1.0f + 0.5f * (float)(m & 1)) * (float)(1 << ((m >> 1) - 1));
+      const float prod = mag * scale;
       const uint32_t b = __nv_cvt_float_to_fp8(prod, __NV_SATFINITE, __NV_E4M3);
       word |= (b & 0xFFu) << (8 * k);
     }
@@ -107,6 +109,30 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   return pack_e4m3x2(a, b) | (pack_e4m3x2(c, d) << 16);
 }
 
+// Two fp32 values as a sum of two E4M3 terms: hi = E4M3(v), lo = E4M3(v - hi)
+// with the remainder formed in f16 (v and hi are exact in f16 to 2^-11).
+// hi + lo carries v to about 8 significant bits instead of E4M3's 4.
+__device__ __forceinline__ void split_e4m3x2(float lo_v, float hi_v, uint32_t& h, uint32_t& l) {
+  uint16_t hh, ll;
+  uint32_t p16, h16, r16;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(hh) : "f"(hi_v), "f"(lo_v));
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(p16) : "f"(hi_v), "f"(lo_v));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(h16) : "h"(hh));
+  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(r16) : "r"(p16), "r"(h16));
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;\n" : "=h"(ll) : "r"(r16));
+  h = hh;
+  l = ll;
+}
+
+__device__ __forceinline__ void split_e4m3x4(float a, float b, float c, float d, uint32_t& h,
+                                             uint32_t& l) {
+  uint32_t h0, l0, h1, l1;
+  split_e4m3x2(a, b, h0, l0);
+  split_e4m3x2(c, d, h1, l1);
+  h = h0 | (h1 << 16);
+  l = l0 | (l1 << 16);
+}
+
 // -------------------------------------------- mbarrier + bulk async copy --
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -142,19 +168,22 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// Bounded wait on an mbarrier phase.  Returns false after the iteration limit
-// (each try_wait itself suspends for a bounded, hardware-defined time).
-constexpr uint32_t kSpinLimit = 1u << 20;
+// Bounded wait on an mbarrier phase.  Each try_wait suspends the thread until
+// the phase completes or the suspend-time hint (about 0.5 ms) runs out, so a
+// waiting warp does not spin; after kSpinLimit attempts (a few seconds at
+// most) the wait gives up and returns false.
+constexpr uint32_t kSpinLimit = 1u << 13;
+constexpr uint32_t kSuspendHintNs = 500000;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
   for (uint32_t it = 0; it < kSpinLimit; ++it) {
     uint32_t ok;
     asm volatile(
-        "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n"
+        "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n"
         "selp.b32 %0, 1, 0, P;\n}\n"
         : "=r"(ok)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     if (ok) return true;
   }
@@ -176,6 +205,124 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 __device__ __forceinline__ float key_float(uint32_t k) {
   const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
   return __uint_as_float(u);
+}
+
+}  // namespace msa
+
+// ------------------------------------------------------------- tcgen05 ----
+// 5th-generation tensor core: MMAs issued by one thread, operands in shared
+// memory described by 64-bit descriptors, fp32 accumulators in tensor memory.
+namespace msa {
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// Warp-wide: allocate ncols (power of 2, >= 32) TMEM columns; address -> *dst.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand tile stored with the 128-byte
+// swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart, the 16-byte chunk
+// c of row r at chunk position c ^ (r % 8); tile base 1024-byte aligned.
+__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t smem_addr) {
+  return (uint64_t)((smem_addr & 0x3FFFFu) >> 4)   // start address
+         | ((uint64_t)1 << 16)                      // leading offset (unused with swizzle)
+         | ((uint64_t)(1024 >> 4) << 32)            // stride between 8-row atoms
+         | ((uint64_t)1 << 46)                      // descriptor version
+         | ((uint64_t)2 << 61);                     // 128-byte swizzle
+}
+
+// Instruction descriptor: kind::f8f6f4, A = B = E4M3, fp32 accumulate,
+// both operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, one K = 32 slice (E4M3).
+__device__ __forceinline__ void tc_mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on *bar once every tcgen05 operation issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+
+// Warp-wide: lane l reads TMEM lane (taddr.lane + l), 32 consecutive columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Max of a float over the 32 lanes of the warp (result in every lane).
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;\n" : "=f"(r) : "f"(v));
+  return r;
 }
 
 }  // namespace msa

@@ -1,38 +1,80 @@
-// msa_indexer.cu -- indexer scores + block max-pool ([post, "MSA primer"]:
-// one index query per GQA group scores every cached key against one shared
-// index-key head; the scores are max-pooled to one score per 128-token block).
+// msa_indexer.cu -- indexer scores + block max-pool on the 5th-generation
+// tensor core ([post, "MSA primer"]: one index query per GQA group scores
+// every cached key against one shared index-key head; the scores are
+// max-pooled to one score per 128-token block).
 // post = vLLM 為 MiniMax-M3.1-Flash 提供 Day-0 支援 (hot.atechcom.net).
 //
-// Work split.  The index-key pages of all sequences form one flat list
-// (sequence-major); each CTA of the grid's x dimension takes one contiguous
-// slice of it, so the load is even however ragged the lengths are.  The y
-// dimension tiles the index queries (T tokens x 4 groups) in chunks of 8*NT.
+// Per page (= one 128-token block) the scores are one dense FP8 contraction
+//   D[128 keys x NQ queries] = K_page[128 x 128] * Qi[NQ x 128]^T
+// with the keys as the M side (so the block max is a reduction over TMEM
+// lanes) and a chunk of NQ index queries (T tokens x 4 groups, padded to a
+// multiple of 8) as the N side.
 //
-// Per CTA: one producer warp streams whole pages (8 KB codes + 1 KB scales,
-// or 16 KB FP8 keys) into a ring of shared-memory stages with bulk async
-// copies completing on mbarriers; four consumer warps each own every fourth
-// page.  A consumer decodes the page straight into FP8 MMA fragments (keys
-// are the M side, 16 per fragment; queries the N side), runs
-// m16n8k32 e4m3 MMAs, masks keys after each query's position, and reduces
-// the 128 keys of the page to one block maximum in registers -- token scores
-// never reach global memory unless the caller asks for them.
+// Work split: the pages of all sequences form one flat list; CTA x takes one
+// contiguous slice of it (even load for ragged lengths); grid y tiles the
+// index queries in chunks of NQ.  Warp roles inside a CTA:
+//   warp 4 (producer): streams each page (8 KB codes + 1 KB scales, or 16 KB
+//     FP8 keys) into a ring of shared-memory stages with bulk async copies
+//     completing on mbarriers;
+//   warps 0-3 (workers): decode NVFP4 -> E4M3 (or copy FP8) into a 128-byte
+//     swizzled K-major tile (double buffered), then, one page behind, read
+//     the accumulator from TMEM (warp w owns TMEM lanes 32w..32w+31), mask
+//     keys after each query's position, reduce the 128 keys with
+//     redux.sync.max.f32 and combine the four warps' partial maxima;
+//   warp 5 (MMA): one elected thread issues 4 tcgen05.mma (K = 32 each) per
+//     page into a double-buffered TMEM accumulator and commits to mbarriers.
+// Every wait is a bounded mbarrier wait; on a timeout a thread records
+// MSA_ERR_TIMEOUT and leaves its loop, and TMEM is freed before exit.
 #include "msa_internal.h"
 
 namespace msa {
 
-template <bool FP8IDX>
-struct IdxStage {
-  static constexpr int kBytes = FP8IDX ? kBlock * kDim : kPageCodes + kPageScales;
-};
+constexpr int kIdxWorkers = 4;
+constexpr int kIdxProducerWarp = 4;
+constexpr int kIdxMmaWarp = 5;
+constexpr int kTileBytes = kBlock * kDim;   // 16 KB decoded page
 
-// Per-page metadata handed from the producer to the consumer of a stage.
 enum : int { kPageLoad = 0, kPageMasked = 1, kPageBad = 2 };
 
-size_t indexer_smem_bytes(bool fp8idx, int batch) {
-  const int stage = fp8idx ? IdxStage<true>::kBytes : IdxStage<false>::kBytes;
-  return (size_t)kIdxStages * stage + 256 * sizeof(uint2) + 2 * kIdxStages * sizeof(uint64_t) +
-         3 * kIdxStages * sizeof(int) + (size_t)(batch + 1) * sizeof(int) +
-         kIdxThreads * sizeof(int) + 64;
+struct IdxLayout {
+  int raw, tile, qbuf, lut, red, bars, meta, tinfo, cnt, tslot, prefix, scratch, total;
+};
+
+__host__ __device__ inline int raw_stage_bytes(bool fp8idx) {
+  return fp8idx ? kBlock * kDim : kPageCodes + kPageScales;
+}
+
+__host__ __device__ inline IdxLayout idx_layout(int nq, bool fp8idx, int batch) {
+  IdxLayout L;
+  int off = 0;
+  L.tile = off;    off += 2 * kTileBytes;                 // 1024-aligned tiles first
+  L.qbuf = off;    off += 2 * nq * 128;                   // nq % 8 == 0 -> 1024-aligned
+  L.raw = off;     off += kIdxRawStages * raw_stage_bytes(fp8idx);
+  L.lut = off;     off += 256 * 8;
+  L.red = off;     off += 2 * kIdxWorkers * nq * 4;
+  L.bars = off;    off += (2 * kIdxRawStages + 8) * 8;
+  L.meta = off;    off += 3 * kIdxRawStages * 4;
+  L.tinfo = off;   off += 4 * 4;
+  L.cnt = off;     off += 2 * 4;
+  L.tslot = off;   off += 16;
+  L.prefix = off;  off += (batch + 1) * 4;
+  L.scratch = off; off += kIdxThreads * 4;
+  L.total = off + 1024;                                   // alignment slack
+  return L;
+}
+
+int idx_nq(int T) {
+  const int nq = kG * T;
+  if (nq <= 8) return 8;
+  if (nq <= 16) return 16;
+  if (nq <= 32) return 32;
+  if (nq <= 64) return 64;
+  if (nq <= 128) return 128;
+  return 256;
+}
+
+size_t indexer_smem_bytes(bool fp8idx, int batch, int T) {
+  return (size_t)idx_layout(idx_nq(T), fp8idx, batch).total;
 }
 
 // Exclusive prefix over the number of blocks of each sequence, in shared
@@ -70,59 +112,91 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
   __syncthreads();
 }
 
-template <int NT, bool FP8IDX>
-__global__ void __launch_bounds__(kIdxThreads) indexer_kernel(IdxArgs a) {
-  constexpr int kStage = IdxStage<FP8IDX>::kBytes;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* stages = smem;
-  uint2* lut = reinterpret_cast<uint2*>(smem + kIdxStages * kStage);
-  uint64_t* full = reinterpret_cast<uint64_t*>(lut + 256);
-  uint64_t* empty = full + kIdxStages;
-  int* meta = reinterpret_cast<int*>(empty + kIdxStages);   // [stage][b, i, kind]
-  int* prefix = meta + 3 * kIdxStages;                       // [B + 1]
-  int* scratch = prefix + a.B + 1;                           // [kIdxThreads]
+__device__ __forceinline__ void sts128(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+
+template <int NQ, bool FP8IDX>
+__global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
+  constexpr int kRaw = FP8IDX ? kBlock * kDim : kPageCodes + kPageScales;
+  constexpr int kCols = (2 * NQ) < 32 ? 32 : 2 * NQ;        // TMEM columns (power of 2)
+  constexpr int kChunk = NQ < 32 ? NQ : 32;                 // columns per TMEM load
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
+  const IdxLayout Ly = idx_layout(NQ, FP8IDX, a.B);
+  uint8_t* tile = smem + Ly.tile;
+  uint8_t* qbuf = smem + Ly.qbuf;
+  uint8_t* raw = smem + Ly.raw;
+  uint2* lut = reinterpret_cast<uint2*>(smem + Ly.lut);
+  float* red = reinterpret_cast<float*>(smem + Ly.red);            // [2][4][NQ]
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + Ly.bars);
+  uint64_t* raw_empty = raw_full + kIdxRawStages;
+  uint64_t* tile_full = raw_empty + kIdxRawStages;                // workers -> MMA
+  uint64_t* tile_empty = tile_full + 2;                            // MMA -> workers
+  uint64_t* acc_full = tile_empty + 2;                             // MMA -> workers
+  uint64_t* acc_empty = acc_full + 2;                              // workers -> MMA
+  int* meta = reinterpret_cast<int*>(smem + Ly.meta);              // [stage][b, i, kind]
+  int* tinfo = reinterpret_cast<int*>(smem + Ly.tinfo);            // [2][skip, qsel]
+  int* cnt = reinterpret_cast<int*>(smem + Ly.cnt);                // [2]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
+  int* prefix = reinterpret_cast<int*>(smem + Ly.prefix);
+  int* scratch = reinterpret_cast<int*>(smem + Ly.scratch);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gid = lane >> 2, tig = lane & 3;
 
-  build_nvfp4_lut(lut, tid, blockDim.x);
+  if (!FP8IDX) build_nvfp4_lut(lut, tid, blockDim.x);
   if (tid == 0) {
-    for (int s = 0; s < kIdxStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < kIdxRawStages; ++s) {
+      mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], kIdxWorkers);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&tile_full[x], kIdxWorkers);
+      mbar_init(&tile_empty[x], 1);
+      mbar_init(&acc_full[x], 1);
+      mbar_init(&acc_empty[x], kIdxWorkers);
+      cnt[x] = 0;
+    }
     mbar_fence_init();
   }
-  page_prefix(a, prefix, scratch);   // contains __syncthreads
+  if (warp == kIdxMmaWarp) {
+    tmem_alloc(tslot, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  page_prefix(a, prefix, scratch);   // ends with __syncthreads
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
 
   const int total = prefix[a.B];
   const int lo = (int)((long long)total * blockIdx.x / gridDim.x);
   const int hi = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
   const int n = hi - lo;
-  const int qbase = blockIdx.y * 8 * NT;          // first index query of this chunk
+  const int qbase = blockIdx.y * NQ;           // first index query of this chunk
   const int t_first = qbase >> 2;
-  const int t_last = min(a.T - 1, (qbase + 8 * NT - 1) >> 2);
+  const int t_last = min(a.T - 1, (qbase + NQ - 1) >> 2);
+  const long long ctx = (long long)a.max_pages * kBlock;
 
-  if (warp == kIdxConsumers) {
+  if (warp == kIdxProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n > 0) {
-      int b = 0;
-      {  // first sequence whose pages reach index lo: prefix[b] <= lo < prefix[b+1]
+      int b;
+      {  // prefix[b] <= lo < prefix[b+1]
         int l = 0, r = a.B;
         while (r - l > 1) { const int m = (l + r) >> 1; if (prefix[m] <= lo) l = m; else r = m; }
         b = l;
       }
       int i = lo - prefix[b];
       for (int k = 0; k < n; ++k) {
-        const int s = k % kIdxStages;
-        if (k >= kIdxStages && !mbar_wait(&empty[s], ((k / kIdxStages) - 1) & 1)) {
-          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, k);
+        const int s = k % kIdxRawStages;
+        if (k >= kIdxRawStages && !mbar_wait(&raw_empty[s], ((k / kIdxRawStages) - 1) & 1)) {
+          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1);
           break;
         }
         while (i >= prefix[b + 1] - prefix[b]) { i -= prefix[b + 1] - prefix[b]; ++b; }
         const int L = a.seq_lens[b];
-        const int max_pos = L - a.T + t_last;
         int kind = kPageLoad;
-        long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + i]
-                                   : (long long)b * a.max_pages + i;
-        if (i * kBlock > max_pos) {
+        const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + i]
+                                         : (long long)b * a.max_pages + i;
+        if (i * kBlock > L - a.T + t_last) {
           kind = kPageMasked;
         } else if (p < 0 || p >= a.num_pages) {
           report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)p);
@@ -131,189 +205,236 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(IdxArgs a) {
         meta[3 * s + 0] = b;
         meta[3 * s + 1] = i;
         meta[3 * s + 2] = kind;
-        uint8_t* dst = stages + s * kStage;
+        uint8_t* dst = raw + s * kRaw;
         if (kind == kPageLoad) {
-          mbar_expect_tx(&full[s], kStage);
+          mbar_expect_tx(&raw_full[s], kRaw);
           if (FP8IDX) {
-            bulk_g2s(dst, a.idx_data + p * (kBlock * kDim), kBlock * kDim, &full[s]);
+            bulk_g2s(dst, a.idx_data + p * (kBlock * kDim), kBlock * kDim, &raw_full[s]);
           } else {
-            bulk_g2s(dst, a.idx_data + p * kPageCodes, kPageCodes, &full[s]);
-            bulk_g2s(dst + kPageCodes, a.idx_scale + p * kPageScales, kPageScales, &full[s]);
+            bulk_g2s(dst, a.idx_data + p * kPageCodes, kPageCodes, &raw_full[s]);
+            bulk_g2s(dst + kPageCodes, a.idx_scale + p * kPageScales, kPageScales, &raw_full[s]);
           }
         } else {
-          mbar_arrive(&full[s]);
+          mbar_arrive(&raw_full[s]);
         }
         ++i;
       }
     }
+  } else if (warp == kIdxMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(128, NQ);
+      for (int k = 0; k < n; ++k) {
+        const int x = k & 1;
+        if (!mbar_wait(&tile_full[x], (k >> 1) & 1)) { report(a.flags, 5, 2); break; }
+        if (k >= 2 && !mbar_wait(&acc_empty[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 3); break; }
+        tc_fence_after();
+        if (!tinfo[2 * x]) {
+          const uint32_t a0 = smem_u32(tile + x * kTileBytes);
+          const uint32_t b0 = smem_u32(qbuf + tinfo[2 * x + 1] * NQ * 128);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_e4m3(tmem + x * NQ, desc_kmajor_sw128(a0 + 32 * kk),
+                        desc_kmajor_sw128(b0 + 32 * kk), idesc, kk > 0);
+        }
+        tc_commit(&tile_empty[x]);
+        tc_commit(&acc_full[x]);
+      }
+    }
   } else {
-    // ------------------------------------------------------------ consumers
-    uint32_t qf[NT][8];
-    int cur_b = -1, L = 0;
-    for (int k = warp; k < n; k += kIdxConsumers) {
-      const int s = k % kIdxStages;
-      if (!mbar_wait(&full[s], (k / kIdxStages) & 1)) {
-        report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, k);
-        break;
-      }
-      const int b = meta[3 * s + 0], i = meta[3 * s + 1], kind = meta[3 * s + 2];
-      if (b != cur_b) {
-        cur_b = b;
-        L = a.seq_lens[b];
-        // B fragments: column gid of n-tile j = index query qbase + 8j + gid;
-        // this thread holds its elements 32*tig .. 32*tig+31.
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          const int qg = qbase + 8 * j + gid;
-          const int t = qg >> 2;
-          if (t < a.T) {
-            const uint8_t* src = a.qi + (((long long)b * a.T + t) * kG + (qg & 3)) * kDim + 32 * tig;
-            const uint4 x0 = *reinterpret_cast<const uint4*>(src);
-            const uint4 x1 = *reinterpret_cast<const uint4*>(src + 16);
-            qf[j][0] = x0.x; qf[j][1] = x0.y; qf[j][2] = x0.z; qf[j][3] = x0.w;
-            qf[j][4] = x1.x; qf[j][5] = x1.y; qf[j][6] = x1.z; qf[j][7] = x1.w;
-          } else {
-#pragma unroll
-            for (int m = 0; m < 8; ++m) qf[j][m] = 0u;
-          }
-        }
-      }
-      const int pos0 = L - a.T;       // position of token 0
-      const long long ctx = (long long)a.max_pages * kBlock;
-      if (kind == kPageLoad) {
-        const uint8_t* sd = stages + s * kStage;
-        const bool need_mask = (i * kBlock + kBlock - 1) > (pos0 + t_first);
-        float bm[NT][2];
-#pragma unroll
-        for (int j = 0; j < NT; ++j) { bm[j][0] = -INFINITY; bm[j][1] = -INFINITY; }
+    // ------------------------------------------------------------ workers
+    // Epilogue of page kk (its accumulator is TMEM buffer kk & 1).
+    auto epilogue = [&](int kk, int pb, int pi, int pkind, int pL) -> bool {
+      const int xe = kk & 1;
+      if (!mbar_wait(&acc_full[xe], (kk >> 1) & 1)) { report(a.flags, 5, 6); return false; }
+      tc_fence_after();
+      if (pkind == kPageLoad) {
+        const int key = pi * kBlock + 32 * warp + lane;
+        const int pos0 = pL - a.T;
+        const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + t_first;
 #pragma unroll 1
-        for (int mt = 0; mt < kBlock / 16; ++mt) {
-          const int r0 = 16 * mt + gid, r1 = r0 + 8;
-          uint32_t k0[8], k1[8];
-          if (FP8IDX) {
-            const uint4 x0 = lds128(sd + r0 * kDim + 32 * tig), x1 = lds128(sd + r0 * kDim + 32 * tig + 16);
-            const uint4 y0 = lds128(sd + r1 * kDim + 32 * tig), y1 = lds128(sd + r1 * kDim + 32 * tig + 16);
-            k0[0] = x0.x; k0[1] = x0.y; k0[2] = x0.z; k0[3] = x0.w;
-            k0[4] = x1.x; k0[5] = x1.y; k0[6] = x1.z; k0[7] = x1.w;
-            k1[0] = y0.x; k1[1] = y0.y; k1[2] = y0.z; k1[3] = y0.w;
-            k1[4] = y1.x; k1[5] = y1.y; k1[6] = y1.z; k1[7] = y1.w;
+        for (int c0 = 0; c0 < NQ; c0 += kChunk) {
+          float v[32];
+          const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + xe * NQ + c0;
+          if constexpr (kChunk == 32) {
+            tmem_ld32(taddr, v);
+          } else if constexpr (kChunk == 16) {
+            float v16[16];
+            tmem_ld16(taddr, v16);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = v16[j];
           } else {
-            const uint8_t* ss = sd + kPageCodes;
-            dq32(lut, lds128(sd + r0 * kRowCodes + 16 * tig), lds16(ss + r0 * kRowScales + 2 * tig), k0);
-            dq32(lut, lds128(sd + r1 * kRowCodes + 16 * tig), lds16(ss + r1 * kRowScales + 2 * tig), k1);
+            static_assert(kChunk == 8, "column chunk");
+            float v8[8];
+            tmem_ld8(taddr, v8);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = v8[j];
           }
-          float acc[NT][4];
+          tmem_wait_ld();
+          if (need_mask) {   // keys after a query's position do not count
 #pragma unroll
-          for (int j = 0; j < NT; ++j) { acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f; }
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-            for (int j = 0; j < NT; ++j)
-              mma_e4m3(acc[j], k0[2 * ks], k1[2 * ks], k0[2 * ks + 1], k1[2 * ks + 1],
-                       qf[j][2 * ks], qf[j][2 * ks + 1]);
+            for (int j = 0; j < kChunk; ++j)
+              if (key > pos0 + ((qbase + c0 + j) >> 2)) v[j] = -INFINITY;
           }
+          if (a.token_scores != nullptr) {
 #pragma unroll
-          for (int j = 0; j < NT; ++j) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int row = (e < 2) ? r0 : r1;
-              const int qg = qbase + 8 * j + 2 * tig + (e & 1);
-              const int t = qg >> 2;
-              const int key = i * kBlock + row;
-              float v = acc[j][e];
-              if (need_mask && (t >= a.T || key > pos0 + t)) v = -INFINITY;
-              if (a.token_scores && t < a.T)
-                a.token_scores[(((long long)cur_b * a.T + t) * kG + (qg & 3)) * ctx + key] =
-                    v * a.score_scale;
-              bm[j][e & 1] = fmaxf(bm[j][e & 1], v);
-            }
-          }
-        }
-        // max over the 8 lanes that share tig (rows gid = 0..7)
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float v = bm[j][c];
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-            bm[j][c] = v;
-          }
-        }
-        if (gid == 0) {
-#pragma unroll
-          for (int j = 0; j < NT; ++j) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const int qg = qbase + 8 * j + 2 * tig + c;
-              const int t = qg >> 2;
+            for (int j = 0; j < kChunk; ++j) {
+              const int qg = qbase + c0 + j, t = qg >> 2;
               if (t < a.T)
-                a.block_scores[(((long long)cur_b * a.T + t) * kG + (qg & 3)) * a.max_pages + i] =
-                    bm[j][c] * a.score_scale;
+                a.token_scores[(((long long)pb * a.T + t) * kG + (qg & 3)) * ctx + key] =
+                    v[j] * a.score_scale;
             }
           }
-        }
-      } else if (kind == kPageMasked) {
-        // no key of this page is visible to any query of the chunk
-        for (int c = lane; c < 8 * NT; c += 32) {
-          const int qg = qbase + c, t = qg >> 2;
-          if (t < a.T)
-            a.block_scores[(((long long)cur_b * a.T + t) * kG + (qg & 3)) * a.max_pages + i] =
-                -INFINITY;
-        }
-        if (a.token_scores) {
-          for (int c = 0; c < 8 * NT; ++c) {
-            const int qg = qbase + c, t = qg >> 2;
-            if (t >= a.T) break;
-            float* row = a.token_scores + (((long long)cur_b * a.T + t) * kG + (qg & 3)) * ctx;
-            for (int r = lane; r < kBlock; r += 32) row[i * kBlock + r] = -INFINITY;
+          float part = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) {
+            const float m = warp_max(v[j]);
+            part = (lane == j) ? m : part;
           }
+          if (lane < kChunk) red[(xe * kIdxWorkers + warp) * NQ + c0 + lane] = part;
         }
       }
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      int last = 0;
+      if (lane == 0) {
+        mbar_arrive(&acc_empty[xe]);
+        __threadfence_block();
+        last = (atomicAdd(&cnt[xe], 1) == kIdxWorkers - 1);
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {   // the last warp of this page combines the four partial maxima
+        __threadfence_block();
+        if (pkind != kPageBad) {
+          for (int col = lane; col < NQ; col += 32) {
+            const int qg = qbase + col, t = qg >> 2;
+            if (t >= a.T) continue;
+            float m = -INFINITY;
+            if (pkind == kPageLoad) {
+#pragma unroll
+              for (int w = 0; w < kIdxWorkers; ++w)
+                m = fmaxf(m, red[(xe * kIdxWorkers + w) * NQ + col]);
+            }
+            a.block_scores[(((long long)pb * a.T + t) * kG + (qg & 3)) * a.max_pages + pi] =
+                m * a.score_scale;
+            if (pkind == kPageMasked && a.token_scores != nullptr) {
+              float* row = a.token_scores + (((long long)pb * a.T + t) * kG + (qg & 3)) * ctx;
+              for (int r = 0; r < kBlock; ++r) row[pi * kBlock + r] = -INFINITY;
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) cnt[xe] = 0;
+      }
+      return true;
+    };
+
+    int cur_b = -1, qsel = 1, L = 0;
+    int pb = 0, pi = 0, pkind = kPageBad, pL = 0;   // the page one behind
+    for (int k = 0; k <= n; ++k) {
+      int nb = 0, ni = 0, nkind = kPageBad;
+      if (k < n) {
+        // ---- decode page k into tile[k & 1]
+        const int x = k & 1, s = k % kIdxRawStages;
+        if (k >= 2 && !mbar_wait(&tile_empty[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 4); break; }
+        if (!mbar_wait(&raw_full[s], (k / kIdxRawStages) & 1)) { report(a.flags, 5, 5); break; }
+        nb = meta[3 * s + 0];
+        ni = meta[3 * s + 1];
+        nkind = meta[3 * s + 2];
+        if (nb != cur_b) {
+          cur_b = nb;
+          L = a.seq_lens[nb];
+          qsel ^= 1;
+          // B operand: the query rows of this chunk for sequence nb, swizzled.
+          // (Its previous user, the MMA of page k-2 or earlier, has completed.)
+          uint8_t* qb = qbuf + qsel * NQ * 128;
+          constexpr int kRowsPerWarp = NQ / kIdxWorkers;
+          for (int idx = lane; idx < kRowsPerWarp * 8; idx += 32) {
+            const int nrow = warp * kRowsPerWarp + idx / 8, c = idx % 8;
+            const int qg = qbase + nrow, t = qg >> 2;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (t < a.T)
+              v = *reinterpret_cast<const uint4*>(
+                  a.qi + (((long long)nb * a.T + t) * kG + (qg & 3)) * kDim + 16 * c);
+            sts128(qb + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
+          }
+        }
+        if (nkind == kPageLoad) {
+          const uint8_t* rs = raw + s * kRaw;
+          uint8_t* tl = tile + x * kTileBytes;
+          if constexpr (FP8IDX) {
+#pragma unroll 4
+            for (int p = 0; p < 8; ++p) {
+              const int r = 32 * warp + 4 * p + (lane >> 3), c = lane & 7;
+              sts128(tl + r * 128 + ((c ^ (r & 7)) << 4), lds128(rs + r * kDim + 16 * c));
+            }
+          } else {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const int r = 32 * warp + 8 * p + (lane >> 2), q = lane & 3;
+              uint32_t o[8];
+              dq32(lut, lds128(rs + r * kRowCodes + 16 * q),
+                   lds16(rs + kPageCodes + r * kRowScales + 2 * q), o);
+              sts128(tl + r * 128 + (((2 * q) ^ (r & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+              sts128(tl + r * 128 + (((2 * q + 1) ^ (r & 7)) << 4),
+                     make_uint4(o[4], o[5], o[6], o[7]));
+            }
+          }
+        }
+        fence_async_smem();   // make the tile writes visible to the tensor core
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&raw_empty[s]);
+          if (warp == 0) { tinfo[2 * x] = (nkind != kPageLoad); tinfo[2 * x + 1] = qsel; }
+          mbar_arrive(&tile_full[x]);
+        }
+      }
+      // ---- epilogue of page k-1 (its MMA ran while page k was decoded)
+      if (k >= 1 && !epilogue(k - 1, pb, pi, pkind, pL)) break;
+      pb = nb; pi = ni; pkind = nkind; pL = L;
     }
   }
+
+  // ---- teardown: every role leaves its loop (normally or on a timeout)
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kIdxMmaWarp) tmem_dealloc(tmem, kCols);
 }
 
-template <int NT, bool FP8IDX>
-static cudaError_t launch_nt(const IdxArgs& a, int gx, int gy, size_t smem, cudaStream_t st) {
-  auto kern = indexer_kernel<NT, FP8IDX>;
+template <int NQ, bool FP8IDX>
+static cudaError_t launch_nq(const IdxArgs& a, int num_sms, cudaStream_t st) {
+  auto kern = indexer_kernel<NQ, FP8IDX>;
+  const size_t smem = (size_t)idx_layout(NQ, FP8IDX, a.B).total;
   static size_t configured = 0;
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
+  const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), kIdxThreads, smem,
+                                 (2 * NQ) < 32 ? 32 : 2 * NQ);
+  const int gy = (kG * a.T + NQ - 1) / NQ;
+  const long long want = ((long long)num_sms * per_sm + gy - 1) / gy;
+  const long long cap = (long long)a.B * a.max_pages;
+  const int gx = (int)(want < 1 ? 1 : (want > cap ? cap : want));
   kern<<<dim3(gx, gy), kIdxThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
-int indexer_ntiles(int T) {
-  const int nq = kG * T;
-  return nq <= 8 ? 1 : (nq <= 16 ? 2 : 4);
-}
-
 cudaError_t launch_indexer(const IdxArgs& a, bool fp8idx, int num_sms, cudaStream_t st) {
-  const int NT = indexer_ntiles(a.T);
-  const int gy = (kG * a.T + 8 * NT - 1) / (8 * NT);
-  const size_t smem = indexer_smem_bytes(fp8idx, a.B);
-  // CTAs resident per SM for this shared-memory footprint (at most 3)
-  int per_sm = (int)((220 * 1024) / smem);
-  per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);
-  long long want = ((long long)num_sms * per_sm + gy - 1) / gy;
-  const long long cap = (long long)a.B * a.max_pages;
-  int gx = (int)(want < 1 ? 1 : (want > cap ? cap : want));
-  if (gx > 65535 * 32) gx = 65535 * 32;
-  if (fp8idx) {
-    if (NT == 1) return launch_nt<1, true>(a, gx, gy, smem, st);
-    if (NT == 2) return launch_nt<2, true>(a, gx, gy, smem, st);
-    return launch_nt<4, true>(a, gx, gy, smem, st);
-  }
-  if (NT == 1) return launch_nt<1, false>(a, gx, gy, smem, st);
-  if (NT == 2) return launch_nt<2, false>(a, gx, gy, smem, st);
-  return launch_nt<4, false>(a, gx, gy, smem, st);
+  const int nq = idx_nq(a.T);
+#define MSA_IDX_CASE(NQV)                                                     \
+  if (nq == NQV)                                                              \
+    return fp8idx ? launch_nq<NQV, true>(a, num_sms, st) : launch_nq<NQV, false>(a, num_sms, st);
+  MSA_IDX_CASE(8)
+  MSA_IDX_CASE(16)
+  MSA_IDX_CASE(32)
+  MSA_IDX_CASE(64)
+  MSA_IDX_CASE(128)
+  MSA_IDX_CASE(256)
+#undef MSA_IDX_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace msa

@@ -10,9 +10,8 @@
 
 namespace msa {
 
-constexpr int kIdxConsumers = 4;
-constexpr int kIdxThreads = (kIdxConsumers + 1) * 32;
-constexpr int kIdxStages = 8;
+constexpr int kIdxThreads = 6 * 32;     // 4 workers, 1 producer, 1 MMA warp
+constexpr int kIdxRawStages = 3;         // raw index-key pages in flight per CTA
 
 struct IdxArgs {
   const uint8_t* idx_data;     // NVFP4 codes [P][128][64] or FP8 keys [P][128][128]
@@ -27,9 +26,14 @@ struct IdxArgs {
   int B, T, max_pages, num_pages;
 };
 
-size_t indexer_smem_bytes(bool fp8idx, int batch);
-int indexer_ntiles(int T);
+size_t indexer_smem_bytes(bool fp8idx, int batch, int T);
+int idx_nq(int T);
 cudaError_t launch_indexer(const IdxArgs& a, bool fp8idx, int num_sms, cudaStream_t st);
+
+// CTAs of `kernel` resident per SM for `threads` threads and `smem` dynamic
+// shared memory (registers, shared memory, and `tmem_cols` of the 512 TMEM
+// columns each CTA allocates; 0 = none).
+int ctas_per_sm(const void* kernel, int threads, size_t smem, int tmem_cols);
 
 // Top-k over block scores of every (b, t, g) row.
 cudaError_t launch_topk(const float* block_scores, const int32_t* seq_lens, int B, int T,
