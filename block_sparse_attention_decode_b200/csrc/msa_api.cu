@@ -92,6 +92,10 @@ msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi,
                        float* token_scores, float* block_scores, void* ws, const Layout& L,
                        cudaStream_t st) {
   IdxArgs a{};
+  const bool fp8 = c->idx_dtype == MSA_IDX_FP8;
+  if (!encode_row_tmap(&a.tmap_idx, c->idx_data, (uint64_t)c->num_pages * MSA_BLOCK_TOKENS,
+                       fp8 ? MSA_HEAD_DIM : MSA_HEAD_DIM / 2))
+    return MSA_ERR_CUDA;
   a.idx_data = c->idx_data;
   a.idx_scale = c->idx_scale;
   a.page_table = s->page_table;
@@ -142,6 +146,34 @@ msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, flo
 }  // namespace
 
 namespace msa {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes) {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr) {
+      cudaGetLastError();
+      return false;
+    }
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  if (row_bytes != 64 && row_bytes != 128) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {row_bytes, (cuuint32_t)kBlock};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUtensorMapSwizzle sw = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 int ctas_per_sm(const void* kernel, int threads, size_t smem, int tmem_cols) {
   int dev = 0, smem_sm = 0, regs_sm = 0, max_threads = 0;

@@ -32,8 +32,8 @@ constexpr int kAttStageBytes = 2 * (kPageCodes + kPageScales);   // K + V of one
 constexpr int kVtWords = kDim * 8 + 32;                           // per warp: [128 dims][8 words] + pad
 
 size_t attn_smem_bytes() {
-  return (size_t)kAttStages * kAttStageBytes + kAttConsumers * kVtWords * 4 + 256 * sizeof(uint2) +
-         2 * kAttStages * sizeof(uint64_t) + 4 * kTopk * sizeof(int) + 64;
+  return (size_t)kAttStages * kAttStageBytes + kAttConsumers * kVtWords * 4 + 4 * 32 * 16 +
+         256 * sizeof(uint2) + 2 * kAttStages * sizeof(uint64_t) + 4 * kTopk * sizeof(int) + 64;
 }
 
 int attn_splits(long long units, int num_sms) {
@@ -70,11 +70,12 @@ __device__ __forceinline__ int vt_index(int d, int q) {
   return d * 8 + 8 * (d >> 5) + 2 * (q & 3) + (q >> 2);
 }
 
-__global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(kAttThreads, 3) attn_kernel(AttnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
   uint32_t* vt_all = reinterpret_cast<uint32_t*>(smem + kAttStages * kAttStageBytes);
-  uint2* lut = reinterpret_cast<uint2*>(vt_all + kAttConsumers * kVtWords);
+  uint32_t* qfrag = vt_all + kAttConsumers * kVtWords;                  // [4][32][4]
+  uint2* lut = reinterpret_cast<uint2*>(qfrag + 4 * 32 * 4);
   uint64_t* full = reinterpret_cast<uint64_t*>(lut + 256);
   uint64_t* empty = full + kAttStages;
   int* list = reinterpret_cast<int*>(empty + kAttStages);   // [16] block ids
@@ -146,20 +147,25 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(AttnArgs a) {
     }
   } else {
     // ------------------------------------------------------------ consumers
-    // Q A-fragments: word m of a row = dims 32tig+4m..+3; k-step ks uses
-    // words 2ks (a0/a1) and 2ks+1 (a2/a3).
-    uint32_t qa[8][2];   // [word][row]
-    {
+    // Q A-fragments live in shared memory (qfrag[k-step][lane] = a0..a3), so
+    // they cost no registers across the block loop: row gid/gid+8 = heads
+    // 16g+gid / 16g+gid+8, k-step st covers dims 32tig+8st..+7.
+    if (warp == 0) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int h = g * kHpg + gid + 8 * r;
         const uint8_t* src = a.q + (((long long)b * a.T + t) * kHq + h) * kDim + 32 * tig;
         const uint4 x0 = *reinterpret_cast<const uint4*>(src);
         const uint4 x1 = *reinterpret_cast<const uint4*>(src + 16);
-        qa[0][r] = x0.x; qa[1][r] = x0.y; qa[2][r] = x0.z; qa[3][r] = x0.w;
-        qa[4][r] = x1.x; qa[5][r] = x1.y; qa[6][r] = x1.z; qa[7][r] = x1.w;
+        const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+          qfrag[(st * 32 + lane) * 4 + r] = w[2 * st];          // a0 / a1
+          qfrag[(st * 32 + lane) * 4 + 2 + r] = w[2 * st + 1];  // a2 / a3
+        }
       }
     }
+    asm volatile("bar.sync 1, %0;\n" ::"n"(kAttConsumers * 32) : "memory");
     uint32_t* vt = vt_all + warp * kVtWords;
     const float sc = a.logit_scale_log2;
     for (int k = 0; k < nlist; ++k) {
@@ -183,29 +189,37 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(AttnArgs a) {
         uint32_t kw[8];
         dq32(lut, lds128(kc + kk * kRowCodes + 16 * tig), lds16(ks_ + kk * kRowScales + 2 * tig), kw);
 #pragma unroll
-        for (int st = 0; st < 4; ++st)
-          mma_e4m3(sacc[j], qa[2 * st][0], qa[2 * st][1], qa[2 * st + 1][0], qa[2 * st + 1][1],
-                   kw[2 * st], kw[2 * st + 1]);
+        for (int st = 0; st < 4; ++st) {
+          const uint4 qa = *reinterpret_cast<const uint4*>(&qfrag[(st * 32 + lane) * 4]);
+          mma_e4m3(sacc[j], qa.x, qa.y, qa.z, qa.w, kw[2 * st], kw[2 * st + 1]);
+        }
       }
 
-      // ---- V^T tile: lane (kq, dc) decodes keys kq + 8r (r = 0..3), dims 32dc..32dc+31
+      // ---- V^T tile: lane (kq, dc) decodes keys kq + 8r (r = 0..3), dims
+      // 32dc..32dc+31, in two halves of 16 dims (one scale byte each)
       {
         const int kq = lane >> 2, dc = lane & 3;
-        uint32_t vw[4][8];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int kk = 32 * warp + kq + 8 * r;
-          dq32(lut, lds128(vc + kk * kRowCodes + 16 * dc), lds16(vs + kk * kRowScales + 2 * dc), vw[r]);
-        }
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t vw[4][4];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          uint32_t y0, y1, y2, y3;
-          transpose4x4(vw[0][m], vw[1][m], vw[2][m], vw[3][m], y0, y1, y2, y3);
-          const int d = 32 * dc + 4 * m;
-          vt[vt_index(d + 0, kq)] = y0;
-          vt[vt_index(d + 1, kq)] = y1;
-          vt[vt_index(d + 2, kq)] = y2;
-          vt[vt_index(d + 3, kq)] = y3;
+          for (int r = 0; r < 4; ++r) {
+            const int kk = 32 * warp + kq + 8 * r;
+            const uint2 c = *reinterpret_cast<const uint2*>(vc + kk * kRowCodes + 16 * dc + 8 * hf);
+            const uint2 row = lut[vs[kk * kRowScales + 2 * dc + hf]];
+            dq8(c.x, row, vw[r][0], vw[r][1]);
+            dq8(c.y, row, vw[r][2], vw[r][3]);
+          }
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            uint32_t y0, y1, y2, y3;
+            transpose4x4(vw[0][m], vw[1][m], vw[2][m], vw[3][m], y0, y1, y2, y3);
+            const int d = 32 * dc + 16 * hf + 4 * m;
+            vt[vt_index(d + 0, kq)] = y0;
+            vt[vt_index(d + 1, kq)] = y1;
+            vt[vt_index(d + 2, kq)] = y2;
+            vt[vt_index(d + 3, kq)] = y3;
+          }
         }
       }
       __syncwarp();

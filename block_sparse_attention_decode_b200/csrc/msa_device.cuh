@@ -326,3 +326,63 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 }  // namespace msa
+
+namespace msa {
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, one K = 32 slice (E4M3).  A: 128 TMEM
+// lanes = rows, 8 consecutive 32-bit columns = 32 K-bytes of each row.
+__device__ __forceinline__ void tc_mma_e4m3_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Warp-wide: lane l writes 8 consecutive 32-bit columns of TMEM lane (taddr.lane + l).
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+// Tiled TMA load of a 2-D box at element coordinates (x, y) into shared memory.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// NVFP4 -> E4M3 split by sign for 8 codes (element n in nibble n):
+// pos = E4M3(|value|) of the positive elements (0 elsewhere), neg likewise for
+// the negative ones, so value = pos - neg.  `r` is the table row of |scale|
+// (all bytes < 0x80); a selector nibble with its top bit set makes prmt
+// return 0x00 (the sign of a non-negative byte), which drops the elements of
+// the other sign.  flip = 0x88888888 when the block scale is negative.
+// PTX prmt in its default mode (the top bit of each selector nibble
+// replicates the sign of the selected byte, unlike __byte_perm).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ void dq8_split(uint32_t w, uint2 r, uint32_t flip, uint32_t& p0,
+                                          uint32_t& p1, uint32_t& n0, uint32_t& n1) {
+  const uint32_t wp = w ^ flip;
+  const uint32_t wn = wp ^ 0x88888888u;
+  p0 = prmt(r.x, r.y, wp);
+  p1 = prmt(r.x, r.y, wp >> 16);
+  n0 = prmt(r.x, r.y, wn);
+  n1 = prmt(r.x, r.y, wn >> 16);
+}
+
+}  // namespace msa

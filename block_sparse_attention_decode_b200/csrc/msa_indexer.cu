@@ -6,23 +6,27 @@
 //
 // Per page (= one 128-token block) the scores are one dense FP8 contraction
 //   D[128 keys x NQ queries] = K_page[128 x 128] * Qi[NQ x 128]^T
-// with the keys as the M side (so the block max is a reduction over TMEM
+// with the keys as the M side (the block max is a reduction over TMEM
 // lanes) and a chunk of NQ index queries (T tokens x 4 groups, padded to a
 // multiple of 8) as the N side.
 //
 // Work split: the pages of all sequences form one flat list; CTA x takes one
 // contiguous slice of it (even load for ragged lengths); grid y tiles the
 // index queries in chunks of NQ.  Warp roles inside a CTA:
-//   warp 4 (producer): streams each page (8 KB codes + 1 KB scales, or 16 KB
-//     FP8 keys) into a ring of shared-memory stages with bulk async copies
-//     completing on mbarriers;
-//   warps 0-3 (workers): decode NVFP4 -> E4M3 (or copy FP8) into a 128-byte
-//     swizzled K-major tile (double buffered), then, one page behind, read
-//     the accumulator from TMEM (warp w owns TMEM lanes 32w..32w+31), mask
-//     keys after each query's position, reduce the 128 keys with
-//     redux.sync.max.f32 and combine the four warps' partial maxima;
-//   warp 5 (MMA): one elected thread issues 4 tcgen05.mma (K = 32 each) per
-//     page into a double-buffered TMEM accumulator and commits to mbarriers.
+//   warp 4 (producer): per page one tiled TMA load of the codes (64-byte
+//     swizzle, so that row-per-thread reads are bank-conflict free) and one
+//     bulk copy of the scales into a ring of shared-memory stages;
+//   warps 0-3 (workers): thread = key row (= TMEM lane).  NVFP4 rows are
+//     decoded by sign: K+ holds E4M3(|v|) of the positive elements, K- of the
+//     negative ones (one prmt per 4 codes each, see dq8_split), and both go
+//     straight to tensor memory with tcgen05.st -- the A operand never
+//     touches shared memory.  One page behind, the workers read the
+//     accumulator from TMEM, mask keys after each query's position and
+//     reduce the 128 keys with redux.sync.max.f32 (combining the four warps'
+//     partial maxima in shared memory);
+//   warp 5 (MMA): one thread issues per page 4 tcgen05.mma with A = K+ and 4
+//     with A = K- and the negate-A bit (K = 32 each, A from TMEM, B = the
+//     queries in shared memory) into a double-buffered TMEM accumulator.
 // Every wait is a bounded mbarrier wait; on a timeout a thread records
 // MSA_ERR_TIMEOUT and leaves its loop, and TMEM is freed before exit.
 #include "msa_internal.h"
@@ -32,27 +36,28 @@ namespace msa {
 constexpr int kIdxWorkers = 4;
 constexpr int kIdxProducerWarp = 4;
 constexpr int kIdxMmaWarp = 5;
-constexpr int kTileBytes = kBlock * kDim;   // 16 KB decoded page
+constexpr int kACols = 64;                  // TMEM columns of the A operand (K+ | K-)
 
 enum : int { kPageLoad = 0, kPageMasked = 1, kPageBad = 2 };
 
 struct IdxLayout {
-  int raw, tile, qbuf, lut, red, bars, meta, tinfo, cnt, tslot, prefix, scratch, total;
+  int qbuf, raw, raw_stride, lut, red, bars, meta, tinfo, cnt, tslot, prefix, scratch, total;
 };
 
-__host__ __device__ inline int raw_stage_bytes(bool fp8idx) {
-  return fp8idx ? kBlock * kDim : kPageCodes + kPageScales;
+// Bytes of one raw page in shared memory (codes [+ scales]), 1024-aligned.
+__host__ __device__ inline int raw_stage_stride(bool fp8idx) {
+  return fp8idx ? kBlock * kDim : ((kPageCodes + kPageScales + 1023) / 1024) * 1024;
 }
 
 __host__ __device__ inline IdxLayout idx_layout(int nq, bool fp8idx, int batch) {
   IdxLayout L;
   int off = 0;
-  L.tile = off;    off += 2 * kTileBytes;                 // 1024-aligned tiles first
   L.qbuf = off;    off += 2 * nq * 128;                   // nq % 8 == 0 -> 1024-aligned
-  L.raw = off;     off += kIdxRawStages * raw_stage_bytes(fp8idx);
+  L.raw_stride = raw_stage_stride(fp8idx);
+  L.raw = off;     off += kIdxRawStages * L.raw_stride;
   L.lut = off;     off += 256 * 8;
   L.red = off;     off += 2 * kIdxWorkers * nq * 4;
-  L.bars = off;    off += (2 * kIdxRawStages + 8) * 8;
+  L.bars = off;    off += (2 * kIdxRawStages + 6) * 8;
   L.meta = off;    off += 3 * kIdxRawStages * 4;
   L.tinfo = off;   off += 4 * 4;
   L.cnt = off;     off += 2 * 4;
@@ -75,6 +80,12 @@ int idx_nq(int T) {
 
 size_t indexer_smem_bytes(bool fp8idx, int batch, int T) {
   return (size_t)idx_layout(idx_nq(T), fp8idx, batch).total;
+}
+
+__host__ __device__ constexpr int pow2_at_least(int x) {
+  int p = 32;
+  while (p < x) p *= 2;
+  return p;
 }
 
 // Exclusive prefix over the number of blocks of each sequence, in shared
@@ -115,26 +126,25 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
 __device__ __forceinline__ void sts128(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
 template <int NQ, bool FP8IDX>
-__global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
-  constexpr int kRaw = FP8IDX ? kBlock * kDim : kPageCodes + kPageScales;
-  constexpr int kCols = (2 * NQ) < 32 ? 32 : 2 * NQ;        // TMEM columns (power of 2)
-  constexpr int kChunk = NQ < 32 ? NQ : 32;                 // columns per TMEM load
+__global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(const __grid_constant__ IdxArgs a) {
+  constexpr int kND = NQ <= 64 ? 2 : 1;                      // accumulator buffers
+  constexpr int kCols = pow2_at_least(kACols + kND * NQ);    // TMEM columns
+  constexpr int kChunk = NQ < 32 ? NQ : 32;                  // columns per TMEM load
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
   const IdxLayout Ly = idx_layout(NQ, FP8IDX, a.B);
-  uint8_t* tile = smem + Ly.tile;
   uint8_t* qbuf = smem + Ly.qbuf;
   uint8_t* raw = smem + Ly.raw;
   uint2* lut = reinterpret_cast<uint2*>(smem + Ly.lut);
   float* red = reinterpret_cast<float*>(smem + Ly.red);            // [2][4][NQ]
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + Ly.bars);
   uint64_t* raw_empty = raw_full + kIdxRawStages;
-  uint64_t* tile_full = raw_empty + kIdxRawStages;                // workers -> MMA
-  uint64_t* tile_empty = tile_full + 2;                            // MMA -> workers
-  uint64_t* acc_full = tile_empty + 2;                             // MMA -> workers
-  uint64_t* acc_empty = acc_full + 2;                              // workers -> MMA
+  uint64_t* a_full = raw_empty + kIdxRawStages;                    // workers -> MMA
+  uint64_t* a_empty = a_full + 1;                                  // MMA -> workers
+  uint64_t* acc_full = a_empty + 1;                                // MMA -> workers [2]
+  uint64_t* acc_empty = acc_full + 2;                              // workers -> MMA [2]
   int* meta = reinterpret_cast<int*>(smem + Ly.meta);              // [stage][b, i, kind]
-  int* tinfo = reinterpret_cast<int*>(smem + Ly.tinfo);            // [2][skip, qsel]
+  int* tinfo = reinterpret_cast<int*>(smem + Ly.tinfo);            // [skip, qsel]
   int* cnt = reinterpret_cast<int*>(smem + Ly.cnt);                // [2]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
   int* prefix = reinterpret_cast<int*>(smem + Ly.prefix);
@@ -148,9 +158,9 @@ __global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
       mbar_init(&raw_full[s], 1);
       mbar_init(&raw_empty[s], kIdxWorkers);
     }
+    mbar_init(a_full, kIdxWorkers);
+    mbar_init(a_empty, 1);
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&tile_full[x], kIdxWorkers);
-      mbar_init(&tile_empty[x], 1);
       mbar_init(&acc_full[x], 1);
       mbar_init(&acc_empty[x], kIdxWorkers);
       cnt[x] = 0;
@@ -205,13 +215,14 @@ __global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
         meta[3 * s + 0] = b;
         meta[3 * s + 1] = i;
         meta[3 * s + 2] = kind;
-        uint8_t* dst = raw + s * kRaw;
+        uint8_t* dst = raw + s * Ly.raw_stride;
         if (kind == kPageLoad) {
-          mbar_expect_tx(&raw_full[s], kRaw);
           if (FP8IDX) {
-            bulk_g2s(dst, a.idx_data + p * (kBlock * kDim), kBlock * kDim, &raw_full[s]);
+            mbar_expect_tx(&raw_full[s], kBlock * kDim);
+            tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
           } else {
-            bulk_g2s(dst, a.idx_data + p * kPageCodes, kPageCodes, &raw_full[s]);
+            mbar_expect_tx(&raw_full[s], kPageCodes + kPageScales);
+            tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
             bulk_g2s(dst + kPageCodes, a.idx_scale + p * kPageScales, kPageScales, &raw_full[s]);
           }
         } else {
@@ -224,38 +235,45 @@ __global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_e4m3_f32(128, NQ);
+      constexpr uint32_t idesc_neg = idesc | (1u << 13);     // negate A
       for (int k = 0; k < n; ++k) {
-        const int x = k & 1;
-        if (!mbar_wait(&tile_full[x], (k >> 1) & 1)) { report(a.flags, 5, 2); break; }
-        if (k >= 2 && !mbar_wait(&acc_empty[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 3); break; }
+        const int x = k % kND;
+        if (!mbar_wait(a_full, k & 1)) { report(a.flags, 5, 2); break; }
+        if (k >= kND && !mbar_wait(&acc_empty[x], ((k / kND) - 1) & 1)) { report(a.flags, 5, 3); break; }
         tc_fence_after();
-        if (!tinfo[2 * x]) {
-          const uint32_t a0 = smem_u32(tile + x * kTileBytes);
-          const uint32_t b0 = smem_u32(qbuf + tinfo[2 * x + 1] * NQ * 128);
+        if (!tinfo[0]) {
+          const uint32_t d = tmem + kACols + x * NQ;
+          const uint32_t b0 = smem_u32(qbuf + tinfo[1] * NQ * 128);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_e4m3(tmem + x * NQ, desc_kmajor_sw128(a0 + 32 * kk),
-                        desc_kmajor_sw128(b0 + 32 * kk), idesc, kk > 0);
+            tc_mma_e4m3_ts(d, tmem + 8 * kk, desc_kmajor_sw128(b0 + 32 * kk), idesc, kk > 0);
+          if (!FP8IDX) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc_mma_e4m3_ts(d, tmem + 32 + 8 * kk, desc_kmajor_sw128(b0 + 32 * kk), idesc_neg, 1);
+          }
         }
-        tc_commit(&tile_empty[x]);
+        tc_commit(a_empty);
         tc_commit(&acc_full[x]);
       }
     }
   } else {
     // ------------------------------------------------------------ workers
-    // Epilogue of page kk (its accumulator is TMEM buffer kk & 1).
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lanes
+    const int row = 32 * warp + lane;                                   // key row of this thread
+    // Epilogue of page kk (accumulator buffer kk % kND).
     auto epilogue = [&](int kk, int pb, int pi, int pkind, int pL) -> bool {
-      const int xe = kk & 1;
-      if (!mbar_wait(&acc_full[xe], (kk >> 1) & 1)) { report(a.flags, 5, 6); return false; }
+      const int xd = kk % kND, xe = kk & 1;
+      if (!mbar_wait(&acc_full[xd], (kk / kND) & 1)) { report(a.flags, 5, 6); return false; }
       tc_fence_after();
       if (pkind == kPageLoad) {
-        const int key = pi * kBlock + 32 * warp + lane;
+        const int key = pi * kBlock + row;
         const int pos0 = pL - a.T;
         const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + t_first;
 #pragma unroll 1
         for (int c0 = 0; c0 < NQ; c0 += kChunk) {
           float v[32];
-          const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + xe * NQ + c0;
+          const uint32_t taddr = lane_base + kACols + xd * NQ + c0;
           if constexpr (kChunk == 32) {
             tmem_ld32(taddr, v);
           } else if constexpr (kChunk == 16) {
@@ -298,7 +316,7 @@ __global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
       __syncwarp();
       int last = 0;
       if (lane == 0) {
-        mbar_arrive(&acc_empty[xe]);
+        mbar_arrive(&acc_empty[xd]);
         __threadfence_block();
         last = (atomicAdd(&cnt[xe], 1) == kIdxWorkers - 1);
       }
@@ -318,8 +336,8 @@ __global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
             a.block_scores[(((long long)pb * a.T + t) * kG + (qg & 3)) * a.max_pages + pi] =
                 m * a.score_scale;
             if (pkind == kPageMasked && a.token_scores != nullptr) {
-              float* row = a.token_scores + (((long long)pb * a.T + t) * kG + (qg & 3)) * ctx;
-              for (int r = 0; r < kBlock; ++r) row[pi * kBlock + r] = -INFINITY;
+              float* rowp = a.token_scores + (((long long)pb * a.T + t) * kG + (qg & 3)) * ctx;
+              for (int r = 0; r < kBlock; ++r) rowp[pi * kBlock + r] = -INFINITY;
             }
           }
         }
@@ -334,10 +352,11 @@ __global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
     for (int k = 0; k <= n; ++k) {
       int nb = 0, ni = 0, nkind = kPageBad;
       if (k < n) {
-        // ---- decode page k into tile[k & 1]
-        const int x = k & 1, s = k % kIdxRawStages;
-        if (k >= 2 && !mbar_wait(&tile_empty[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 4); break; }
+        // ---- decode page k into the A operand in TMEM
+        const int s = k % kIdxRawStages;
         if (!mbar_wait(&raw_full[s], (k / kIdxRawStages) & 1)) { report(a.flags, 5, 5); break; }
+        if (k >= 1 && !mbar_wait(a_empty, (k - 1) & 1)) { report(a.flags, 5, 4); break; }
+        tc_fence_after();
         nb = meta[3 * s + 0];
         ni = meta[3 * s + 1];
         nkind = meta[3 * s + 2];
@@ -345,8 +364,8 @@ __global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
           cur_b = nb;
           L = a.seq_lens[nb];
           qsel ^= 1;
-          // B operand: the query rows of this chunk for sequence nb, swizzled.
-          // (Its previous user, the MMA of page k-2 or earlier, has completed.)
+          // B operand: the query rows of this chunk for sequence nb, swizzled
+          // (its previous user, an MMA of page k-2 or earlier, has completed).
           uint8_t* qb = qbuf + qsel * NQ * 128;
           constexpr int kRowsPerWarp = NQ / kIdxWorkers;
           for (int idx = lane; idx < kRowsPerWarp * 8; idx += 32) {
@@ -358,35 +377,50 @@ __global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(IdxArgs a) {
                   a.qi + (((long long)nb * a.T + t) * kG + (qg & 3)) * kDim + 16 * c);
             sts128(qb + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
           }
+          fence_async_smem();
         }
         if (nkind == kPageLoad) {
-          const uint8_t* rs = raw + s * kRaw;
-          uint8_t* tl = tile + x * kTileBytes;
+          const uint8_t* rs = raw + s * Ly.raw_stride;
           if constexpr (FP8IDX) {
-#pragma unroll 4
-            for (int p = 0; p < 8; ++p) {
-              const int r = 32 * warp + 4 * p + (lane >> 3), c = lane & 7;
-              sts128(tl + r * 128 + ((c ^ (r & 7)) << 4), lds128(rs + r * kDim + 16 * c));
+            // 128-byte rows loaded with the 128-byte swizzle: chunk c of row r
+            // sits at chunk position c ^ (r % 8).
+#pragma unroll
+            for (int c2 = 0; c2 < 4; ++c2) {
+              const uint4 x0 = lds128(rs + row * 128 + (((2 * c2) ^ (row & 7)) << 4));
+              const uint4 x1 = lds128(rs + row * 128 + (((2 * c2 + 1) ^ (row & 7)) << 4));
+              const uint32_t w8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+              tmem_st8(lane_base + 8 * c2, w8);
             }
           } else {
+            // 64-byte code rows loaded with the 64-byte swizzle: chunk c of
+            // row r sits at chunk position c ^ ((r / 2) % 4).
+            const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
+            const int sw = (row >> 1) & 3;
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const int r = 32 * warp + 8 * p + (lane >> 2), q = lane & 3;
-              uint32_t o[8];
-              dq32(lut, lds128(rs + r * kRowCodes + 16 * q),
-                   lds16(rs + kPageCodes + r * kRowScales + 2 * q), o);
-              sts128(tl + r * 128 + (((2 * q) ^ (r & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
-              sts128(tl + r * 128 + (((2 * q + 1) ^ (r & 7)) << 4),
-                     make_uint4(o[4], o[5], o[6], o[7]));
+            for (int c = 0; c < 4; ++c) {
+              const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
+              const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));   // scales 2c, 2c+1
+              const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
+              const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
+              const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
+              const uint32_t f1 = (s1 & 0x80u) ? 0x88888888u : 0u;
+              uint32_t pw[8], nw[8];
+              dq8_split(w4.x, r0, f0, pw[0], pw[1], nw[0], nw[1]);
+              dq8_split(w4.y, r0, f0, pw[2], pw[3], nw[2], nw[3]);
+              dq8_split(w4.z, r1, f1, pw[4], pw[5], nw[4], nw[5]);
+              dq8_split(w4.w, r1, f1, pw[6], pw[7], nw[6], nw[7]);
+              tmem_st8(lane_base + 8 * c, pw);
+              tmem_st8(lane_base + 32 + 8 * c, nw);
             }
           }
+          tmem_wait_st();
         }
-        fence_async_smem();   // make the tile writes visible to the tensor core
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&raw_empty[s]);
-          if (warp == 0) { tinfo[2 * x] = (nkind != kPageLoad); tinfo[2 * x + 1] = qsel; }
-          mbar_arrive(&tile_full[x]);
+          if (warp == 0) { tinfo[0] = (nkind != kPageLoad); tinfo[1] = qsel; }
+          mbar_arrive(a_full);
         }
       }
       // ---- epilogue of page k-1 (its MMA ran while page k was decoded)
@@ -413,7 +447,7 @@ static cudaError_t launch_nq(const IdxArgs& a, int num_sms, cudaStream_t st) {
     configured = smem;
   }
   const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), kIdxThreads, smem,
-                                 (2 * NQ) < 32 ? 32 : 2 * NQ);
+                                 pow2_at_least(kACols + (NQ <= 64 ? 2 : 1) * NQ));
   const int gy = (kG * a.T + NQ - 1) / NQ;
   const long long want = ((long long)num_sms * per_sm + gy - 1) / gy;
   const long long cap = (long long)a.B * a.max_pages;

@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "msa_device.cuh"
@@ -11,9 +12,10 @@
 namespace msa {
 
 constexpr int kIdxThreads = 6 * 32;     // 4 workers, 1 producer, 1 MMA warp
-constexpr int kIdxRawStages = 3;         // raw index-key pages in flight per CTA
+constexpr int kIdxRawStages = 4;         // raw index-key pages in flight per CTA
 
 struct IdxArgs {
+  CUtensorMap tmap_idx;        // rows of idx_data: 64-byte rows (64B swizzle) or 128 (128B swizzle)
   const uint8_t* idx_data;     // NVFP4 codes [P][128][64] or FP8 keys [P][128][128]
   const uint8_t* idx_scale;    // [P][128][8] (NVFP4 only)
   const int32_t* page_table;   // [B][max_pages] or null
@@ -35,6 +37,10 @@ cudaError_t launch_indexer(const IdxArgs& a, bool fp8idx, int num_sms, cudaStrea
 // columns each CTA allocates; 0 = none).
 int ctas_per_sm(const void* kernel, int threads, size_t smem, int tmem_cols);
 
+// Encode a tensor map over `rows` rows of `row_bytes` (64 or 128) bytes with
+// 128-row boxes and the matching shared-memory swizzle.  False on failure.
+bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes);
+
 // Top-k over block scores of every (b, t, g) row.
 cudaError_t launch_topk(const float* block_scores, const int32_t* seq_lens, int B, int T,
                         int max_pages, int32_t* sel, Flags* flags, cudaStream_t st);
@@ -44,7 +50,7 @@ cudaError_t launch_maxpool(const float* token_scores, const int32_t* seq_lens, i
 
 constexpr int kAttConsumers = 4;
 constexpr int kAttThreads = (kAttConsumers + 1) * 32;
-constexpr int kAttStages = 4;
+constexpr int kAttStages = 3;
 constexpr int kPartialFloats = kHpg * kDim + 2 * kHpg;   // O[16][128], m[16], l[16]
 
 struct AttnArgs {

@@ -17,39 +17,20 @@
 namespace msa {
 
 constexpr int kTopkThreads = 128;
-constexpr int kTopkWarps = kTopkThreads / 32;
-
-// Exclusive block-wide prefix count of `pred`; *total receives the sum.
-__device__ __forceinline__ int block_excl_count(bool pred, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned bal = __ballot_sync(0xffffffffu, pred);
-  const int in_warp = __popc(bal & ((1u << lane) - 1u));
-  if (lane == 0) warp_sums[warp] = __popc(bal);
-  __syncthreads();
-  int before = 0, sum = 0;
-#pragma unroll
-  for (int w = 0; w < kTopkWarps; ++w) {
-    const int v = warp_sums[w];
-    if (w < warp) before += v;
-    sum += v;
-  }
-  __syncthreads();
-  *total = sum;
-  return before + in_warp;
-}
+constexpr int kTopkCache = 4096;   // rows up to this many candidates are cached in smem
 
 __global__ void __launch_bounds__(kTopkThreads)
 topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_lens, int B, int T,
             int max_pages, int32_t* __restrict__ sel, Flags* flags) {
+  __shared__ unsigned keys[kTopkCache];
   __shared__ unsigned hist[256];
   __shared__ unsigned s_prefix;
   __shared__ int s_need;
-  __shared__ int warp_sums[kTopkWarps];
 
   const long long row = blockIdx.x;          // (b * T + t) * 4 + g
   const int b = (int)(row / (kG * T));
   const int t = (int)((row / kG) % T);
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* out = sel + row * kTopk;
   const int L = seq_lens[b];
   if (L < T || L > max_pages * kBlock) {
@@ -65,6 +46,14 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_le
   }
   const float* S = scores + row * max_pages;
   const int n = nb - 1;                      // candidates 0 .. nb-2
+  const bool cached = n <= kTopkCache;
+  if (cached)
+    for (int i = tid; i < n; i += kTopkThreads) keys[i] = float_key(S[i]);
+  auto key_at = [&](int i) -> unsigned { return cached ? keys[i] : float_key(S[i]); };
+
+  // Radix select, 8 bits per pass from the top: after the passes `prefix`
+  // is the key of the 15th best candidate and `need` how many candidates
+  // equal to it belong to the selection.
   unsigned prefix = 0;
   int need = kTopk - 1;
   for (int pass = 3; pass >= 0; --pass) {
@@ -72,45 +61,59 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_le
     for (int d = tid; d < 256; d += kTopkThreads) hist[d] = 0;
     __syncthreads();
     for (int i = tid; i < n; i += kTopkThreads) {
-      const unsigned k = float_key(S[i]);
+      const unsigned k = key_at(i);
       if (pass == 3 || (k >> (shift + 8)) == (prefix >> (shift + 8)))
         atomicAdd(&hist[(k >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      int above = 0;
-      for (int d = 255; d >= 0; --d) {
-        const int c = (int)hist[d];
-        if (above + c >= need) {
-          s_prefix = prefix | ((unsigned)d << shift);
-          s_need = need - above;
-          break;
+    if (warp == 0) {   // digit search: lane l owns bins 255-8l .. 248-8l (descending)
+      unsigned c[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { c[j] = hist[255 - 8 * lane - j]; sum += c[j]; }
+      unsigned incl = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)need);
+      if (lane == __ffs(hit) - 1) {
+        unsigned above = incl - sum;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (above + c[j] >= (unsigned)need) {
+            s_prefix = prefix | ((unsigned)(255 - 8 * lane - j) << shift);
+            s_need = need - (int)above;
+            break;
+          }
+          above += c[j];
         }
-        above += c;
       }
     }
     __syncthreads();
     prefix = s_prefix;
     need = s_need;
-    __syncthreads();
   }
-  // prefix = key of the 15th best candidate; take `need` of the blocks equal
-  // to it (lowest ids first) and every block above it.
-  int eq_seen = 0, emitted = 0;
-  for (int base = 0; base < n; base += kTopkThreads) {
-    const int i = base + tid;
-    const unsigned k = i < n ? float_key(S[i]) : 0u;
-    const bool gt = i < n && k > prefix;
-    const bool eq = i < n && k == prefix;
-    int eq_total, take_total;
-    const int eq_rank = eq_seen + block_excl_count(eq, warp_sums, &eq_total);
-    const bool take = gt || (eq && eq_rank < need);
-    const int slot = emitted + block_excl_count(take, warp_sums, &take_total);
-    if (take && slot < kTopk - 1) out[slot] = i;
-    eq_seen += eq_total;
-    emitted += take_total;
+  // One warp emits the selection in id order: every candidate above the
+  // threshold key and the `need` lowest ids equal to it, then the latest.
+  if (warp == 0) {
+    int eq_seen = 0, emitted = 0;
+    for (int base = 0; base < n && emitted < kTopk - 1; base += 32) {
+      const int i = base + lane;
+      const unsigned k = i < n ? key_at(i) : 0u;
+      const bool gt = i < n && k > prefix;
+      const bool eq = i < n && k == prefix;
+      const unsigned lt = (1u << lane) - 1u;
+      const unsigned beq = __ballot_sync(0xffffffffu, eq);
+      const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need);
+      const unsigned btake = __ballot_sync(0xffffffffu, take);
+      const int slot = emitted + __popc(btake & lt);
+      if (take && slot < kTopk - 1) out[slot] = i;
+      eq_seen += __popc(beq);
+      emitted += __popc(btake);
+    }
+    if (lane == 0) out[kTopk - 1] = nb - 1;
   }
-  if (tid == 0) out[kTopk - 1] = nb - 1;
 }
 
 __global__ void maxpool_kernel(const float* __restrict__ ts, const int32_t* __restrict__ seq_lens,
