@@ -1,24 +1,28 @@
 // msa_attn.cu -- exact attention over the selected blocks ([post, "MSA
 // primer"] and its Figure 1 caption: every query head of a GQA group attends
 // over that group's selected blocks) with NVFP4 K/V dequantised to E4M3 in
-// the kernel and fed to FP8 MMA ([post, "NVIDIA Blackwell optimized MSA
-// kernels"]).  post = vLLM 為 MiniMax-M3.1-Flash 提供 Day-0 支援
-// (hot.atechcom.net).
+// the kernel ([post, "NVIDIA Blackwell optimized MSA kernels"]).
+// post = vLLM 為 MiniMax-M3.1-Flash 提供 Day-0 支援 (hot.atechcom.net).
 //
 // Work unit: one (sequence, query token, group) = 16 query heads = one m16
-// MMA tile, split over its <= 16 selected blocks into `splits` CTAs.
-// Per CTA a producer warp gathers each selected block of the group's KV head
-// through the page table with four bulk async copies (K codes, K scales,
-// V codes, V scales = 18 KB) into a ring of stages; four consumer warps each
-// take 32 keys of every block:
-//   S  = Q K^T   A = Q (16 heads x 128 dims, registers, loaded once),
+// tile, split over its <= 16 selected blocks into `splits` CTAs.  A producer
+// warp gathers each selected block of the group's KV head through the page
+// table with four bulk async copies (K codes, K scales, V codes, V scales =
+// 18 KB) into a ring of stages; four consumer warps each take 32 keys of
+// every block.
+//
+// Arithmetic: K and V are decoded to their E4M3 values (the FP8 operands the
+// method prescribes) and widened exactly to f16, and both contractions run on
+// f16 tensor-core MMA with fp32 accumulation (m16n8k16).  On sm_100a the
+// warp-level FP8 MMA is not native (it costs about twenty issue slots per
+// instruction, measured), while the f16 one is; the products of E4M3 values
+// are exact in either, so the result is the FP8 contraction's.
+//   S  = Q K^T   A = Q (f16 fragments staged once in shared memory),
 //                B = K decoded from the stage straight into fragments;
 //   online softmax in the exp2 domain, masked beyond the query position;
-//   O += P V     A = P rounded to E4M3 from the S accumulators (the key order
-//                of S's columns is chosen so that each thread already holds
-//                the P values its A fragment needs), B = V, which the warp
-//                decodes and transposes (4x4 byte blocks) into a small
-//                per-warp V^T tile so each B fragment is one 64-bit load.
+//   O += P V     A = P (f16, from the S accumulators, FlashAttention-2
+//                layout), B = V decoded into a swizzled 16-key f16 tile and
+//                read transposed with ldmatrix.
 // The four warps' (m, l, O) merge in shared memory; with one split the CTA
 // writes bf16, otherwise it writes an fp32 partial and the last CTA of the
 // unit to finish (atomic counter, no waiting) combines the partials.
@@ -29,10 +33,10 @@
 namespace msa {
 
 constexpr int kAttStageBytes = 2 * (kPageCodes + kPageScales);   // K + V of one KV head
-constexpr int kVtWords = kDim * 8 + 32;                           // per warp: [128 dims][8 words] + pad
+constexpr int kVtBytes = 16 * kDim * 2;                           // per warp: 16 keys x 128 f16
 
 size_t attn_smem_bytes() {
-  return (size_t)kAttStages * kAttStageBytes + kAttConsumers * kVtWords * 4 + 4 * 32 * 16 +
+  return (size_t)kAttStages * kAttStageBytes + kAttConsumers * kVtBytes + 8 * 32 * 16 +
          256 * sizeof(uint2) + 2 * kAttStages * sizeof(uint64_t) + 4 * kTopk * sizeof(int) + 64;
 }
 
@@ -42,40 +46,12 @@ int attn_splits(long long units, int num_sms) {
   return s;
 }
 
-// Key (within a warp's 32) held as S column n of n-tile j:
-//   pi(j, n) = 4*(2j + n%2) + n/2.
-// Thread tig then holds the keys congruent to tig mod 4, which is exactly the
-// set its P A-fragment needs when the V^T word of key quad q holds keys
-// q, q+8, q+16, q+24; and each K or V load instruction of the warp covers 8
-// consecutive rows of the stage (bank-conflict free).
-__device__ __forceinline__ int key_of(int j, int n) {
-  return 4 * (2 * j + (n & 1)) + (n >> 1);
-}
-
-// 4x4 byte transpose: x[r] byte e -> y[e] byte r.
-__device__ __forceinline__ void transpose4x4(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3,
-                                             uint32_t& y0, uint32_t& y1, uint32_t& y2,
-                                             uint32_t& y3) {
-  const uint32_t t0 = __byte_perm(x0, x1, 0x5140), t1 = __byte_perm(x0, x1, 0x7362);
-  const uint32_t t2 = __byte_perm(x2, x3, 0x5140), t3 = __byte_perm(x2, x3, 0x7362);
-  y0 = __byte_perm(t0, t2, 0x5410);
-  y1 = __byte_perm(t0, t2, 0x7632);
-  y2 = __byte_perm(t1, t3, 0x5410);
-  y3 = __byte_perm(t1, t3, 0x7632);
-}
-
-// V^T word index of (dim d, key quad q): rows of 8 words, 8 words of padding
-// every 32 dims so the transposing writers hit 32 distinct banks.
-__device__ __forceinline__ int vt_index(int d, int q) {
-  return d * 8 + 8 * (d >> 5) + 2 * (q & 3) + (q >> 2);
-}
-
-__global__ void __launch_bounds__(kAttThreads, 3) attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(AttnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
-  uint32_t* vt_all = reinterpret_cast<uint32_t*>(smem + kAttStages * kAttStageBytes);
-  uint32_t* qfrag = vt_all + kAttConsumers * kVtWords;                  // [4][32][4]
-  uint2* lut = reinterpret_cast<uint2*>(qfrag + 4 * 32 * 4);
+  uint8_t* vt_all = smem + kAttStages * kAttStageBytes;                // [4 warps][16][256 B]
+  uint32_t* qfrag = reinterpret_cast<uint32_t*>(vt_all + kAttConsumers * kVtBytes);   // [8][32][4]
+  uint2* lut = reinterpret_cast<uint2*>(qfrag + 8 * 32 * 4);
   uint64_t* full = reinterpret_cast<uint64_t*>(lut + 256);
   uint64_t* empty = full + kAttStages;
   int* list = reinterpret_cast<int*>(empty + kAttStages);   // [16] block ids
@@ -147,26 +123,27 @@ __global__ void __launch_bounds__(kAttThreads, 3) attn_kernel(AttnArgs a) {
     }
   } else {
     // ------------------------------------------------------------ consumers
-    // Q A-fragments live in shared memory (qfrag[k-step][lane] = a0..a3), so
-    // they cost no registers across the block loop: row gid/gid+8 = heads
-    // 16g+gid / 16g+gid+8, k-step st covers dims 32tig+8st..+7.
+    // Q A-fragments (f16), k-step ks: a0/a1 = rows gid/gid+8, dims
+    // 32tig+4ks+{0,1}; a2/a3 = dims 32tig+4ks+{2,3}.  Staged once by warp 0.
     if (warp == 0) {
+      uint32_t w[2][8];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int h = g * kHpg + gid + 8 * r;
         const uint8_t* src = a.q + (((long long)b * a.T + t) * kHq + h) * kDim + 32 * tig;
         const uint4 x0 = *reinterpret_cast<const uint4*>(src);
         const uint4 x1 = *reinterpret_cast<const uint4*>(src + 16);
-        const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-        for (int st = 0; st < 4; ++st) {
-          qfrag[(st * 32 + lane) * 4 + r] = w[2 * st];          // a0 / a1
-          qfrag[(st * 32 + lane) * 4 + 2 + r] = w[2 * st + 1];  // a2 / a3
-        }
+        w[r][0] = x0.x; w[r][1] = x0.y; w[r][2] = x0.z; w[r][3] = x0.w;
+        w[r][4] = x1.x; w[r][5] = x1.y; w[r][6] = x1.z; w[r][7] = x1.w;
       }
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        *reinterpret_cast<uint4*>(&qfrag[(ks * 32 + lane) * 4]) =
+            make_uint4(e4m3x2_to_f16x2(w[0][ks]), e4m3x2_to_f16x2(w[1][ks]),
+                       e4m3x2_to_f16x2(w[0][ks] >> 16), e4m3x2_to_f16x2(w[1][ks] >> 16));
     }
     asm volatile("bar.sync 1, %0;\n" ::"n"(kAttConsumers * 32) : "memory");
-    uint32_t* vt = vt_all + warp * kVtWords;
+    uint8_t* vt = vt_all + warp * kVtBytes;     // this warp's 16-key f16 V tile
     const float sc = a.logit_scale_log2;
     for (int k = 0; k < nlist; ++k) {
       const int s = k % kAttStages;
@@ -180,50 +157,21 @@ __global__ void __launch_bounds__(kAttThreads, 3) attn_kernel(AttnArgs a) {
       const uint8_t* vs = vc + kPageCodes;
       const int key0 = list[k] * kBlock + 32 * warp;   // global position of this warp's key 0
 
-      // ---- S = Q K^T over this warp's 32 keys
+      // ---- S = Q K^T over this warp's 32 keys (n-tile j = keys 8j..8j+7)
       float sacc[4][4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
-        const int kk = 32 * warp + key_of(j, gid);
+        const int kk = 32 * warp + 8 * j + gid;
         uint32_t kw[8];
         dq32(lut, lds128(kc + kk * kRowCodes + 16 * tig), lds16(ks_ + kk * kRowScales + 2 * tig), kw);
 #pragma unroll
-        for (int st = 0; st < 4; ++st) {
+        for (int st = 0; st < 8; ++st) {
           const uint4 qa = *reinterpret_cast<const uint4*>(&qfrag[(st * 32 + lane) * 4]);
-          mma_e4m3(sacc[j], qa.x, qa.y, qa.z, qa.w, kw[2 * st], kw[2 * st + 1]);
+          mma_f16(sacc[j], qa.x, qa.y, qa.z, qa.w, e4m3x2_to_f16x2(kw[st]),
+                  e4m3x2_to_f16x2(kw[st] >> 16));
         }
       }
-
-      // ---- V^T tile: lane (kq, dc) decodes keys kq + 8r (r = 0..3), dims
-      // 32dc..32dc+31, in two halves of 16 dims (one scale byte each)
-      {
-        const int kq = lane >> 2, dc = lane & 3;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t vw[4][4];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int kk = 32 * warp + kq + 8 * r;
-            const uint2 c = *reinterpret_cast<const uint2*>(vc + kk * kRowCodes + 16 * dc + 8 * hf);
-            const uint2 row = lut[vs[kk * kRowScales + 2 * dc + hf]];
-            dq8(c.x, row, vw[r][0], vw[r][1]);
-            dq8(c.y, row, vw[r][2], vw[r][3]);
-          }
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            uint32_t y0, y1, y2, y3;
-            transpose4x4(vw[0][m], vw[1][m], vw[2][m], vw[3][m], y0, y1, y2, y3);
-            const int d = 32 * dc + 16 * hf + 4 * m;
-            vt[vt_index(d + 0, kq)] = y0;
-            vt[vt_index(d + 1, kq)] = y1;
-            vt[vt_index(d + 2, kq)] = y2;
-            vt[vt_index(d + 3, kq)] = y3;
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);   // stage no longer read by this warp
 
       // ---- mask, online softmax (exp2 domain)
       float mb[2] = {-INFINITY, -INFINITY};
@@ -231,7 +179,7 @@ __global__ void __launch_bounds__(kAttThreads, 3) attn_kernel(AttnArgs a) {
       for (int j = 0; j < 4; ++j) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int key = key0 + key_of(j, 2 * tig + (e & 1));
+          const int key = key0 + 8 * j + 2 * tig + (e & 1);
           float v = sacc[j][e] * sc;
           if (key > pos) v = -INFINITY;
           sacc[j][e] = v;
@@ -267,24 +215,41 @@ __global__ void __launch_bounds__(kAttThreads, 3) attn_kernel(AttnArgs a) {
           o[nt][2] *= alpha[1]; o[nt][3] *= alpha[1];
         }
       }
-      // ---- P fragments: logical k 4tig+e <-> key tig+8e (S n-tile e, column
-      // 2tig), logical 16+4tig+e <-> key tig+4+8e (n-tile e, column 2tig+1).
-      // P = Ph + Pl, both E4M3, so the FP8 MMA sees P to ~8 significant bits
-      // (one E4M3 term alone moves the weights of a few-key softmax by ~3%).
-      uint32_t ph0, pl0, ph1, pl1, ph2, pl2, ph3, pl3;
-      split_e4m3x4(sacc[0][0], sacc[1][0], sacc[2][0], sacc[3][0], ph0, pl0);
-      split_e4m3x4(sacc[0][2], sacc[1][2], sacc[2][2], sacc[3][2], ph1, pl1);
-      split_e4m3x4(sacc[0][1], sacc[1][1], sacc[2][1], sacc[3][1], ph2, pl2);
-      split_e4m3x4(sacc[0][3], sacc[1][3], sacc[2][3], sacc[3][3], ph3, pl3);
-      // ---- O += Ph V + Pl V
+
+      // ---- O += P V, 16 keys at a time (PV k-step kk = S n-tiles 2kk, 2kk+1)
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        const int d = 8 * nt + gid;
-        const uint2 bb = *reinterpret_cast<const uint2*>(vt + vt_index(d, tig));
-        mma_e4m3(o[nt], ph0, ph1, ph2, ph3, bb.x, bb.y);
-        mma_e4m3(o[nt], pl0, pl1, pl2, pl3, bb.x, bb.y);
+      for (int kk = 0; kk < 2; ++kk) {
+        const uint32_t pa0 = f32x2_to_f16x2(sacc[2 * kk][0], sacc[2 * kk][1]);
+        const uint32_t pa1 = f32x2_to_f16x2(sacc[2 * kk][2], sacc[2 * kk][3]);
+        const uint32_t pa2 = f32x2_to_f16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
+        const uint32_t pa3 = f32x2_to_f16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
+        // V tile: rows = the 16 keys 32w+16kk+0..15 (256 B of f16 each);
+        // 16-byte chunk c of row r at chunk position c ^ (r % 8).
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          const int r = 8 * p + gid, vk = 32 * warp + 16 * kk + r;
+          uint32_t vw[8];
+          dq32(lut, lds128(vc + vk * kRowCodes + 16 * tig), lds16(vs + vk * kRowScales + 2 * tig), vw);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)   // dims 32tig + 8i .. +7 = chunk 4tig + i
+            *reinterpret_cast<uint4*>(vt + r * 256 + (((4 * tig + i) ^ (r & 7)) << 4)) =
+                make_uint4(e4m3x2_to_f16x2(vw[2 * i]), e4m3x2_to_f16x2(vw[2 * i] >> 16),
+                           e4m3x2_to_f16x2(vw[2 * i + 1]), e4m3x2_to_f16x2(vw[2 * i + 1] >> 16));
+        }
+        __syncwarp();
+        // ldmatrix.x4.trans: matrix mi (lanes 8mi..8mi+7) = keys 8(mi&1)..+7 x dims 16n2+8(mi>>1)..+7
+        const int mi = lane >> 3, lr = (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int n2 = 0; n2 < 8; ++n2) {
+          const int chunk = 2 * n2 + (mi >> 1);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_trans(vt + lr * 256 + ((chunk ^ (lr & 7)) << 4), b0, b1, b2, b3);
+          mma_f16(o[2 * n2], pa0, pa1, pa2, pa3, b0, b1);
+          mma_f16(o[2 * n2 + 1], pa0, pa1, pa2, pa3, b2, b3);
+        }
+        __syncwarp();   // the tile is rewritten by the next 16 keys
       }
-      __syncwarp();   // V^T tile reused by the next block
+      if (lane == 0) mbar_arrive(&empty[s]);   // stage no longer read by this warp
     }
     // full row sums: add the 4 lanes of a row
 #pragma unroll

@@ -386,3 +386,44 @@ __device__ __forceinline__ void dq8_split(uint32_t w, uint2 r, uint32_t flip, ui
 }
 
 }  // namespace msa
+
+namespace msa {
+
+// Two E4M3 values (low 16 bits of w, low byte first) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(d) : "h"((uint16_t)(w & 0xFFFFu)));
+  return d;
+}
+
+// fp32 pair -> f16x2, lo in the low half (round to nearest even).
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// D(16x8 f32) += A(16x16 f16, row) * B(16x8 f16, col).
+//   a0:(row g, k 2t..2t+1) a1:(row g+8, same) a2:(row g, k 2t+8..) a3:(row g+8, k 2t+8..)
+//   b0:(k 2t..2t+1, col g) b1:(k 2t+8..2t+9, col g); d as in mma_e4m3.
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four 8x8 b16 matrices, transposed: lane 8i+j gives the address of row j of
+// matrix i; register i receives matrix i with thread (g, t) holding column g,
+// rows 2t and 2t+1.
+__device__ __forceinline__ void ldsm_x4_trans(const void* row_addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(row_addr))
+               : "memory");
+}
+
+}  // namespace msa
