@@ -23,8 +23,9 @@ BLOCK, TOPK, HEAD_DIM, KV_HEADS, Q_HEADS = 128, 16, 128, 4, 64
 EXPORTED = [
     "msa_workspace_size", "msa_workspace_init", "msa_indexer_score", "msa_block_maxpool_topk",
     "msa_sparse_attn_decode", "msa_decode", "msa_get_last_error", "msa_debug_nvfp4_table",
-    "msa_status_string",
+    "msa_status_string", "msa_decode_static",
 ]
+STATIC_WORKSPACE_BYTES = 16 << 20
 
 
 class MsaError(RuntimeError):
@@ -75,6 +76,8 @@ def load() -> ctypes.CDLL:
     L.msa_sparse_attn_decode.argtypes = [P(msa_cache), P(msa_seqs), vp, f32, vp, f32, vp, vp, sz, vp]
     L.msa_decode.restype = ctypes.c_int
     L.msa_decode.argtypes = [P(msa_cache), P(msa_seqs), vp, f32, vp, f32, f32, vp, vp, vp, sz, vp]
+    L.msa_decode_static.restype = ctypes.c_int
+    L.msa_decode_static.argtypes = [P(msa_cache), P(msa_seqs), vp, f32, vp, f32, f32, vp, vp, vp]
     L.msa_get_last_error.restype = ctypes.c_int
     L.msa_get_last_error.argtypes = [vp, vp, P(i32)]
     L.msa_debug_nvfp4_table.restype = ctypes.c_int
@@ -186,6 +189,15 @@ def msa_decode(cache: Cache, seqs: Seqs, qi, s_qi: float, q, s_q: float, softmax
     _check(load().msa_decode(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi), s_qi, _ptr(q),
                              s_q, softmax_scale, _ptr(out), _ptr(sel_out), _ptr(ws), ws.numel(),
                              _stream(stream)), "msa_decode")
+
+
+def msa_decode_static(cache: Cache, seqs: Seqs, qi, s_qi: float, q, s_q: float,
+                      softmax_scale: float, out, sel_out, stream=None):
+    """msa_decode with the library's fixed scratch array instead of a workspace
+    (for callers that cannot allocate device memory on the calling path)."""
+    _check(load().msa_decode_static(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi), s_qi,
+                                    _ptr(q), s_q, softmax_scale, _ptr(out), _ptr(sel_out),
+                                    _stream(stream)), "msa_decode_static")
 
 
 def msa_get_last_error(ws, stream=None):

@@ -179,6 +179,36 @@ MSA_API msa_status msa_get_last_error(void* ws, msa_stream_t stream, int32_t* de
  * E4M3 byte of rne_satfinite(e2m1(c) * e4m3(s)). */
 MSA_API msa_status msa_debug_nvfp4_table(uint8_t* out, msa_stream_t stream);
 
+/* Size of the library-owned scratch used by msa_decode_static (16 MiB); every
+ * GPU that loads the library holds it until the process exits. */
+#define MSA_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/* msa_decode without a caller-provided workspace: the pages have no
+ * counterpart for this entry point.  It is for callers that cannot allocate
+ * device memory where they call it -- code that runs under another
+ * framework's caching allocator it does not control, plugin or custom-op
+ * interfaces whose execution path forbids device allocations, or hot serving
+ * loops where a cudaMalloc would synchronise the device.  Inputs and outputs
+ * are caller-owned as for msa_decode; the scratch is a fixed device array of
+ * MSA_STATIC_WORKSPACE_BYTES inside the library, and nothing is allocated or
+ * freed by this call.
+ *   - Returns MSA_ERR_WORKSPACE when msa_workspace_size(seqs) is larger than
+ *     MSA_STATIC_WORKSPACE_BYTES (the batch needs a caller workspace and
+ *     msa_decode), MSA_ERR_INVALID_ARG / MSA_ERR_CUDA as msa_decode.
+ *   - The first call on a device looks up the array's device address for
+ *     that device (cudaGetSymbolAddress, with the device current); make that
+ *     first call before any stream capture on the device.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents; each call clears what must start at zero.  Calls that
+ *     overlap on the GPU (different streams, or different host threads
+ *     without ordering) race on the array: serialise them.
+ *   - Device-side bounds errors are recorded in the shared array, which the
+ *     next call clears; this entry point does not report them. */
+MSA_API msa_status msa_decode_static(const msa_cache* cache, const msa_seqs* seqs,
+                                     const uint8_t* qi, float s_qi, const uint8_t* q, float s_q,
+                                     float softmax_scale, uint16_t* out, int32_t* sel_out,
+                                     msa_stream_t stream);
+
 /* Static description of an error code. */
 MSA_API const char* msa_status_string(msa_status status);
 
