@@ -46,7 +46,7 @@ int attn_splits(long long units, int num_sms) {
   return s;
 }
 
-__global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(kAttThreads, 3) attn_kernel(AttnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
   uint8_t* vt_all = smem + kAttStages * kAttStageBytes;                // [4 warps][16][256 B]

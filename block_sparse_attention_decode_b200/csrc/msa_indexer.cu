@@ -126,7 +126,7 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
 __device__ __forceinline__ void sts128(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
 template <int NQ, bool FP8IDX>
-__global__ void __launch_bounds__(kIdxThreads, 3) indexer_kernel(const __grid_constant__ IdxArgs a) {
+__global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_constant__ IdxArgs a) {
   constexpr int kND = NQ <= 64 ? 2 : 1;                      // accumulator buffers
   constexpr int kCols = pow2_at_least(kACols + kND * NQ);    // TMEM columns
   constexpr int kChunk = NQ < 32 ? NQ : 32;                  // columns per TMEM load

@@ -50,7 +50,7 @@ cudaError_t launch_maxpool(const float* token_scores, const int32_t* seq_lens, i
 
 constexpr int kAttConsumers = 4;
 constexpr int kAttThreads = (kAttConsumers + 1) * 32;
-constexpr int kAttStages = 3;
+constexpr int kAttStages = 2;
 constexpr int kPartialFloats = kHpg * kDim + 2 * kHpg;   // O[16][128], m[16], l[16]
 
 struct AttnArgs {
