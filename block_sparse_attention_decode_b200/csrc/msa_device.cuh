@@ -426,4 +426,39 @@ __device__ __forceinline__ void ldsm_x4_trans(const void* row_addr, uint32_t& r0
                : "memory");
 }
 
+// Warp-wide 16x256b TMEM load, R = 1, 2 or 4 repetitions along columns:
+// thread (g = lane/4, t = lane%4) receives, for column group c < R,
+//   v[4c+0] = (lane g,   col 8c+2t), v[4c+1] = (lane g,   col 8c+2t+1),
+//   v[4c+2] = (lane g+8, col 8c+2t), v[4c+3] = (lane g+8, col 8c+2t+1),
+// lanes relative to taddr's lane (which must be a multiple of 16 within the
+// warp's 32-lane quarter).
+template <int R>
+__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, float (&v)[4 * R]) {
+  uint32_t r[4 * R];
+  if constexpr (R == 1) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+  } else if constexpr (R == 2) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+  } else {
+    static_assert(R == 4, "16x256b repetitions");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+  }
+#pragma unroll
+  for (int i = 0; i < 4 * R; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 }  // namespace msa

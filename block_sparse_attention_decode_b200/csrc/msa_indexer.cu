@@ -267,49 +267,61 @@ __global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_co
       if (!mbar_wait(&acc_full[xd], (kk / kND) & 1)) { report(a.flags, 5, 6); return false; }
       tc_fence_after();
       if (pkind == kPageLoad) {
-        const int key = pi * kBlock + row;
         const int pos0 = pL - a.T;
         const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + t_first;
+        // 16x256b loads: thread (g, t) holds keys g, g+8 (first load) and
+        // g+16, g+24 (second) of this warp's 32, columns 8c+2t and 8c+2t+1.
+        constexpr int kR = kChunk / 8;                       // column groups per load
+        const int g = lane >> 2, tq = lane & 3;
 #pragma unroll 1
         for (int c0 = 0; c0 < NQ; c0 += kChunk) {
-          float v[32];
-          const uint32_t taddr = lane_base + kACols + xd * NQ + c0;
-          if constexpr (kChunk == 32) {
-            tmem_ld32(taddr, v);
-          } else if constexpr (kChunk == 16) {
-            float v16[16];
-            tmem_ld16(taddr, v16);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = v16[j];
-          } else {
-            static_assert(kChunk == 8, "column chunk");
-            float v8[8];
-            tmem_ld8(taddr, v8);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = v8[j];
-          }
+          float va[4 * kR], vb[4 * kR];
+          tmem_ld_16x256b<kR>(lane_base + kACols + xd * NQ + c0, va);
+          tmem_ld_16x256b<kR>(lane_base + (16u << 16) + kACols + xd * NQ + c0, vb);
           tmem_wait_ld();
+          const int kb = pi * kBlock + 32 * warp + g;        // key of va[.][0..1]
           if (need_mask) {   // keys after a query's position do not count
 #pragma unroll
-            for (int j = 0; j < kChunk; ++j)
-              if (key > pos0 + ((qbase + c0 + j) >> 2)) v[j] = -INFINITY;
+            for (int i = 0; i < 4 * kR; ++i) {
+              const int col = c0 + 8 * (i >> 2) + 2 * tq + (i & 1);
+              const int lim = pos0 + ((qbase + col) >> 2);
+              const int dk = (i & 2) ? 8 : 0;
+              if (kb + dk > lim) va[i] = -INFINITY;
+              if (kb + 16 + dk > lim) vb[i] = -INFINITY;
+            }
           }
           if (a.token_scores != nullptr) {
 #pragma unroll
-            for (int j = 0; j < kChunk; ++j) {
-              const int qg = qbase + c0 + j, t = qg >> 2;
-              if (t < a.T)
-                a.token_scores[(((long long)pb * a.T + t) * kG + (qg & 3)) * ctx + key] =
-                    v[j] * a.score_scale;
+            for (int i = 0; i < 4 * kR; ++i) {
+              const int col = c0 + 8 * (i >> 2) + 2 * tq + (i & 1);
+              const int qg = qbase + col, t = qg >> 2;
+              const int dk = (i & 2) ? 8 : 0;
+              if (t < a.T) {
+                float* rowp = a.token_scores + (((long long)pb * a.T + t) * kG + (qg & 3)) * ctx;
+                rowp[kb + dk] = va[i] * a.score_scale;
+                rowp[kb + 16 + dk] = vb[i] * a.score_scale;
+              }
             }
           }
-          float part = -INFINITY;
+          // max over this thread's 4 keys, then over the 8 lane groups g
+          float m[2 * kR];
 #pragma unroll
-          for (int j = 0; j < kChunk; ++j) {
-            const float m = warp_max(v[j]);
-            part = (lane == j) ? m : part;
+          for (int c = 0; c < kR; ++c) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              m[2 * c + e] = fmaxf(fmaxf(va[4 * c + e], va[4 * c + 2 + e]),
+                                   fmaxf(vb[4 * c + e], vb[4 * c + 2 + e]));
           }
-          if (lane < kChunk) red[(xe * kIdxWorkers + warp) * NQ + c0 + lane] = part;
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 2 * kR; ++i) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], off));
+          }
+          if (g == 0) {
+            float* dst = red + (xe * kIdxWorkers + warp) * NQ + c0 + 2 * tq;
+#pragma unroll
+            for (int c = 0; c < kR; ++c) { dst[8 * c] = m[2 * c]; dst[8 * c + 1] = m[2 * c + 1]; }
+          }
         }
       }
       tc_fence_before();
