@@ -375,6 +375,31 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
+// x >> 16 as a multiply-high, which issues on the FMA pipe and leaves the
+// integer ALU pipe (which also runs prmt and the logic ops) to the decode.
+__device__ __forceinline__ uint32_t hi16(uint32_t x) {
+  uint32_t d;
+  asm("mul.hi.u32 %0, %1, 65536;\n" : "=r"(d) : "r"(x));
+  return d;
+}
+
+// dq8_split for a non-negative block scale (the usual case).
+__device__ __forceinline__ void dq8_split_pos(uint32_t w, uint2 r, uint32_t& p0, uint32_t& p1,
+                                              uint32_t& n0, uint32_t& n1) {
+  const uint32_t wn = w ^ 0x88888888u;
+  p0 = prmt(r.x, r.y, w);
+  p1 = prmt(r.x, r.y, hi16(w));
+  n0 = prmt(r.x, r.y, wn);
+  n1 = prmt(r.x, r.y, hi16(wn));
+}
+
+// max of three floats in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ void dq8_split(uint32_t w, uint2 r, uint32_t flip, uint32_t& p0,
                                           uint32_t& p1, uint32_t& n0, uint32_t& n1) {
   const uint32_t wp = w ^ flip;

@@ -309,8 +309,8 @@ __global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_co
           for (int c = 0; c < kR; ++c) {
 #pragma unroll
             for (int e = 0; e < 2; ++e)
-              m[2 * c + e] = fmaxf(fmaxf(va[4 * c + e], va[4 * c + 2 + e]),
-                                   fmaxf(vb[4 * c + e], vb[4 * c + 2 + e]));
+              m[2 * c + e] = fmaxf(fmax3(va[4 * c + e], va[4 * c + 2 + e], vb[4 * c + e]),
+                                   vb[4 * c + 2 + e]);
           }
 #pragma unroll
           for (int off = 4; off < 32; off <<= 1) {
@@ -408,21 +408,39 @@ __global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_co
             // row r sits at chunk position c ^ ((r / 2) % 4).
             const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
             const int sw = (row >> 1) & 3;
+            // warp-uniform branch: tcgen05.st is a .sync.aligned warp instruction
+            if (__all_sync(0xffffffffu, ((sc.x | sc.y) & 0x80808080u) == 0u)) {
+              // every block scale of the warp's 32 rows is non-negative
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-              const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));   // scales 2c, 2c+1
-              const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
-              const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
-              const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
-              const uint32_t f1 = (s1 & 0x80u) ? 0x88888888u : 0u;
-              uint32_t pw[8], nw[8];
-              dq8_split(w4.x, r0, f0, pw[0], pw[1], nw[0], nw[1]);
-              dq8_split(w4.y, r0, f0, pw[2], pw[3], nw[2], nw[3]);
-              dq8_split(w4.z, r1, f1, pw[4], pw[5], nw[4], nw[5]);
-              dq8_split(w4.w, r1, f1, pw[6], pw[7], nw[6], nw[7]);
-              tmem_st8(lane_base + 8 * c, pw);
-              tmem_st8(lane_base + 32 + 8 * c, nw);
+              for (int c = 0; c < 4; ++c) {
+                const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
+                const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));   // scales 2c, 2c+1
+                const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+                uint32_t pw[8], nw[8];
+                dq8_split_pos(w4.x, r0, pw[0], pw[1], nw[0], nw[1]);
+                dq8_split_pos(w4.y, r0, pw[2], pw[3], nw[2], nw[3]);
+                dq8_split_pos(w4.z, r1, pw[4], pw[5], nw[4], nw[5]);
+                dq8_split_pos(w4.w, r1, pw[6], pw[7], nw[6], nw[7]);
+                tmem_st8(lane_base + 8 * c, pw);
+                tmem_st8(lane_base + 32 + 8 * c, nw);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
+                const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));
+                const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
+                const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
+                const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
+                const uint32_t f1 = (s1 & 0x80u) ? 0x88888888u : 0u;
+                uint32_t pw[8], nw[8];
+                dq8_split(w4.x, r0, f0, pw[0], pw[1], nw[0], nw[1]);
+                dq8_split(w4.y, r0, f0, pw[2], pw[3], nw[2], nw[3]);
+                dq8_split(w4.z, r1, f1, pw[4], pw[5], nw[4], nw[5]);
+                dq8_split(w4.w, r1, f1, pw[6], pw[7], nw[6], nw[7]);
+                tmem_st8(lane_base + 8 * c, pw);
+                tmem_st8(lane_base + 32 + 8 * c, nw);
+              }
             }
           }
           tmem_wait_st();

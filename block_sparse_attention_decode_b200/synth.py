@@ -127,9 +127,12 @@ def _page_map(batch, nblk, max_pages, paged, seed, device):
 def make_workload(name: str, batch: int, seq_lens, q_tokens: int, *, paged: bool,
                   seed: int, device="cpu", idx_fp8: bool = False, max_pages: int | None = None,
                   plant_every: int = 0, scale_floor_byte: int = 0,
-                  chunk_pages: int = 2048) -> Workload:
+                  neg_scale_frac: float = 0.0, chunk_pages: int = 2048) -> Workload:
     """Build a workload.  seq_lens counts the q_tokens new tokens (which are the
-    last q_tokens positions of each sequence)."""
+    last q_tokens positions of each sequence).
+
+    ``neg_scale_frac`` > 0 sets the sign bit of that fraction of the block-scale
+    bytes (index, K and V), to exercise signed E4M3 block scales."""
     seq_lens = [int(L) for L in seq_lens]
     assert len(seq_lens) == batch and all(L >= q_tokens >= 1 for L in seq_lens)
     nblk = [(L + BLOCK - 1) // BLOCK for L in seq_lens]
@@ -199,6 +202,14 @@ def make_workload(name: str, batch: int, seq_lens, q_tokens: int, *, paged: bool
         v_data[p0:p1], v_scale[p0:p1] = encode_nvfp4(xv, S_NVFP4, scale_floor_byte)
         del xv
 
+    if neg_scale_frac > 0:
+        gn = _gen(seed, 8, device)
+        for t in (idx_scale, k_scale, v_scale):
+            if t is None:
+                continue
+            flip = torch.rand(t.shape, generator=gn, device=device) < neg_scale_frac
+            t |= flip.to(torch.uint8) << 7
+
     s_idx = S_Q if idx_fp8 else S_NVFP4
     return Workload(
         name=name, batch=batch, q_tokens=q_tokens,
@@ -208,7 +219,8 @@ def make_workload(name: str, batch: int, seq_lens, q_tokens: int, *, paged: bool
         v_data=v_data, v_scale=v_scale,
         qi=encode_fp8(qi_f, S_Q), q=encode_fp8(q_f, S_Q),
         s_idx=s_idx, meta={"seed": seed, "paged": paged, "plant_every": plant_every,
-                           "scale_floor_byte": scale_floor_byte},
+                           "scale_floor_byte": scale_floor_byte,
+                           "neg_scale_frac": neg_scale_frac},
     )
 
 

@@ -105,6 +105,8 @@ SMALL = [
                                scale_floor_byte=0x68)),
     ("planted", dict(batch=2, seq_lens=[8192, 8192], q_tokens=1, paged=False, seed=29,
                      plant_every=8)),
+    ("neg_scales", dict(batch=2, seq_lens=[5000, 2600], q_tokens=4, paged=True, seed=30,
+                        neg_scale_frac=0.05)),
 ]
 
 
@@ -208,7 +210,10 @@ def test_topk_token_level_input():
 
 
 # ----------------------------------------------------------- attention -----
-@pytest.mark.parametrize("name,kw", SMALL[:5], ids=[s[0] for s in SMALL[:5]])
+ATT_CASES = SMALL[:5] + SMALL[-1:]
+
+
+@pytest.mark.parametrize("name,kw", ATT_CASES, ids=[s[0] for s in ATT_CASES])
 def test_attention_given_oracle_selection(name, kw):
     w = dev_workload(name, **kw)
     c, _ = parity.host_cache(w)
