@@ -104,6 +104,7 @@ msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi,
   a.token_scores = token_scores;
   a.block_scores = block_scores;
   a.flags = at<Flags>(ws, L.flags);
+  a.work = at<int>(ws, L.flags + kWorkOffset);
   a.score_scale = s_qi * c->s_idx;
   a.B = s->batch;
   a.T = s->q_tokens;

@@ -29,11 +29,14 @@ constexpr int kRowScales = 8;    // E4M3 scale bytes per 128-vector
 constexpr int kPageCodes = kBlock * kRowCodes;    // 8192
 constexpr int kPageScales = kBlock * kRowScales;  // 1024
 
-// Workspace header: device error flags (first 256 bytes of the workspace).
+// Workspace header (first 256 bytes of the workspace, zeroed by
+// msa_workspace_init): the device error flags at offset 0, the indexer's
+// work-distribution counters at kWorkOffset.
 struct Flags {
   int code;     // first msa_status recorded on the device (0 = none)
   int detail;   // the offending value
 };
+constexpr int kWorkOffset = 64;   // int[2]: next work item, CTAs finished (0 between calls)
 
 __device__ __forceinline__ void report(Flags* f, int code, int detail) {
   if (atomicCAS(&f->code, 0, code) == 0) atomicExch(&f->detail, detail);

@@ -10,38 +10,53 @@
 // lanes) and a chunk of NQ index queries (T tokens x 4 groups, padded to a
 // multiple of 8) as the N side.
 //
-// Work split: the pages of all sequences form one flat list; CTA x takes one
-// contiguous slice of it (even load for ragged lengths); grid y tiles the
-// index queries in chunks of NQ.  Warp roles inside a CTA:
-//   warp 4 (producer): per page one tiled TMA load of the codes (64-byte
+// Work split: the pages of all sequences form one flat list, cut into chunks
+// of kChunkPages; a work item is (query tile of NQ index queries, chunk).
+// Persistent CTAs (two per SM) take items from a counter in the workspace
+// header as they go, so that CTAs sharing an SM -- which the warp schedulers
+// do not serve equally -- and ragged batches still finish together; the last
+// CTA to finish resets the counter.  Warp roles inside a CTA, all running a
+// few pages apart:
+//   warp 16 (producer): per page one tiled TMA load of the codes (64-byte
 //     swizzle, so that row-per-thread reads are bank-conflict free) and one
 //     bulk copy of the scales into a ring of shared-memory stages;
-//   warps 0-3 (workers): thread = key row (= TMEM lane).  NVFP4 rows are
-//     decoded by sign: K+ holds E4M3(|v|) of the positive elements, K- of the
-//     negative ones (one prmt per 4 codes each, see dq8_split), and both go
-//     straight to tensor memory with tcgen05.st -- the A operand never
-//     touches shared memory.  One page behind, the workers read the
-//     accumulator from TMEM, mask keys after each query's position and
-//     reduce the 128 keys with redux.sync.max.f32 (combining the four warps'
-//     partial maxima in shared memory);
-//   warp 5 (MMA): one thread issues per page 4 tcgen05.mma with A = K+ and 4
+//   warps 0-7 (decoders): warps w and w+4 share the TMEM lanes (= key rows)
+//     32(w%4)..32(w%4)+31; thread = key row, warp w decoding dims 0-63 of
+//     its row and warp w+4 dims 64-127.  NVFP4 rows are decoded by sign: K+
+//     holds E4M3(|v|) of the positive elements, K- of the negative ones (one
+//     prmt per 4 codes each, see dq8_split), and both go straight to tensor
+//     memory with tcgen05.st into one of two A buffers -- the A operand never
+//     touches shared memory, and page k+1 is decoded while page k's MMA runs;
+//   warp 17 (MMA): one thread issues per page 4 tcgen05.mma with A = K+ and 4
 //     with A = K- and the negate-A bit (K = 32 each, A from TMEM, B = the
-//     queries in shared memory) into a double-buffered TMEM accumulator.
+//     queries in shared memory) into a double-buffered TMEM accumulator;
+//   warps 8-15 (epilogue, two groups of four taking the even and the odd
+//     pages, so that two pages are reduced at once): warp 8+4j+q reads the
+//     accumulator lanes of quarter q,
+//     masks keys after each query's position, and reduces over keys: in-thread
+//     over the four keys a 16x256b load gives each thread, then xor shuffles
+//     across lane groups; after a rendezvous on an mbarrier each warp
+//     combines the four quarters' partial maxima of a quarter of the columns
+//     and writes those block scores.
 // Every wait is a bounded mbarrier wait; on a timeout a thread records
 // MSA_ERR_TIMEOUT and leaves its loop, and TMEM is freed before exit.
 #include "msa_internal.h"
 
 namespace msa {
 
-constexpr int kIdxWorkers = 4;
-constexpr int kIdxProducerWarp = 4;
-constexpr int kIdxMmaWarp = 5;
-constexpr int kACols = 64;                  // TMEM columns of the A operand (K+ | K-)
+constexpr int kIdxDecoders = 8;             // two per TMEM lane quarter
+constexpr int kIdxEpilogue = 4;             // per group: one per TMEM lane quarter
+constexpr int kIdxEpiWarp0 = 8;             // two groups: even and odd pages
+constexpr int kIdxProducerWarp = 16;
+constexpr int kIdxMmaWarp = 17;
+constexpr int kABufCols = 64;               // TMEM columns of one A buffer (K+ | K-)
+constexpr int kACols = 2 * kABufCols;       // two A buffers
 
-enum : int { kPageLoad = 0, kPageMasked = 1, kPageBad = 2 };
+enum : int { kPageLoad = 0, kPageMasked = 1, kPageBad = 2, kPageEnd = 3 };
+constexpr int kChunkPages = 8;              // pages per work item
 
 struct IdxLayout {
-  int qbuf, raw, raw_stride, lut, red, bars, meta, tinfo, cnt, tslot, prefix, scratch, total;
+  int qbuf, raw, raw_stride, lut, red, bars, meta, tinfo, pinfo, tslot, prefix, scratch, total;
 };
 
 // Bytes of one raw page in shared memory (codes [+ scales]), 1024-aligned.
@@ -56,11 +71,11 @@ __host__ __device__ inline IdxLayout idx_layout(int nq, bool fp8idx, int batch) 
   L.raw_stride = raw_stage_stride(fp8idx);
   L.raw = off;     off += kIdxRawStages * L.raw_stride;
   L.lut = off;     off += 256 * 8;
-  L.red = off;     off += 2 * kIdxWorkers * nq * 4;
-  L.bars = off;    off += (2 * kIdxRawStages + 6) * 8;
-  L.meta = off;    off += 3 * kIdxRawStages * 4;
-  L.tinfo = off;   off += 4 * 4;
-  L.cnt = off;     off += 2 * 4;
+  L.red = off;     off += 2 * kIdxEpilogue * nq * 4;          // [group][quarter][nq]
+  L.bars = off;    off += (2 * kIdxRawStages + 10) * 8;
+  L.meta = off;    off += 4 * kIdxRawStages * 4;           // per stage: b, i, kind, tile
+  L.tinfo = off;   off += 2 * 2 * 4;                       // per A buffer: what, qsel
+  L.pinfo = off;   off += 4 * 8 * 4;                       // ring of 4: b, i, kind, L, tile
   L.tslot = off;   off += 16;
   L.prefix = off;  off += (batch + 1) * 4;
   L.scratch = off; off += kIdxThreads * 4;
@@ -126,26 +141,27 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
 __device__ __forceinline__ void sts128(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
 template <int NQ, bool FP8IDX>
-__global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_constant__ IdxArgs a) {
+__global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_constant__ IdxArgs a) {
   constexpr int kND = NQ <= 64 ? 2 : 1;                      // accumulator buffers
   constexpr int kCols = pow2_at_least(kACols + kND * NQ);    // TMEM columns
-  constexpr int kChunk = NQ < 32 ? NQ : 32;                  // columns per TMEM load
+  constexpr int kChunk = NQ < 32 ? NQ : (NQ >= 128 ? 16 : 32);   // columns per TMEM load
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
   const IdxLayout Ly = idx_layout(NQ, FP8IDX, a.B);
   uint8_t* qbuf = smem + Ly.qbuf;
   uint8_t* raw = smem + Ly.raw;
   uint2* lut = reinterpret_cast<uint2*>(smem + Ly.lut);
-  float* red = reinterpret_cast<float*>(smem + Ly.red);            // [2][4][NQ]
+  float* red = reinterpret_cast<float*>(smem + Ly.red);            // [group][quarter][NQ]
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + Ly.bars);
   uint64_t* raw_empty = raw_full + kIdxRawStages;
-  uint64_t* a_full = raw_empty + kIdxRawStages;                    // workers -> MMA
-  uint64_t* a_empty = a_full + 1;                                  // MMA -> workers
-  uint64_t* acc_full = a_empty + 1;                                // MMA -> workers [2]
-  uint64_t* acc_empty = acc_full + 2;                              // workers -> MMA [2]
-  int* meta = reinterpret_cast<int*>(smem + Ly.meta);              // [stage][b, i, kind]
-  int* tinfo = reinterpret_cast<int*>(smem + Ly.tinfo);            // [skip, qsel]
-  int* cnt = reinterpret_cast<int*>(smem + Ly.cnt);                // [2]
+  uint64_t* a_full = raw_empty + kIdxRawStages;                    // decoders -> MMA [2]
+  uint64_t* a_empty = a_full + 2;                                  // MMA -> decoders [2]
+  uint64_t* acc_full = a_empty + 2;                                // MMA -> epilogue [2]
+  uint64_t* acc_empty = acc_full + 2;                              // epilogue -> MMA [2]
+  uint64_t* red_full = acc_empty + 2;                              // group rendezvous [2]
+  int* meta = reinterpret_cast<int*>(smem + Ly.meta);              // [stage][b, i, kind, tile]
+  int* tinfo = reinterpret_cast<int*>(smem + Ly.tinfo);            // [A buffer][what, qsel]
+  int* pinfo = reinterpret_cast<int*>(smem + Ly.pinfo);            // [k % 4][b, i, kind, L, tile]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
   int* prefix = reinterpret_cast<int*>(smem + Ly.prefix);
   int* scratch = reinterpret_cast<int*>(smem + Ly.scratch);
@@ -156,14 +172,14 @@ __global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_co
   if (tid == 0) {
     for (int s = 0; s < kIdxRawStages; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], kIdxWorkers);
+      mbar_init(&raw_empty[s], kIdxDecoders);
     }
-    mbar_init(a_full, kIdxWorkers);
-    mbar_init(a_empty, 1);
     for (int x = 0; x < 2; ++x) {
+      mbar_init(&a_full[x], kIdxDecoders);
+      mbar_init(&a_empty[x], 1);
       mbar_init(&acc_full[x], 1);
-      mbar_init(&acc_empty[x], kIdxWorkers);
-      cnt[x] = 0;
+      mbar_init(&acc_empty[x], kIdxEpilogue);
+      mbar_init(&red_full[x], kIdxEpilogue);
     }
     mbar_fence_init();
   }
@@ -177,58 +193,79 @@ __global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_co
   const uint32_t tmem = *tslot;
 
   const int total = prefix[a.B];
-  const int lo = (int)((long long)total * blockIdx.x / gridDim.x);
-  const int hi = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
-  const int n = hi - lo;
-  const int qbase = blockIdx.y * NQ;           // first index query of this chunk
-  const int t_first = qbase >> 2;
-  const int t_last = min(a.T - 1, (qbase + NQ - 1) >> 2);
+  const int gy = (kG * a.T + NQ - 1) / NQ;                  // query tiles
+  const int nchunks = (total + kChunkPages - 1) / kChunkPages;
+  const int items = nchunks * gy;
   const long long ctx = (long long)a.max_pages * kBlock;
 
   if (warp == kIdxProducerWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n > 0) {
-      int b;
-      {  // prefix[b] <= lo < prefix[b+1]
-        int l = 0, r = a.B;
-        while (r - l > 1) { const int m = (l + r) >> 1; if (prefix[m] <= lo) l = m; else r = m; }
-        b = l;
-      }
-      int i = lo - prefix[b];
-      for (int k = 0; k < n; ++k) {
-        const int s = k % kIdxRawStages;
-        if (k >= kIdxRawStages && !mbar_wait(&raw_empty[s], ((k / kIdxRawStages) - 1) & 1)) {
-          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1);
-          break;
+    if (lane == 0) {
+      int k = 0;                                  // page slot (stage k % kIdxRawStages)
+      bool ok = true;
+      auto slot = [&](int kk) -> bool {           // wait until stage kk % S is free
+        return kk < kIdxRawStages ||
+               mbar_wait(&raw_empty[kk % kIdxRawStages], ((kk / kIdxRawStages) - 1) & 1);
+      };
+      int item = atomicAdd(&a.work[0], 1);
+      while (item < items && ok) {
+        const int nxt = atomicAdd(&a.work[0], 1);  // claimed early: its latency overlaps this item
+        const int y = item / nchunks, p0 = (item % nchunks) * kChunkPages;
+        const int p1 = min(total, p0 + kChunkPages);
+        const int t_last = min(a.T - 1, (y * NQ + NQ - 1) >> 2);
+        int b;
+        {  // prefix[b] <= p0 < prefix[b+1]
+          int l = 0, r = a.B;
+          while (r - l > 1) { const int m = (l + r) >> 1; if (prefix[m] <= p0) l = m; else r = m; }
+          b = l;
         }
-        while (i >= prefix[b + 1] - prefix[b]) { i -= prefix[b + 1] - prefix[b]; ++b; }
-        const int L = a.seq_lens[b];
-        int kind = kPageLoad;
-        const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + i]
-                                         : (long long)b * a.max_pages + i;
-        if (i * kBlock > L - a.T + t_last) {
-          kind = kPageMasked;
-        } else if (p < 0 || p >= a.num_pages) {
-          report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)p);
-          kind = kPageBad;
-        }
-        meta[3 * s + 0] = b;
-        meta[3 * s + 1] = i;
-        meta[3 * s + 2] = kind;
-        uint8_t* dst = raw + s * Ly.raw_stride;
-        if (kind == kPageLoad) {
-          if (FP8IDX) {
-            mbar_expect_tx(&raw_full[s], kBlock * kDim);
-            tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
-          } else {
-            mbar_expect_tx(&raw_full[s], kPageCodes + kPageScales);
-            tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
-            bulk_g2s(dst + kPageCodes, a.idx_scale + p * kPageScales, kPageScales, &raw_full[s]);
+        int i = p0 - prefix[b];
+        for (int pg = p0; pg < p1; ++pg, ++k) {
+          if (!slot(k)) { report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1); ok = false; break; }
+          const int s = k % kIdxRawStages;
+          while (i >= prefix[b + 1] - prefix[b]) { i -= prefix[b + 1] - prefix[b]; ++b; }
+          const int L = a.seq_lens[b];
+          int kind = kPageLoad;
+          const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + i]
+                                           : (long long)b * a.max_pages + i;
+          if (i * kBlock > L - a.T + t_last) {
+            kind = kPageMasked;
+          } else if (p < 0 || p >= a.num_pages) {
+            report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)p);
+            kind = kPageBad;
           }
-        } else {
-          mbar_arrive(&raw_full[s]);
+          meta[4 * s + 0] = b;
+          meta[4 * s + 1] = i;
+          meta[4 * s + 2] = kind;
+          meta[4 * s + 3] = y;
+          uint8_t* dst = raw + s * Ly.raw_stride;
+          if (kind == kPageLoad) {
+            if (FP8IDX) {
+              mbar_expect_tx(&raw_full[s], kBlock * kDim);
+              tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
+            } else {
+              mbar_expect_tx(&raw_full[s], kPageCodes + kPageScales);
+              tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
+              bulk_g2s(dst + kPageCodes, a.idx_scale + p * kPageScales, kPageScales, &raw_full[s]);
+            }
+          } else {
+            mbar_arrive(&raw_full[s]);
+          }
+          ++i;
         }
-        ++i;
+        item = nxt;
+      }
+      // two end markers: one for each epilogue group
+      for (int e = 0; e < 2 && ok; ++e, ++k) {
+        if (!slot(k)) { report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1); break; }
+        meta[4 * (k % kIdxRawStages) + 2] = kPageEnd;
+        mbar_arrive(&raw_full[k % kIdxRawStages]);
+      }
+      // every CTA has made its last claim once all have arrived here
+      __threadfence();
+      if (atomicAdd(&a.work[1], 1) == (int)gridDim.x - 1) {
+        atomicExch(&a.work[0], 0);
+        atomicExch(&a.work[1], 0);
       }
     }
   } else if (warp == kIdxMmaWarp) {
@@ -236,50 +273,78 @@ __global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_co
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_e4m3_f32(128, NQ);
       constexpr uint32_t idesc_neg = idesc | (1u << 13);     // negate A
-      for (int k = 0; k < n; ++k) {
-        const int x = k % kND;
-        if (!mbar_wait(a_full, k & 1)) { report(a.flags, 5, 2); break; }
-        if (k >= kND && !mbar_wait(&acc_empty[x], ((k / kND) - 1) & 1)) { report(a.flags, 5, 3); break; }
+      // B descriptors of the two query buffers; a K = 32 slice starts 32
+      // bytes further (2 in the descriptor's 16-byte address units)
+      const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(qbuf));
+      const uint64_t bdesc1 = desc_kmajor_sw128(smem_u32(qbuf + NQ * 128));
+      // Page k uses A buffer k % 2 and accumulator k % kND; with two
+      // accumulators one commit (to acc_full[k % 2]) releases both.
+      auto issue = [&](int k, int ab, int x, int& ends) -> bool {
+        if (!mbar_wait(&a_full[ab], (k >> 1) & 1)) { report(a.flags, 5, 2); return false; }
+        if (k >= kND && !mbar_wait(&acc_empty[x], ((k / kND) - 1) & 1)) { report(a.flags, 5, 3); return false; }
         tc_fence_after();
-        if (!tinfo[0]) {
+        const int what = tinfo[2 * ab];            // 0 = MMA, 1 = nothing to score, 2 = end
+        ends += (what == 2);
+        if (what == 0) {
           const uint32_t d = tmem + kACols + x * NQ;
-          const uint32_t b0 = smem_u32(qbuf + tinfo[1] * NQ * 128);
+          const uint32_t ta = tmem + ab * kABufCols;
+          const uint64_t bd = tinfo[2 * ab + 1] ? bdesc1 : bdesc0;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma_e4m3_ts(d, tmem + 8 * kk, desc_kmajor_sw128(b0 + 32 * kk), idesc, kk > 0);
+          for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc, kk > 0);
           if (!FP8IDX) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              tc_mma_e4m3_ts(d, tmem + 32 + 8 * kk, desc_kmajor_sw128(b0 + 32 * kk), idesc_neg, 1);
+            for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 32 + 8 * kk, bd + 2 * kk, idesc_neg, 1);
           }
         }
-        tc_commit(a_empty);
-        tc_commit(&acc_full[x]);
+        if constexpr (kND == 2) {
+          tc_commit(&acc_full[ab]);
+        } else {
+          tc_commit(&a_empty[ab]);
+          tc_commit(&acc_full[x]);
+        }
+        return true;
+      };
+      int ends = 0;
+      for (int k = 0; ends < 2; k += 2) {
+        if (!issue(k, 0, 0, ends)) break;
+        if (ends < 2 && !issue(k + 1, 1, kND == 2 ? 1 : 0, ends)) break;
       }
     }
-  } else {
-    // ------------------------------------------------------------ workers
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lanes
-    const int row = 32 * warp + lane;                                   // key row of this thread
-    // Epilogue of page kk (accumulator buffer kk % kND).
-    auto epilogue = [&](int kk, int pb, int pi, int pkind, int pL) -> bool {
-      const int xd = kk % kND, xe = kk & 1;
-      if (!mbar_wait(&acc_full[xd], (kk / kND) & 1)) { report(a.flags, 5, 6); return false; }
+  } else if (warp >= kIdxEpiWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3, group = (warp - kIdxEpiWarp0) >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);   // this warp's TMEM lanes
+    const int g = lane >> 2, tq = lane & 3;
+    // With two accumulators the groups alternate pages; with one (NQ >= 128)
+    // group 0 takes every page, since a waiter two phases ahead of an
+    // mbarrier would read its parity wrong.
+    constexpr int kStep = kND == 2 ? 2 : 1;
+    const bool active = kND == 2 || group == 0;
+    for (int kk = group; active; kk += kStep) {
+      const int xd = kk % kND, xe = group, jr = kk / kStep;   // jr: this group's page count
+      if (!mbar_wait(&acc_full[xd], (kk / kND) & 1)) { report(a.flags, 5, 6); break; }
       tc_fence_after();
+      const int* pf = pinfo + 8 * (kk & 3);
+      const int pb = pf[0], pi = pf[1], pkind = pf[2], pL = pf[3];
+      if (pkind == kPageEnd) {
+        if (lane == 0) mbar_arrive(&acc_empty[xd]);
+        break;
+      }
+      const int qbase = pf[4] * NQ;                // first index query of this page's tile
+      const int t_first = qbase >> 2;
       if (pkind == kPageLoad) {
         const int pos0 = pL - a.T;
         const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + t_first;
         // 16x256b loads: thread (g, t) holds keys g, g+8 (first load) and
-        // g+16, g+24 (second) of this warp's 32, columns 8c+2t and 8c+2t+1.
+        // g+16, g+24 (second) of this quarter's 32, columns 8c+2t and 8c+2t+1.
         constexpr int kR = kChunk / 8;                       // column groups per load
-        const int g = lane >> 2, tq = lane & 3;
 #pragma unroll 1
         for (int c0 = 0; c0 < NQ; c0 += kChunk) {
           float va[4 * kR], vb[4 * kR];
           tmem_ld_16x256b<kR>(lane_base + kACols + xd * NQ + c0, va);
           tmem_ld_16x256b<kR>(lane_base + (16u << 16) + kACols + xd * NQ + c0, vb);
           tmem_wait_ld();
-          const int kb = pi * kBlock + 32 * warp + g;        // key of va[.][0..1]
+          const int kb = pi * kBlock + 32 * quarter + g;     // key of va[.][0..1]
           if (need_mask) {   // keys after a query's position do not count
 #pragma unroll
             for (int i = 0; i < 4 * kR; ++i) {
@@ -318,7 +383,7 @@ __global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_co
             for (int i = 0; i < 2 * kR; ++i) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], off));
           }
           if (g == 0) {
-            float* dst = red + (xe * kIdxWorkers + warp) * NQ + c0 + 2 * tq;
+            float* dst = red + (xe * kIdxEpilogue + quarter) * NQ + c0 + 2 * tq;
 #pragma unroll
             for (int c = 0; c < kR; ++c) { dst[8 * c] = m[2 * c]; dst[8 * c + 1] = m[2 * c + 1]; }
           }
@@ -326,136 +391,146 @@ __global__ void __launch_bounds__(kIdxThreads, 4) indexer_kernel(const __grid_co
       }
       tc_fence_before();
       __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        mbar_arrive(&acc_empty[xd]);
-        __threadfence_block();
-        last = (atomicAdd(&cnt[xe], 1) == kIdxWorkers - 1);
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {   // the last warp of this page combines the four partial maxima
-        __threadfence_block();
-        if (pkind != kPageBad) {
-          for (int col = lane; col < NQ; col += 32) {
-            const int qg = qbase + col, t = qg >> 2;
-            if (t >= a.T) continue;
-            float m = -INFINITY;
-            if (pkind == kPageLoad) {
+      // rendezvous of the four quarters (bounded mbarrier wait), then each
+      // warp combines a quarter of the columns
+      if (lane == 0) mbar_arrive(&red_full[xe]);
+      if (!mbar_wait(&red_full[xe], jr & 1)) { report(a.flags, 5, 7); break; }
+      if (pkind != kPageBad) {
+        constexpr int kPer = NQ / kIdxEpilogue;
+        for (int j = lane; j < kPer; j += 32) {
+          const int col = quarter * kPer + j;
+          const int qg = qbase + col, t = qg >> 2;
+          if (t >= a.T) continue;
+          float m = -INFINITY;
+          if (pkind == kPageLoad) {
 #pragma unroll
-              for (int w = 0; w < kIdxWorkers; ++w)
-                m = fmaxf(m, red[(xe * kIdxWorkers + w) * NQ + col]);
-            }
-            a.block_scores[(((long long)pb * a.T + t) * kG + (qg & 3)) * a.max_pages + pi] =
-                m * a.score_scale;
-            if (pkind == kPageMasked && a.token_scores != nullptr) {
-              float* rowp = a.token_scores + (((long long)pb * a.T + t) * kG + (qg & 3)) * ctx;
-              for (int r = 0; r < kBlock; ++r) rowp[pi * kBlock + r] = -INFINITY;
-            }
+            for (int w = 0; w < kIdxEpilogue; ++w) m = fmaxf(m, red[(xe * kIdxEpilogue + w) * NQ + col]);
+          }
+          a.block_scores[(((long long)pb * a.T + t) * kG + (qg & 3)) * a.max_pages + pi] =
+              m * a.score_scale;
+          if (pkind == kPageMasked && a.token_scores != nullptr) {
+            float* rowp = a.token_scores + (((long long)pb * a.T + t) * kG + (qg & 3)) * ctx;
+            for (int r = 0; r < kBlock; ++r) rowp[pi * kBlock + r] = -INFINITY;
           }
         }
-        __syncwarp();
-        if (lane == 0) cnt[xe] = 0;
       }
-      return true;
-    };
-
-    int cur_b = -1, qsel = 1, L = 0;
-    int pb = 0, pi = 0, pkind = kPageBad, pL = 0;   // the page one behind
-    for (int k = 0; k <= n; ++k) {
-      int nb = 0, ni = 0, nkind = kPageBad;
-      if (k < n) {
-        // ---- decode page k into the A operand in TMEM
-        const int s = k % kIdxRawStages;
-        if (!mbar_wait(&raw_full[s], (k / kIdxRawStages) & 1)) { report(a.flags, 5, 5); break; }
-        if (k >= 1 && !mbar_wait(a_empty, (k - 1) & 1)) { report(a.flags, 5, 4); break; }
-        tc_fence_after();
-        nb = meta[3 * s + 0];
-        ni = meta[3 * s + 1];
-        nkind = meta[3 * s + 2];
-        if (nb != cur_b) {
-          cur_b = nb;
-          L = a.seq_lens[nb];
-          qsel ^= 1;
-          // B operand: the query rows of this chunk for sequence nb, swizzled
-          // (its previous user, an MMA of page k-2 or earlier, has completed).
-          uint8_t* qb = qbuf + qsel * NQ * 128;
-          constexpr int kRowsPerWarp = NQ / kIdxWorkers;
-          for (int idx = lane; idx < kRowsPerWarp * 8; idx += 32) {
-            const int nrow = warp * kRowsPerWarp + idx / 8, c = idx % 8;
-            const int qg = qbase + nrow, t = qg >> 2;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < a.T)
-              v = *reinterpret_cast<const uint4*>(
-                  a.qi + (((long long)nb * a.T + t) * kG + (qg & 3)) * kDim + 16 * c);
-            sts128(qb + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
-          }
-          fence_async_smem();
+      __syncwarp();
+      // The accumulator (and, through the MMA order, this page's partial
+      // maxima and info slot) is released only after the combine: the MMA
+      // that refills it waits for all four arrivals, so red[xe] is not
+      // rewritten (page kk+2) before every warp has read it.
+      if (lane == 0) mbar_arrive(&acc_empty[xd]);
+    }
+  } else {
+    // ------------------------------------------------------------ decoders
+    const int quarter = warp & 3, half = warp >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);   // this warp's TMEM lanes
+    const int row = 32 * quarter + lane;                                  // key row of this thread
+    int cur_b = -1, cur_y = -1, qsel = 1, L = 0, ends = 0;
+    for (int k = 0; ends < 2; ++k) {
+      const int s = k % kIdxRawStages, ab = k & 1;
+      if (!mbar_wait(&raw_full[s], (k / kIdxRawStages) & 1)) { report(a.flags, 5, 5); break; }
+      if (k >= 2 && !mbar_wait(kND == 2 ? &acc_full[ab] : &a_empty[ab], ((k >> 1) - 1) & 1)) {
+        report(a.flags, 5, 4);
+        break;
+      }
+      tc_fence_after();
+      const int nb = meta[4 * s + 0], ni = meta[4 * s + 1], nkind = meta[4 * s + 2];
+      const int ny = meta[4 * s + 3];
+      ends += (nkind == kPageEnd);
+      if (nkind != kPageEnd && (nb != cur_b || ny != cur_y)) {
+        cur_b = nb;
+        cur_y = ny;
+        L = a.seq_lens[nb];
+        qsel ^= 1;
+        // B operand: the index queries of tile ny of sequence nb, swizzled
+        // (its previous user, an MMA of page k-2 or earlier, has completed:
+        // the wait above).
+        uint8_t* qb = qbuf + qsel * NQ * 128;
+        const int qbase = ny * NQ;
+        for (int idx = warp * 32 + lane; idx < NQ * 8; idx += kIdxDecoders * 32) {
+          const int nrow = idx / 8, c = idx % 8;
+          const int qg = qbase + nrow, t = qg >> 2;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (t < a.T)
+            v = *reinterpret_cast<const uint4*>(
+                a.qi + (((long long)nb * a.T + t) * kG + (qg & 3)) * kDim + 16 * c);
+          sts128(qb + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
         }
-        if (nkind == kPageLoad) {
-          const uint8_t* rs = raw + s * Ly.raw_stride;
-          if constexpr (FP8IDX) {
-            // 128-byte rows loaded with the 128-byte swizzle: chunk c of row r
-            // sits at chunk position c ^ (r % 8).
+        fence_async_smem();
+      }
+      if (nkind == kPageLoad) {
+        const uint8_t* rs = raw + s * Ly.raw_stride;
+        const uint32_t abase = lane_base + ab * kABufCols;
+        if constexpr (FP8IDX) {
+          // 128-byte rows loaded with the 128-byte swizzle: chunk c of row r
+          // sits at chunk position c ^ (r % 8).  This warp: dims 64h..64h+63.
 #pragma unroll
-            for (int c2 = 0; c2 < 4; ++c2) {
-              const uint4 x0 = lds128(rs + row * 128 + (((2 * c2) ^ (row & 7)) << 4));
-              const uint4 x1 = lds128(rs + row * 128 + (((2 * c2 + 1) ^ (row & 7)) << 4));
-              const uint32_t w8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-              tmem_st8(lane_base + 8 * c2, w8);
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c2 = 2 * half + cc;
+            const uint4 x0 = lds128(rs + row * 128 + (((2 * c2) ^ (row & 7)) << 4));
+            const uint4 x1 = lds128(rs + row * 128 + (((2 * c2 + 1) ^ (row & 7)) << 4));
+            const uint32_t w8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            tmem_st8(abase + 8 * c2, w8);
+          }
+        } else {
+          // 64-byte code rows loaded with the 64-byte swizzle: chunk c of
+          // row r sits at chunk position c ^ ((r / 2) % 4).  This warp:
+          // chunks 2h, 2h+1 (dims 64h..64h+63, block scales 4h..4h+3).
+          const uint32_t scw =
+              *reinterpret_cast<const uint32_t*>(rs + kPageCodes + row * kRowScales + 4 * half);
+          const int sw = (row >> 1) & 3;
+          // warp-uniform branch: tcgen05.st is a .sync.aligned warp instruction
+          if (__all_sync(0xffffffffu, (scw & 0x80808080u) == 0u)) {
+            // every block scale of the warp's 32 half rows is non-negative
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const int c = 2 * half + cc;
+              const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
+              const uint32_t sb = scw >> (16 * cc);                     // scales 2c, 2c+1
+              const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+              uint32_t pw[8], nw[8];
+              dq8_split_pos(w4.x, r0, pw[0], pw[1], nw[0], nw[1]);
+              dq8_split_pos(w4.y, r0, pw[2], pw[3], nw[2], nw[3]);
+              dq8_split_pos(w4.z, r1, pw[4], pw[5], nw[4], nw[5]);
+              dq8_split_pos(w4.w, r1, pw[6], pw[7], nw[6], nw[7]);
+              tmem_st8(abase + 8 * c, pw);
+              tmem_st8(abase + 32 + 8 * c, nw);
             }
           } else {
-            // 64-byte code rows loaded with the 64-byte swizzle: chunk c of
-            // row r sits at chunk position c ^ ((r / 2) % 4).
-            const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
-            const int sw = (row >> 1) & 3;
-            // warp-uniform branch: tcgen05.st is a .sync.aligned warp instruction
-            if (__all_sync(0xffffffffu, ((sc.x | sc.y) & 0x80808080u) == 0u)) {
-              // every block scale of the warp's 32 rows is non-negative
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-                const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));   // scales 2c, 2c+1
-                const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
-                uint32_t pw[8], nw[8];
-                dq8_split_pos(w4.x, r0, pw[0], pw[1], nw[0], nw[1]);
-                dq8_split_pos(w4.y, r0, pw[2], pw[3], nw[2], nw[3]);
-                dq8_split_pos(w4.z, r1, pw[4], pw[5], nw[4], nw[5]);
-                dq8_split_pos(w4.w, r1, pw[6], pw[7], nw[6], nw[7]);
-                tmem_st8(lane_base + 8 * c, pw);
-                tmem_st8(lane_base + 32 + 8 * c, nw);
-              }
-            } else {
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-                const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));
-                const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
-                const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
-                const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
-                const uint32_t f1 = (s1 & 0x80u) ? 0x88888888u : 0u;
-                uint32_t pw[8], nw[8];
-                dq8_split(w4.x, r0, f0, pw[0], pw[1], nw[0], nw[1]);
-                dq8_split(w4.y, r0, f0, pw[2], pw[3], nw[2], nw[3]);
-                dq8_split(w4.z, r1, f1, pw[4], pw[5], nw[4], nw[5]);
-                dq8_split(w4.w, r1, f1, pw[6], pw[7], nw[6], nw[7]);
-                tmem_st8(lane_base + 8 * c, pw);
-                tmem_st8(lane_base + 32 + 8 * c, nw);
-              }
+            for (int cc = 0; cc < 2; ++cc) {
+              const int c = 2 * half + cc;
+              const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
+              const uint32_t sb = scw >> (16 * cc);
+              const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
+              const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
+              const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
+              const uint32_t f1 = (s1 & 0x80u) ? 0x88888888u : 0u;
+              uint32_t pw[8], nw[8];
+              dq8_split(w4.x, r0, f0, pw[0], pw[1], nw[0], nw[1]);
+              dq8_split(w4.y, r0, f0, pw[2], pw[3], nw[2], nw[3]);
+              dq8_split(w4.z, r1, f1, pw[4], pw[5], nw[4], nw[5]);
+              dq8_split(w4.w, r1, f1, pw[6], pw[7], nw[6], nw[7]);
+              tmem_st8(abase + 8 * c, pw);
+              tmem_st8(abase + 32 + 8 * c, nw);
             }
           }
-          tmem_wait_st();
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&raw_empty[s]);
-          if (warp == 0) { tinfo[0] = (nkind != kPageLoad); tinfo[1] = qsel; }
-          mbar_arrive(a_full);
-        }
+        tmem_wait_st();
       }
-      // ---- epilogue of page k-1 (its MMA ran while page k was decoded)
-      if (k >= 1 && !epilogue(k - 1, pb, pi, pkind, pL)) break;
-      pb = nb; pi = ni; pkind = nkind; pL = L;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&raw_empty[s]);
+        if (warp == 0) {
+          tinfo[2 * ab] = nkind == kPageEnd ? 2 : (nkind != kPageLoad);
+          tinfo[2 * ab + 1] = qsel;
+          int* pf = pinfo + 8 * (k & 3);
+          pf[0] = nb; pf[1] = ni; pf[2] = nkind; pf[3] = L; pf[4] = ny;
+        }
+        mbar_arrive(&a_full[ab]);
+      }
     }
   }
 
@@ -478,11 +553,8 @@ static cudaError_t launch_nq(const IdxArgs& a, int num_sms, cudaStream_t st) {
   }
   const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), kIdxThreads, smem,
                                  pow2_at_least(kACols + (NQ <= 64 ? 2 : 1) * NQ));
-  const int gy = (kG * a.T + NQ - 1) / NQ;
-  const long long want = ((long long)num_sms * per_sm + gy - 1) / gy;
-  const long long cap = (long long)a.B * a.max_pages;
-  const int gx = (int)(want < 1 ? 1 : (want > cap ? cap : want));
-  kern<<<dim3(gx, gy), kIdxThreads, smem, st>>>(a);
+  const int gx = num_sms * per_sm;              // persistent: items are claimed in the kernel
+  kern<<<gx, kIdxThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 

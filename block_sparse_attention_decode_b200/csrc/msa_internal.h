@@ -11,8 +11,8 @@
 
 namespace msa {
 
-constexpr int kIdxThreads = 6 * 32;     // 4 workers, 1 producer, 1 MMA warp
-constexpr int kIdxRawStages = 4;         // raw index-key pages in flight per CTA
+constexpr int kIdxThreads = 18 * 32;    // 8 decoders, 8 epilogue warps, producer, MMA warp
+constexpr int kIdxRawStages = 6;         // raw index-key pages in flight per CTA
 
 struct IdxArgs {
   CUtensorMap tmap_idx;        // rows of idx_data: 64-byte rows (64B swizzle) or 128 (128B swizzle)
@@ -24,6 +24,7 @@ struct IdxArgs {
   float* token_scores;         // [B][T][4][max_pages*128] or null
   float* block_scores;         // [B][T][4][max_pages]
   Flags* flags;
+  int* work;                   // [2] in the workspace header: next item, CTAs done (0 on entry)
   float score_scale;           // s_qi * s_idx
   int B, T, max_pages, num_pages;
 };
