@@ -121,7 +121,15 @@ msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, flo
     cudaError_t e = cudaMemsetAsync(at<int>(ws, L.counters), 0, (size_t)rows * sizeof(int), st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
   }
+  // TMA row coordinates are 32-bit: (page * 4 + group) * 128 must fit
+  if ((long long)c->num_pages * MSA_KV_HEADS * MSA_BLOCK_TOKENS > 0x7FFFFFFFLL) return MSA_ERR_UNSUPPORTED;
   AttnArgs a{};
+  const uint64_t kv_rows = (uint64_t)c->num_pages * MSA_KV_HEADS * MSA_BLOCK_TOKENS;
+  if (!encode_row_tmap(&a.tmap_k, c->k_data, kv_rows, MSA_HEAD_DIM / 2) ||
+      !encode_row_tmap(&a.tmap_v, c->v_data, kv_rows, MSA_HEAD_DIM / 2) ||
+      !encode_row_tmap(&a.tmap_q, q, (uint64_t)rows * (MSA_Q_HEADS / MSA_KV_HEADS), MSA_HEAD_DIM,
+                       MSA_Q_HEADS / MSA_KV_HEADS))
+    return MSA_ERR_CUDA;
   a.k_data = c->k_data;
   a.k_scale = c->k_scale;
   a.v_data = c->v_data;
@@ -134,6 +142,7 @@ msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, flo
   a.partials = at<float>(ws, L.partials);
   a.counters = at<int>(ws, L.counters);
   a.flags = at<Flags>(ws, L.flags);
+  a.work = at<int>(ws, L.flags + kAttWorkOffset);
   a.logit_scale_log2 = (float)((double)softmax_scale * s_q * c->s_k * 1.4426950408889634);
   a.out_scale = c->s_v;
   a.B = s->batch;
@@ -141,7 +150,7 @@ msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, flo
   a.max_pages = s->max_pages;
   a.num_pages = c->num_pages;
   a.splits = L.splits;
-  return cuda_status(launch_attn(a, st));
+  return cuda_status(launch_attn(a, device_sms(), st));
 }
 
 }  // namespace
@@ -153,7 +162,8 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes) {
+bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes,
+                     uint32_t box_rows) {
   static EncodeTiledFn fn = nullptr;
   if (fn == nullptr) {
     void* p = nullptr;
@@ -165,10 +175,10 @@ bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t
     }
     fn = reinterpret_cast<EncodeTiledFn>(p);
   }
-  if (row_bytes != 64 && row_bytes != 128) return false;
+  if ((row_bytes != 64 && row_bytes != 128) || box_rows < 1 || box_rows > 256) return false;
   const cuuint64_t dims[2] = {row_bytes, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {row_bytes, (cuuint32_t)kBlock};
+  const cuuint32_t box[2] = {row_bytes, box_rows};
   const cuuint32_t estride[2] = {1, 1};
   const CUtensorMapSwizzle sw = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,

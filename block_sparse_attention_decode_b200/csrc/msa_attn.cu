@@ -1,370 +1,697 @@
 // msa_attn.cu -- exact attention over the selected blocks ([post, "MSA
 // primer"] and its Figure 1 caption: every query head of a GQA group attends
 // over that group's selected blocks) with NVFP4 K/V dequantised to E4M3 in
-// the kernel ([post, "NVIDIA Blackwell optimized MSA kernels"]).
+// the kernel and both contractions on the FP8 tensor core ([post, "NVIDIA
+// Blackwell optimized MSA kernels"]).
 // post = vLLM 為 MiniMax-M3.1-Flash 提供 Day-0 支援 (hot.atechcom.net).
 //
-// Work unit: one (sequence, query token, group) = 16 query heads = one m16
-// tile, split over its <= 16 selected blocks into `splits` CTAs.  A producer
-// warp gathers each selected block of the group's KV head through the page
-// table with four bulk async copies (K codes, K scales, V codes, V scales =
-// 18 KB) into a ring of stages; four consumer warps each take 32 keys of
-// every block.
+// Work item: one (sequence, query token, group) row -- its 16 query heads --
+// or, for small batches, one of `splits` slices of that row's selected
+// blocks.  Persistent CTAs (two per SM) claim items from a counter in the
+// workspace header and stream their blocks through a pipeline:
 //
-// Arithmetic: K and V are decoded to their E4M3 values (the FP8 operands the
-// method prescribes) and widened exactly to f16, and both contractions run on
-// f16 tensor-core MMA with fp32 accumulation (m16n8k16).  On sm_100a the
-// warp-level FP8 MMA is not native (it costs about twenty issue slots per
-// instruction, measured), while the f16 one is; the products of E4M3 values
-// are exact in either, so the result is the FP8 contraction's.
-//   S  = Q K^T   A = Q (f16 fragments staged once in shared memory),
-//                B = K decoded from the stage straight into fragments;
-//   online softmax in the exp2 domain, masked beyond the query position;
-//   O += P V     A = P (f16, from the S accumulators, FlashAttention-2
-//                layout), B = V decoded into a swizzled 16-key f16 tile and
-//                read transposed with ldmatrix.
-// The four warps' (m, l, O) merge in shared memory; with one split the CTA
-// writes bf16, otherwise it writes an fp32 partial and the last CTA of the
-// unit to finish (atomic counter, no waiting) combines the partials.
+//   warp 12 (producer): per item one TMA load of the 16 query rows (128-byte
+//     swizzle: the B operand of S); per block, through the page table, two
+//     tiled TMA loads of the K and V codes (64-byte swizzle) and two bulk
+//     copies of their scales into a ring of shared-memory stages;
+//   warps 0-7 (decoders): thread = key row, warp w decoding dims
+//     64(w/4)..64(w/4)+63 of rows 32(w%4)..32(w%4)+31.  K is decoded split
+//     by sign (K+ and K- magnitudes, as in the indexer) straight into tensor
+//     memory; V is decoded signed into shared memory as E4M3 rows of 128
+//     bytes with the 128-byte swizzle -- the A operand of O^T = V^T P^T in
+//     MN-major form;
+//   warp 13 (MMA, one thread): per block
+//       S^T[128 keys x 16 heads]  = K+ Q^T - K- Q^T   (8 MMAs, A from TMEM)
+//       O^T[128 dims x 32]       += V^T [P_hi | P_lo]^T  (4 MMAs, A and B in
+//                                   shared memory, both MN-major),
+//     issuing block k+1's S before block k's O so that the softmax of the
+//     next block overlaps the O update;
+//   warps 8-11 (softmax): warp 8+q reads the S^T lanes of quarter q (thread
+//     = key), masks keys after the query position, takes the per-head block
+//     maximum (warp reduction, then across the four warps through shared
+//     memory), and writes P = 2^(s*c - m + 4) split into two E4M3 terms
+//     (P_hi + P_lo holds P to about 2^-8 relative) as 16-byte rows per key.
+//     The running maximum m is raised lazily -- only when a block's maximum
+//     exceeds it by more than 2^4 -- so that P stays below 2^8 (inside E4M3)
+//     and O^T in tensor memory is rescaled rarely.  At the end of an item
+//     the same warps (thread = dim) read O^T, divide by the row sums and
+//     write bf16, or, with splits, an fp32 partial that the last CTA of the
+//     row combines (atomic counter, no waiting).
+// Every wait is a bounded mbarrier wait; on a timeout a thread records
+// MSA_ERR_TIMEOUT and leaves its loop, and TMEM is freed before exit.
 #include "msa_internal.h"
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 namespace msa {
 
-constexpr int kAttStageBytes = 2 * (kPageCodes + kPageScales);   // K + V of one KV head
-constexpr int kVtBytes = 16 * kDim * 2;                           // per warp: 16 keys x 128 f16
+constexpr int kAttDecoders = 8;
+constexpr int kAttSoftWarp0 = 8;            // softmax warps 8-11
+constexpr int kAttProducerWarp = 12;
+constexpr int kAttMmaWarp = 13;
+constexpr int kAttRawStride = 2 * (kPageCodes + kPageScales);   // 18432 = 18 x 1024
+constexpr int kAttTmemCols = 256;           // A[2] 0..127, S[2] 128..159, O[2] 160..223
+constexpr int kColA = 0, kColS = 128, kColO = 160;
+constexpr float kPExp = 4.f;                // P carries a factor 2^4 (E4M3 normal range)
+constexpr float kLazy = 4.f;                // raise m only when a block max exceeds it by 2^4
 
-size_t attn_smem_bytes() {
-  return (size_t)kAttStages * kAttStageBytes + kAttConsumers * kVtBytes + 8 * 32 * 16 +
-         256 * sizeof(uint2) + 2 * kAttStages * sizeof(uint64_t) + 4 * kTopk * sizeof(int) + 64;
+enum : int { kBlkLoad = 0, kBlkEmpty = 1, kBlkEnd = 2 };
+
+// Block info (producer -> decoders via the stage meta, decoders -> MMA and
+// softmax via a ring of 4): kind, block id, first, last, item sequence
+// number, row, split, query position.
+constexpr int kInfo = 8;
+
+struct AttLayout {
+  int raw, vbuf, pbuf, qbuf, lut, red, bc, lsum, bars, meta, binfo, tslot, misc, total;
+};
+
+__host__ __device__ inline AttLayout att_layout() {
+  AttLayout L;
+  int off = 0;
+  L.raw = off;   off += kAttStages * kAttRawStride;
+  L.vbuf = off;  off += 2 * kBlock * kDim;                 // V rows, E4M3, 128-byte swizzle
+  L.qbuf = off;  off += 2 * kHpg * kDim;                   // Q rows, E4M3, 128-byte swizzle
+  L.pbuf = off;  off += 2 * 2 * kBlock * kHpg;             // [2][hi, lo][key][16 heads]
+  L.lut = off;   off += 256 * 8;
+  L.red = off;   off += 2 * 4 * kHpg * 4;                  // block maxima [parity][quarter][16]
+  L.bc = off;    off += 4 * 2 * kHpg * 4;                  // per softmax warp: offsets, alphas
+  L.lsum = off;  off += 2 * 4 * kHpg * 4;                  // row sums [parity][quarter][16]
+  L.bars = off;  off += (2 * kAttStages + 16) * 8;
+  L.meta = off;  off += kAttStages * kInfo * 4;
+  L.binfo = off; off += 4 * kInfo * 4;
+  L.tslot = off; off += 16;
+  L.misc = off;  off += 16;
+  L.total = off + 1024;                                    // alignment slack
+  return L;
 }
 
-int attn_splits(long long units, int num_sms) {
+size_t attn_smem_bytes() { return (size_t)att_layout().total; }
+
+int attn_splits(long long rows, int num_sms) {
   int s = 1;
-  while (s < kTopk && units * s < 2LL * num_sms) s *= 2;
+  while (s < kTopk && rows * s < 4LL * num_sms) s *= 2;
   return s;
 }
 
-__global__ void __launch_bounds__(kAttThreads, 3) attn_kernel(AttnArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* stages = smem;
-  uint8_t* vt_all = smem + kAttStages * kAttStageBytes;                // [4 warps][16][256 B]
-  uint32_t* qfrag = reinterpret_cast<uint32_t*>(vt_all + kAttConsumers * kVtBytes);   // [8][32][4]
-  uint2* lut = reinterpret_cast<uint2*>(qfrag + 8 * 32 * 4);
-  uint64_t* full = reinterpret_cast<uint64_t*>(lut + 256);
-  uint64_t* empty = full + kAttStages;
-  int* list = reinterpret_cast<int*>(empty + kAttStages);   // [16] block ids
-  int* pages = list + kTopk;                                 // [16] page ids (-1 = bad)
-  int* misc = pages + kTopk;                                 // [0] = count, [1] = is_last
+// Signed NVFP4 -> E4M3 decode of 8 codes (element n in nibble n) with table
+// row r = lut[scale byte] (signed scales included): o0 = elements 0..3, o1 =
+// 4..7.  The magnitudes come from one prmt per 4 codes; the sign byte 0x80
+// of a negative code comes from a prmt with sign replication on a table of
+// 0x7F bytes (0x7F for a non-negative code, 0x00 for a negative one), plus 1
+// and inverted, and is xor-ed in (so a negative scale flips it back).
+__device__ __forceinline__ void dq8s(uint32_t w, uint2 r, uint32_t& o0, uint32_t& o1) {
+  const uint32_t mag = w & 0x77777777u;
+  const uint32_t s0 = prmt(0x7F7F7F7Fu, 0x7F7F7F7Fu, w);
+  const uint32_t s1 = prmt(0x7F7F7F7Fu, 0x7F7F7F7Fu, hi16(w));
+  o0 = prmt(r.x, r.y, mag) ^ (~(s0 + 0x01010101u) & 0x80808080u);
+  o1 = prmt(r.x, r.y, hi16(mag)) ^ (~(s1 + 0x01010101u) & 0x80808080u);
+}
+
+// Shared-memory descriptor, MN-major operand with the 128-byte swizzle: rows
+// of 128 bytes (128 M elements) per K index, 8-row atoms `sbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t addr, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(16384 >> 4) << 16) |
+         ((uint64_t)(sbo >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Shared-memory descriptor, MN-major operand without swizzle: core matrices
+// of 8 K rows x 16 bytes (128 contiguous bytes), `lbo` bytes apart along K
+// and `sbo` bytes apart along N.
+__device__ __forceinline__ uint64_t desc_mn_plain(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
+         ((uint64_t)(sbo >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
+// D[tmem] (+)= A[smem] * B[smem] (E4M3), one K = 32 slice.
+__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Split x (0 <= x <= 256) into hi + lo with hi holding 4 significant bits
+// (Veltkamp's splitting with the factor 2^20 + 1 for a 24-bit significand);
+// both are then exact or rounded once as E4M3.
+__device__ __forceinline__ void split4(float x, float& hi, float& lo) {
+  const float c = __fmul_rn(1048577.f, x);
+  hi = __fsub_rn(c, __fsub_rn(c, x));
+  lo = __fsub_rn(x, hi);
+}
+
+// 2^x with the SFU's approximate exp2 (relative error below 2^-22).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t fp8x2(float a, float b) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+__global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_constant__ AttnArgs a) {
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
+  const AttLayout Ly = att_layout();
+  uint8_t* raw = smem + Ly.raw;
+  uint8_t* vbuf = smem + Ly.vbuf;
+  uint8_t* qbuf = smem + Ly.qbuf;
+  uint8_t* pbuf = smem + Ly.pbuf;
+  uint2* lut = reinterpret_cast<uint2*>(smem + Ly.lut);
+  float* red = reinterpret_cast<float*>(smem + Ly.red);
+  float* bc = reinterpret_cast<float*>(smem + Ly.bc);
+  float* lsum = reinterpret_cast<float*>(smem + Ly.lsum);
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + Ly.bars);
+  uint64_t* raw_empty = raw_full + kAttStages;
+  uint64_t* q_full = raw_empty + kAttStages;     // [2] producer (TMA) -> MMA
+  uint64_t* q_empty = q_full + 2;                // [2] MMA -> producer
+  uint64_t* kv_full = q_empty + 2;               // [2] decoders -> MMA
+  uint64_t* s_full = kv_full + 2;                // [2] MMA -> softmax
+  uint64_t* p_full = s_full + 2;                 // [2] softmax -> MMA
+  uint64_t* pv_done = p_full + 2;                // [2] MMA -> decoders, softmax
+  uint64_t* o_free = pv_done + 2;                // [2] softmax -> MMA
+  uint64_t* red_full = o_free + 2;               // [1] softmax rendezvous
+  uint64_t* misc_bar = red_full + 1;             // [1] softmax rendezvous (item end)
+  int* meta = reinterpret_cast<int*>(smem + Ly.meta);
+  int* binfo = reinterpret_cast<int*>(smem + Ly.binfo);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
+  int* misc = reinterpret_cast<int*>(smem + Ly.misc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  const long long unit = blockIdx.x / a.splits;
-  const int sp = blockIdx.x % a.splits;
-  const int b = (int)(unit / (kG * a.T));
-  const int t = (int)((unit / kG) % a.T);
-  const int g = (int)(unit % kG);
-  const int L = a.seq_lens[b];
-  const bool len_ok = L >= a.T && L <= a.max_pages * kBlock;
-  const int pos = L - a.T + t;
+  const long long rows = (long long)a.B * a.T * kG;
+  const long long items = rows * a.splits;
 
   build_nvfp4_lut(lut, tid, blockDim.x);
   if (tid == 0) {
-    for (int s = 0; s < kAttStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kAttConsumers); }
-    mbar_fence_init();
-    int cnt = 0;
-    if (!len_ok) {
-      if (sp == 0 && g == 0 && t == 0) report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
-    } else {
-      const int nvis = pos / kBlock + 1;
-      const int k0 = kTopk * sp / a.splits, k1 = kTopk * (sp + 1) / a.splits;
-      for (int k = k0; k < k1; ++k) {
-        const int blk = a.sel[unit * kTopk + k];
-        if (blk < 0) continue;
-        if (blk >= nvis) { report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, blk); continue; }
-        const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + blk]
-                                         : (long long)b * a.max_pages + blk;
-        if (p < 0 || p >= a.num_pages) { report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)p); continue; }
-        list[cnt] = blk;
-        pages[cnt] = (int)p;
-        ++cnt;
-      }
+    for (int s = 0; s < kAttStages; ++s) {
+      mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], kAttDecoders);
     }
-    misc[0] = cnt;
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&kv_full[x], kAttDecoders);
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 4);
+      mbar_init(&pv_done[x], 1);
+      mbar_init(&o_free[x], 4);
+    }
+    mbar_init(red_full, 4);
+    mbar_init(misc_bar, 4);
+    mbar_fence_init();
   }
+  if (warp == kAttMmaWarp) {
+    tmem_alloc(tslot, kAttTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  const int nlist = misc[0];
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
 
-  // per-warp softmax state for heads 16g+gid (row 0) and 16g+gid+8 (row 1)
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-  float o[16][4];
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-
-  if (warp == kAttConsumers) {
+  if (warp == kAttProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      for (int k = 0; k < nlist; ++k) {
+      int k = 0, ki = 0;            // block slot, item sequence number
+      bool ok = true;
+      auto slot = [&](int kk) -> bool {
+        return kk < kAttStages ||
+               mbar_wait(&raw_empty[kk % kAttStages], ((kk / kAttStages) - 1) & 1);
+      };
+      auto emit = [&](int kind, int blk, int first, int last, long long row, int sp, int pos,
+                      long long page, int g) -> bool {
+        if (!slot(k)) { report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 20); return false; }
         const int s = k % kAttStages;
-        if (k >= kAttStages && !mbar_wait(&empty[s], ((k / kAttStages) - 1) & 1)) {
-          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, k);
+        int* m = meta + s * kInfo;
+        m[0] = kind; m[1] = blk; m[2] = first; m[3] = last;
+        m[4] = ki; m[5] = (int)row; m[6] = sp; m[7] = pos;
+        if (kind == kBlkLoad) {
+          uint8_t* dst = raw + s * kAttRawStride;
+          const long long r0 = (page * kG + g) * kBlock;      // first (page, head, token) row
+          mbar_expect_tx(&raw_full[s], kAttRawStride);
+          tma_load_2d(dst, &a.tmap_k, 0, (int)r0, &raw_full[s]);
+          tma_load_2d(dst + kPageCodes, &a.tmap_v, 0, (int)r0, &raw_full[s]);
+          bulk_g2s(dst + 2 * kPageCodes, a.k_scale + r0 * kRowScales, kPageScales, &raw_full[s]);
+          bulk_g2s(dst + 2 * kPageCodes + kPageScales, a.v_scale + r0 * kRowScales, kPageScales,
+                   &raw_full[s]);
+        } else {
+          mbar_arrive(&raw_full[s]);
+        }
+        ++k;
+        return true;
+      };
+      long long item = atomicAdd(&a.work[0], 1);
+      while (item < items && ok) {
+        const long long nxt = atomicAdd(&a.work[0], 1);   // claimed early: latency overlaps
+        const long long row = item / a.splits;
+        const int sp = (int)(item % a.splits);
+        const int b = (int)(row / (kG * a.T));
+        const int t = (int)((row / kG) % a.T);
+        const int g = (int)(row % kG);
+        const int L = a.seq_lens[b];
+        const bool len_ok = L >= a.T && L <= a.max_pages * kBlock;
+        const int pos = L - a.T + t;
+        const int nvis = pos / kBlock + 1;
+        const int k0 = kTopk * sp / a.splits, k1 = kTopk * (sp + 1) / a.splits;
+        if (!len_ok && sp == 0 && g == 0 && t == 0) report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
+        // pass 1: the valid blocks of this slice (ids in order, pages)
+        int nval = 0, lastk = -1;
+        if (len_ok) {
+          for (int kk = k0; kk < k1; ++kk) {
+            const int blk = a.sel[row * kTopk + kk];
+            if (blk < 0) continue;
+            if (blk >= nvis) { report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, blk); continue; }
+            const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + blk]
+                                             : (long long)b * a.max_pages + blk;
+            if (p < 0 || p >= a.num_pages) { report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)p); continue; }
+            ++nval;
+            lastk = kk;
+          }
+        }
+        // the query rows of this item (previous user: item ki-2's last S MMA)
+        const int qs = ki & 1;
+        if (ki >= 2 && !mbar_wait(&q_empty[qs], ((ki >> 1) - 1) & 1)) {
+          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 21);
+          ok = false;
           break;
         }
-        const long long row0 = ((long long)pages[k] * kG + g) * kBlock;   // first (page, head, token) row
-        uint8_t* dst = stages + s * kAttStageBytes;
-        mbar_expect_tx(&full[s], kAttStageBytes);
-        bulk_g2s(dst, a.k_data + row0 * kRowCodes, kPageCodes, &full[s]);
-        bulk_g2s(dst + kPageCodes, a.k_scale + row0 * kRowScales, kPageScales, &full[s]);
-        bulk_g2s(dst + kPageCodes + kPageScales, a.v_data + row0 * kRowCodes, kPageCodes, &full[s]);
-        bulk_g2s(dst + 2 * kPageCodes + kPageScales, a.v_scale + row0 * kRowScales, kPageScales,
-                 &full[s]);
+        if (nval > 0) {
+          mbar_expect_tx(&q_full[qs], kHpg * kDim);
+          tma_load_2d(qbuf + qs * kHpg * kDim, &a.tmap_q, 0,
+                      (int)(((long long)b * a.T + t) * kHq + kHpg * g), &q_full[qs]);
+        } else {
+          mbar_arrive(&q_full[qs]);   // keeps the phase count; nothing waits on it
+        }
+        // pass 2: emit
+        if (nval == 0) {
+          ok = emit(kBlkEmpty, 0, 1, 1, row, sp, pos, 0, g);
+        } else {
+          int e = 0;
+          for (int kk = k0; kk < k1 && ok; ++kk) {
+            const int blk = a.sel[row * kTopk + kk];
+            if (blk < 0 || blk >= nvis) continue;
+            const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + blk]
+                                             : (long long)b * a.max_pages + blk;
+            if (p < 0 || p >= a.num_pages) continue;
+            ok = emit(kBlkLoad, blk, e == 0, kk == lastk, row, sp, pos, p, g);
+            ++e;
+          }
+        }
+        ++ki;
+        item = nxt;
+      }
+      if (ok) emit(kBlkEnd, 0, 0, 0, 0, 0, 0, 0, 0);
+      // every CTA has made its last claim once all have arrived here
+      __threadfence();
+      if (atomicAdd(&a.work[1], 1) == (int)gridDim.x - 1) {
+        atomicExch(&a.work[0], 0);
+        atomicExch(&a.work[1], 0);
       }
     }
-  } else {
-    // ------------------------------------------------------------ consumers
-    // Q A-fragments (f16), k-step ks: a0/a1 = rows gid/gid+8, dims
-    // 32tig+4ks+{0,1}; a2/a3 = dims 32tig+4ks+{2,3}.  Staged once by warp 0.
-    if (warp == 0) {
-      uint32_t w[2][8];
+  } else if (warp == kAttMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_e4m3_f32(128, kHpg);
+      constexpr uint32_t idesc_sn = idesc_s | (1u << 13);                       // negate A
+      constexpr uint32_t idesc_o = idesc_e4m3_f32(128, 2 * kHpg) | (1u << 15) | (1u << 16);
+      const uint64_t qd[2] = {desc_kmajor_sw128(smem_u32(qbuf)),
+                              desc_kmajor_sw128(smem_u32(qbuf + kHpg * kDim))};
+      // S for block k; returns its kind (-1 on a timeout)
+      auto issue_s = [&](int k) -> int {
+        const int x = k & 1;
+        if (!mbar_wait(&kv_full[x], (k >> 1) & 1)) { report(a.flags, 5, 22); return -1; }
+        tc_fence_after();
+        const int* bi = binfo + (k & 3) * kInfo;
+        const int kind = bi[0], first = bi[2], last = bi[3], ki = bi[4];
+        if (kind == kBlkLoad) {
+          if (first && !mbar_wait(&q_full[ki & 1], (ki >> 1) & 1)) { report(a.flags, 5, 23); return -1; }
+          const uint32_t d = tmem + kColS + kHpg * x;
+          const uint32_t ta = tmem + kColA + 64 * x;
+          const uint64_t bd = qd[ki & 1];
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int h = g * kHpg + gid + 8 * r;
-        const uint8_t* src = a.q + (((long long)b * a.T + t) * kHq + h) * kDim + 32 * tig;
-        const uint4 x0 = *reinterpret_cast<const uint4*>(src);
-        const uint4 x1 = *reinterpret_cast<const uint4*>(src + 16);
-        w[r][0] = x0.x; w[r][1] = x0.y; w[r][2] = x0.z; w[r][3] = x0.w;
-        w[r][4] = x1.x; w[r][5] = x1.y; w[r][6] = x1.z; w[r][7] = x1.w;
+          for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc_s, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 32 + 8 * kk, bd + 2 * kk, idesc_sn, 1);
+        }
+        tc_commit(&s_full[x]);
+        if (kind != kBlkEnd && last) tc_commit(&q_empty[ki & 1]);
+        return kind;
+      };
+      // O update for block k
+      auto issue_o = [&](int k) -> bool {
+        const int x = k & 1;
+        if (!mbar_wait(&p_full[x], (k >> 1) & 1)) { report(a.flags, 5, 24); return false; }
+        tc_fence_after();
+        const int* bi = binfo + (k & 3) * kInfo;
+        const int kind = bi[0], first = bi[2], ki = bi[4];
+        const int ob = ki & 1;
+        if (first && ki >= 2 && !mbar_wait(&o_free[ob], ((ki >> 1) - 1) & 1)) {
+          report(a.flags, 5, 25);
+          return false;
+        }
+        tc_fence_after();
+        if (kind == kBlkLoad) {
+          const uint32_t d = tmem + kColO + 2 * kHpg * ob;
+          const uint32_t va = smem_u32(vbuf + x * kBlock * kDim);
+          const uint32_t pa = smem_u32(pbuf + x * 2 * kBlock * kHpg);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // 32 keys per slice
+            tc_mma_ss(d, desc_mn_sw128(va + kk * 32 * kDim, 1024),
+                      desc_mn_plain(pa + kk * 32 * kHpg, 8 * kHpg, kBlock * kHpg), idesc_o,
+                      (first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(&pv_done[x]);
+        return true;
+      };
+      int kind = issue_s(0);
+      for (int k = 0; kind >= 0 && kind != kBlkEnd; ++k) {
+        const int next = issue_s(k + 1);
+        if (!issue_o(k)) break;
+        kind = next;
       }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        *reinterpret_cast<uint4*>(&qfrag[(ks * 32 + lane) * 4]) =
-            make_uint4(e4m3x2_to_f16x2(w[0][ks]), e4m3x2_to_f16x2(w[1][ks]),
-                       e4m3x2_to_f16x2(w[0][ks] >> 16), e4m3x2_to_f16x2(w[1][ks] >> 16));
     }
-    asm volatile("bar.sync 1, %0;\n" ::"n"(kAttConsumers * 32) : "memory");
-    uint8_t* vt = vt_all + warp * kVtBytes;     // this warp's 16-key f16 V tile
-    const float sc = a.logit_scale_log2;
-    for (int k = 0; k < nlist; ++k) {
-      const int s = k % kAttStages;
-      if (!mbar_wait(&full[s], (k / kAttStages) & 1)) {
-        report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, k);
-        break;
-      }
-      const uint8_t* kc = stages + s * kAttStageBytes;
-      const uint8_t* ks_ = kc + kPageCodes;
-      const uint8_t* vc = ks_ + kPageScales;
-      const uint8_t* vs = vc + kPageCodes;
-      const int key0 = list[k] * kBlock + 32 * warp;   // global position of this warp's key 0
-
-      // ---- S = Q K^T over this warp's 32 keys (n-tile j = keys 8j..8j+7)
-      float sacc[4][4];
+  } else if (warp >= kAttSoftWarp0) {
+    // ------------------------------------------------------------ softmax
+    const int q = warp & 3;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    const float c = a.logit_scale_log2;               // softmax_scale * s_q * s_k * log2(e)
+    float* mybc = bc + q * 2 * kHpg;                  // this warp's broadcast slot
+    float lt[kHpg];                                   // this key lane's share of the row sums
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
-        const int kk = 32 * warp + 8 * j + gid;
-        uint32_t kw[8];
-        dq32(lut, lds128(kc + kk * kRowCodes + 16 * tig), lds16(ks_ + kk * kRowScales + 2 * tig), kw);
+    for (int h = 0; h < kHpg; ++h) lt[h] = 0.f;
+    float m_used = -INFINITY;                         // lanes 0-15: running max of head `lane`
+    int nred = 0, nmisc = 0, nitem = 0;
+    for (int k = 0;; ++k) {
+      const int x = k & 1;
+      if (!mbar_wait(&s_full[x], (k >> 1) & 1)) { report(a.flags, 5, 26); break; }
+      tc_fence_after();
+      const int* bi = binfo + (k & 3) * kInfo;
+      const int kind = bi[0], blk = bi[1], first = bi[2], last = bi[3], ki = bi[4];
+      const long long row = bi[5];
+      const int sp = bi[6], pos = bi[7];
+      if (kind == kBlkEnd) break;
+      const int ob = ki & 1;
+      if (k >= 2 && !mbar_wait(&pv_done[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 27); break; }
+      if (kind == kBlkLoad) {
+        float s[kHpg];
+        tmem_ld16(lane_base + kColS + kHpg * x, s);
+        tmem_wait_ld();
+        if (blk * kBlock + 32 * q + lane > pos) {      // key after the query position
 #pragma unroll
-        for (int st = 0; st < 8; ++st) {
-          const uint4 qa = *reinterpret_cast<const uint4*>(&qfrag[(st * 32 + lane) * 4]);
-          mma_f16(sacc[j], qa.x, qa.y, qa.z, qa.w, e4m3x2_to_f16x2(kw[st]),
-                  e4m3x2_to_f16x2(kw[st] >> 16));
+          for (int h = 0; h < kHpg; ++h) s[h] = -INFINITY;
         }
-      }
-
-      // ---- mask, online softmax (exp2 domain)
-      float mb[2] = {-INFINITY, -INFINITY};
+        // block maximum per head: this warp's 32 keys, then the four warps
+        float* rq = red + ((nred & 1) * 4 + q) * kHpg;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = key0 + 8 * j + 2 * tig + (e & 1);
-          float v = sacc[j][e] * sc;
-          if (key > pos) v = -INFINITY;
-          sacc[j][e] = v;
-          mb[e >> 1] = fmaxf(mb[e >> 1], v);
-        }
-      }
-      float alpha[2], mu[2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        mb[r] = fmaxf(mb[r], __shfl_xor_sync(0xffffffffu, mb[r], 1));
-        mb[r] = fmaxf(mb[r], __shfl_xor_sync(0xffffffffu, mb[r], 2));
-        const float m_new = fmaxf(m_run[r], mb[r]);
-        mu[r] = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[r] = exp2f(m_run[r] - mu[r]);
-        m_run[r] = m_new;
-      }
-      float ps[2] = {0.f, 0.f};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p = exp2f(sacc[j][e] - mu[e >> 1]);
-          sacc[j][e] = p;
-          ps[e >> 1] += p;
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 2; ++r) l_run[r] = l_run[r] * alpha[r] + ps[r];
-      if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          o[nt][0] *= alpha[0]; o[nt][1] *= alpha[0];
-          o[nt][2] *= alpha[1]; o[nt][3] *= alpha[1];
-        }
-      }
-
-      // ---- O += P V, 16 keys at a time (PV k-step kk = S n-tiles 2kk, 2kk+1)
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        const uint32_t pa0 = f32x2_to_f16x2(sacc[2 * kk][0], sacc[2 * kk][1]);
-        const uint32_t pa1 = f32x2_to_f16x2(sacc[2 * kk][2], sacc[2 * kk][3]);
-        const uint32_t pa2 = f32x2_to_f16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
-        const uint32_t pa3 = f32x2_to_f16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
-        // V tile: rows = the 16 keys 32w+16kk+0..15 (256 B of f16 each);
-        // 16-byte chunk c of row r at chunk position c ^ (r % 8).
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          const int r = 8 * p + gid, vk = 32 * warp + 16 * kk + r;
-          uint32_t vw[8];
-          dq32(lut, lds128(vc + vk * kRowCodes + 16 * tig), lds16(vs + vk * kRowScales + 2 * tig), vw);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)   // dims 32tig + 8i .. +7 = chunk 4tig + i
-            *reinterpret_cast<uint4*>(vt + r * 256 + (((4 * tig + i) ^ (r & 7)) << 4)) =
-                make_uint4(e4m3x2_to_f16x2(vw[2 * i]), e4m3x2_to_f16x2(vw[2 * i] >> 16),
-                           e4m3x2_to_f16x2(vw[2 * i + 1]), e4m3x2_to_f16x2(vw[2 * i + 1] >> 16));
+        for (int h = 0; h < kHpg; ++h) {
+          const float mh = warp_max(s[h]);
+          if (lane == h) rq[h] = mh;
         }
         __syncwarp();
-        // ldmatrix.x4.trans: matrix mi (lanes 8mi..8mi+7) = keys 8(mi&1)..+7 x dims 16n2+8(mi>>1)..+7
-        const int mi = lane >> 3, lr = (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-        for (int n2 = 0; n2 < 8; ++n2) {
-          const int chunk = 2 * n2 + (mi >> 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_trans(vt + lr * 256 + ((chunk ^ (lr & 7)) << 4), b0, b1, b2, b3);
-          mma_f16(o[2 * n2], pa0, pa1, pa2, pa3, b0, b1);
-          mma_f16(o[2 * n2 + 1], pa0, pa1, pa2, pa3, b2, b3);
+        if (lane == 0) mbar_arrive(red_full);
+        if (!mbar_wait(red_full, nred & 1)) { report(a.flags, 5, 28); break; }
+        int resc = 0;
+        if (lane < kHpg) {
+          const float* rr = red + (nred & 1) * 4 * kHpg + lane;
+          const float mb = fmaxf(fmaxf(rr[0], rr[kHpg]), fmaxf(rr[2 * kHpg], rr[3 * kHpg]));
+          float alpha = 1.f;
+          if (first) {
+            m_used = mb;
+          } else if ((mb - m_used) * c > kLazy) {
+            alpha = ex2((m_used - mb) * c);
+            m_used = mb;
+            resc = 1;
+          }
+          mybc[lane] = m_used * c - kPExp;               // exponent offset of head `lane`
+          mybc[kHpg + lane] = alpha;
         }
-        __syncwarp();   // the tile is rewritten by the next 16 keys
-      }
-      if (lane == 0) mbar_arrive(&empty[s]);   // stage no longer read by this warp
-    }
-    // full row sums: add the 4 lanes of a row
+        ++nred;
+        resc = __any_sync(0xffffffffu, resc);
+        __syncwarp();
+        if (resc) {   // raise m: rescale the row sums and O^T (after block k-1's update)
+          const float* al = mybc + kHpg;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
-      l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+          for (int h = 0; h < kHpg; ++h) lt[h] *= al[h];
+          if (!mbar_wait(&pv_done[x ^ 1], ((k - 1) >> 1) & 1)) { report(a.flags, 5, 29); break; }
+          tc_fence_after();
+          const uint32_t oa = lane_base + kColO + 2 * kHpg * ob;
+#pragma unroll 1
+          for (int j = 0; j < 4; ++j) {   // columns 8j..8j+7 = heads (8j..8j+7) % 16
+            float o8[8];
+            tmem_ld8(oa + 8 * j, o8);
+            tmem_wait_ld();
+            uint32_t w8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(o8[i] * al[(8 * j + i) & 15]);
+            tmem_st8(oa + 8 * j, w8);
+          }
+          tmem_wait_st();
+        }
+        // P = 2^(s c - m c + 4) as hi + lo E4M3, one 16-byte row per key
+        uint32_t ph[4], pl[4];
+#pragma unroll
+        for (int h2 = 0; h2 < kHpg / 2; ++h2) {
+          const float2 mo = *reinterpret_cast<const float2*>(mybc + 2 * h2);   // exponent offsets
+          const float p0 = ex2(fmaf(s[2 * h2], c, -mo.x));
+          const float p1 = ex2(fmaf(s[2 * h2 + 1], c, -mo.y));
+          lt[2 * h2] += p0;
+          lt[2 * h2 + 1] += p1;
+          float h0, l0, h1, l1;
+          split4(p0, h0, l0);
+          split4(p1, h1, l1);
+          const uint32_t hw = fp8x2(h0, h1), lw = fp8x2(l0, l1);
+          if (h2 & 1) { ph[h2 >> 1] |= hw << 16; pl[h2 >> 1] |= lw << 16; }
+          else { ph[h2 >> 1] = hw; pl[h2 >> 1] = lw; }
+        }
+        uint8_t* pb = pbuf + x * 2 * kBlock * kHpg + (32 * q + lane) * kHpg;
+        *reinterpret_cast<uint4*>(pb) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(pb + kBlock * kHpg) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        fence_async_smem();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[x]);
+      if (!last) continue;
+
+      // ---------------------------------------------------- end of the item
+      // row sums: this warp's 32 keys, then the four warps
+      if (kind == kBlkLoad) {
+        if (!mbar_wait(&pv_done[x], (k >> 1) & 1)) { report(a.flags, 5, 30); break; }
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int h = 0; h < kHpg; ++h) {
+        float v = lt[h];
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        if (lane == h) lsum[((nitem & 1) * 4 + q) * kHpg + h] = v;
+        lt[h] = 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(misc_bar);
+      if (!mbar_wait(misc_bar, (nmisc++) & 1)) { report(a.flags, 5, 31); break; }
+      const float* ls = lsum + (nitem & 1) * 4 * kHpg;   // [quarter][16] row sums
+      // m of this item (lanes 0-15 hold head `lane`), in log2 units
+      const float mc = m_used * c;
+      const int d = 32 * q + lane;                     // this thread's dimension
+      const int b = (int)(row / (kG * a.T));
+      const int t = (int)((row / kG) % a.T);
+      const int g = (int)(row % kG);
+      // O = O_hi + O_lo of heads 8j..8j+7, then release O^T
+      float o[kHpg];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float hi8[8], lo8[8];
+        if (kind == kBlkLoad) {
+          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + 8 * j, hi8);
+          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + kHpg + 8 * j, lo8);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) hi8[i] = lo8[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[8 * j + i] = hi8[i] + lo8[i];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[ob]);
+      if (a.splits == 1) {
+        uint16_t* dst = a.out + (((long long)b * a.T + t) * kHq + kHpg * g) * kDim + d;
+#pragma unroll
+        for (int h = 0; h < kHpg; ++h) {
+          const float l = ls[h] + ls[kHpg + h] + ls[2 * kHpg + h] + ls[3 * kHpg + h];
+          const float v = l > 0.f ? o[h] * (a.out_scale / l) : 0.f;
+          const __nv_bfloat16 bv = __float2bfloat16_rn(v);
+          dst[(long long)h * kDim] = *reinterpret_cast<const uint16_t*>(&bv);
+        }
+      } else {
+        // fp32 partial of this split: O (in units of 2^4 P), m (log2 units), l
+        float* part = a.partials + (row * a.splits + sp) * kPartialFloats;
+#pragma unroll
+        for (int h = 0; h < kHpg; ++h) part[h * kDim + d] = o[h];
+        if (q == 0 && lane < kHpg) {
+          part[kHpg * kDim + lane] = kind == kBlkLoad ? mc : -INFINITY;
+          part[kHpg * kDim + kHpg + lane] =
+              ls[lane] + ls[kHpg + lane] + ls[2 * kHpg + lane] + ls[3 * kHpg + lane];
+        }
+        // all four warps' partials written and fenced, then one thread counts
+        // this split in; the result reaches the four warps through shared memory
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(misc_bar);
+        if (!mbar_wait(misc_bar, (nmisc++) & 1)) { report(a.flags, 5, 32); break; }
+        if (q == 0 && lane == 0) misc[nitem & 1] = (atomicAdd(&a.counters[row], 1) == a.splits - 1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(misc_bar);
+        if (!mbar_wait(misc_bar, (nmisc++) & 1)) { report(a.flags, 5, 35); break; }
+        if (misc[nitem & 1]) {
+          __threadfence();
+          // 128 threads: head hr = tid'/8, 16 dims from (tid'%8)*16
+          const int tq = 32 * q + lane, hr = tq >> 3, d0 = (tq & 7) * 16;
+          const float* base = a.partials + row * a.splits * kPartialFloats;
+          float Mx = -INFINITY;
+          for (int s2 = 0; s2 < a.splits; ++s2)
+            Mx = fmaxf(Mx, __ldcg(base + s2 * kPartialFloats + kHpg * kDim + hr));
+          const float Mu = (Mx == -INFINITY) ? 0.f : Mx;
+          float tot[16];
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) tot[cc] = 0.f;
+          float Lt = 0.f;
+          for (int s2 = 0; s2 < a.splits; ++s2) {
+            const float* ps2 = base + s2 * kPartialFloats;
+            const float f = exp2f(__ldcg(ps2 + kHpg * kDim + hr) - Mu);
+            Lt += __ldcg(ps2 + kHpg * kDim + kHpg + hr) * f;
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) tot[cc] += __ldcg(ps2 + hr * kDim + d0 + cc) * f;
+          }
+          const float inv = Lt > 0.f ? a.out_scale / Lt : 0.f;
+          uint32_t packed[8];
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(tot[2 * cc] * inv, tot[2 * cc + 1] * inv);
+            packed[cc] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(
+              a.out + (((long long)b * a.T + t) * kHq + kHpg * g + hr) * kDim + d0);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          if (tq == 0) a.counters[row] = 0;   // ready for the next call
+        }
+      }
+      ++nitem;
+      m_used = -INFINITY;
+    }
+  } else {
+    // ------------------------------------------------------------ decoders
+    const int quarter = warp & 3, half = warp >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
+    const int row = 32 * quarter + lane;             // key row of this thread
+    const int sw = (row >> 1) & 3;                   // 64-byte swizzle of the code rows
+    for (int k = 0;; ++k) {
+      const int s = k % kAttStages, x = k & 1;
+      if (!mbar_wait(&raw_full[s], (k / kAttStages) & 1)) { report(a.flags, 5, 33); break; }
+      if (k >= 2 && !mbar_wait(&pv_done[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 34); break; }
+      tc_fence_after();
+      const int* m = meta + s * kInfo;
+      const int kind = m[0];
+      if (kind == kBlkLoad) {
+        const uint8_t* rs = raw + s * kAttRawStride;
+        const uint8_t* kc = rs;
+        const uint8_t* vc = rs + kPageCodes;
+        const uint8_t* ks = rs + 2 * kPageCodes;
+        const uint8_t* vs = ks + kPageScales;
+        // K: dims 64h..64h+63 split by sign into A[x] (K+ cols 0-31, K- 32-63)
+        const uint32_t abase = lane_base + kColA + 64 * x;
+        const uint32_t kscw = *reinterpret_cast<const uint32_t*>(ks + row * kRowScales + 4 * half);
+        if (__all_sync(0xffffffffu, (kscw & 0x80808080u) == 0u)) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int cix = 2 * half + cc;
+            const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
+            const uint32_t sb = kscw >> (16 * cc);
+            const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+            uint32_t pw[8], nw[8];
+            dq8_split_pos(w4.x, r0, pw[0], pw[1], nw[0], nw[1]);
+            dq8_split_pos(w4.y, r0, pw[2], pw[3], nw[2], nw[3]);
+            dq8_split_pos(w4.z, r1, pw[4], pw[5], nw[4], nw[5]);
+            dq8_split_pos(w4.w, r1, pw[6], pw[7], nw[6], nw[7]);
+            tmem_st8(abase + 8 * cix, pw);
+            tmem_st8(abase + 32 + 8 * cix, nw);
+          }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int cix = 2 * half + cc;
+            const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
+            const uint32_t sb = kscw >> (16 * cc);
+            const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
+            const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
+            const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
+            const uint32_t f1 = (s1 & 0x80u) ? 0x88888888u : 0u;
+            uint32_t pw[8], nw[8];
+            dq8_split(w4.x, r0, f0, pw[0], pw[1], nw[0], nw[1]);
+            dq8_split(w4.y, r0, f0, pw[2], pw[3], nw[2], nw[3]);
+            dq8_split(w4.z, r1, f1, pw[4], pw[5], nw[4], nw[5]);
+            dq8_split(w4.w, r1, f1, pw[6], pw[7], nw[6], nw[7]);
+            tmem_st8(abase + 8 * cix, pw);
+            tmem_st8(abase + 32 + 8 * cix, nw);
+          }
+        }
+        // V: dims 64h..64h+63 signed, as E4M3 into the 128-byte V row of this
+        // key (16-byte chunk j at chunk position j ^ (key % 8))
+        const uint32_t vscw = *reinterpret_cast<const uint32_t*>(vs + row * kRowScales + 4 * half);
+        uint8_t* vrow = vbuf + x * kBlock * kDim + row * kDim;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int cix = 2 * half + cc;
+          const uint4 w4 = lds128(vc + row * kRowCodes + ((cix ^ sw) << 4));
+          const uint32_t sb = vscw >> (16 * cc);
+          const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+          uint32_t o[8];
+          dq8s(w4.x, r0, o[0], o[1]);
+          dq8s(w4.y, r0, o[2], o[3]);
+          dq8s(w4.z, r1, o[4], o[5]);
+          dq8s(w4.w, r1, o[6], o[7]);
+          // code chunk cix = dims 32cix..32cix+31 = V chunks 2cix, 2cix+1
+          *reinterpret_cast<uint4*>(vrow + (((2 * cix) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(vrow + (((2 * cix + 1) ^ (row & 7)) << 4)) =
+              make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        tmem_wait_st();
+        fence_async_smem();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&raw_empty[s]);
+        if (warp == 0) {
+          int* bi = binfo + (k & 3) * kInfo;
+#pragma unroll
+          for (int i = 0; i < kInfo; ++i) bi[i] = m[i];
+        }
+        mbar_arrive(&kv_full[x]);
+      }
+      if (kind == kBlkEnd) break;
     }
   }
 
-  // ---------------------------------------------- merge the 4 warps' states
-  __syncthreads();   // all stages consumed: reuse the stage ring as scratch
-  float* ow = reinterpret_cast<float*>(stages);                // [4][16][128]
-  float* mw = ow + kAttConsumers * kHpg * kDim;                // [4][16]
-  float* lw = mw + kAttConsumers * kHpg;                       // [4][16]
-  if (warp < kAttConsumers) {
-    if (tig == 0) {
-      mw[warp * kHpg + gid] = m_run[0];
-      mw[warp * kHpg + gid + 8] = m_run[1];
-      lw[warp * kHpg + gid] = l_run[0];
-      lw[warp * kHpg + gid + 8] = l_run[1];
-    }
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      float* r0 = ow + (warp * kHpg + gid) * kDim + 8 * nt + 2 * tig;
-      float* r1 = r0 + 8 * kDim;
-      r0[0] = o[nt][0]; r0[1] = o[nt][1];
-      r1[0] = o[nt][2]; r1[1] = o[nt][3];
-    }
-  }
+  // ---- teardown: every role leaves its loop (normally or on a timeout)
+  tc_fence_before();
   __syncthreads();
-  // 128 threads: thread -> head row tid/8, 16 dims starting at (tid%8)*16
-  const int hr = tid >> 3, d0 = (tid & 7) * 16;
-  float acc[16];
-  float M = -INFINITY, Lsum = 0.f;
-  if (tid < 128) {
-#pragma unroll
-    for (int w = 0; w < kAttConsumers; ++w) M = fmaxf(M, mw[w * kHpg + hr]);
-    const float Mu = (M == -INFINITY) ? 0.f : M;
-#pragma unroll
-    for (int c = 0; c < 16; ++c) acc[c] = 0.f;
-#pragma unroll
-    for (int w = 0; w < kAttConsumers; ++w) {
-      const float f = exp2f(mw[w * kHpg + hr] - Mu);
-      Lsum += lw[w * kHpg + hr] * f;
-      const float* src = ow + (w * kHpg + hr) * kDim + d0;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) acc[c] += src[c] * f;
-    }
-  }
-  const int h = g * kHpg + hr;
-  uint16_t* dst = a.out + (((long long)b * a.T + t) * kHq + h) * kDim + d0;
-  if (a.splits == 1) {
-    if (tid < 128) {
-      const float inv = Lsum > 0.f ? a.out_scale / Lsum : 0.f;
-      uint32_t packed[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * c] * inv, acc[2 * c + 1] * inv);
-        packed[c] = *reinterpret_cast<const uint32_t*>(&v);
-      }
-      reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-    }
-    return;
-  }
-  // split-K: write this CTA's partial, the last CTA of the unit combines
-  float* part = a.partials + ((long long)unit * a.splits + sp) * kPartialFloats;
-  if (tid < 128) {
-#pragma unroll
-    for (int c = 0; c < 16; ++c) part[hr * kDim + d0 + c] = acc[c];
-    if ((tid & 7) == 0) {
-      part[kHpg * kDim + hr] = M;
-      part[kHpg * kDim + kHpg + hr] = Lsum;
-    }
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int prev = atomicAdd(&a.counters[unit], 1);
-    misc[1] = (prev == a.splits - 1);
-  }
-  __syncthreads();
-  if (!misc[1]) return;
-  __threadfence();
-  if (tid < 128) {
-    const float* base = a.partials + (long long)unit * a.splits * kPartialFloats;
-    float Mx = -INFINITY;
-    for (int s2 = 0; s2 < a.splits; ++s2)
-      Mx = fmaxf(Mx, __ldcg(base + s2 * kPartialFloats + kHpg * kDim + hr));
-    const float Mu = (Mx == -INFINITY) ? 0.f : Mx;
-    float tot[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) tot[c] = 0.f;
-    float Lt = 0.f;
-    for (int s2 = 0; s2 < a.splits; ++s2) {
-      const float* ps2 = base + s2 * kPartialFloats;
-      const float f = exp2f(__ldcg(ps2 + kHpg * kDim + hr) - Mu);
-      Lt += __ldcg(ps2 + kHpg * kDim + kHpg + hr) * f;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) tot[c] += __ldcg(ps2 + hr * kDim + d0 + c) * f;
-    }
-    const float inv = Lt > 0.f ? a.out_scale / Lt : 0.f;
-    uint32_t packed[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const __nv_bfloat162 v = __floats2bfloat162_rn(tot[2 * c] * inv, tot[2 * c + 1] * inv);
-      packed[c] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-    reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-  }
-  if (tid == 0) a.counters[unit] = 0;   // ready for the next call
+  tc_fence_after();
+  if (warp == kAttMmaWarp) tmem_dealloc(tmem, kAttTmemCols);
 }
 
-cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_attn(const AttnArgs& a, int num_sms, cudaStream_t st) {
   const size_t smem = attn_smem_bytes();
   static bool configured = false;
   if (!configured) {
@@ -373,14 +700,15 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const long long units = (long long)a.B * a.T * kG;
-  const long long grid = units * a.splits;
-  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  attn_kernel<<<(unsigned)grid, kAttThreads, smem, st>>>(a);
+  const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(attn_kernel), kAttThreads, smem,
+                                 kAttTmemCols);
+  attn_kernel<<<num_sms * per_sm, kAttThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 // ----------------------------------------------------- parity debug hook --
+// The kernels' NVFP4 -> E4M3 table through the signed decode the V operand
+// uses (dq8s): out[s*16 + c] for scale byte s and code c.
 __global__ void nvfp4_table_kernel(uint8_t* out) {
   __shared__ uint2 lut[256];
   build_nvfp4_lut(lut, threadIdx.x, blockDim.x);
@@ -388,8 +716,8 @@ __global__ void nvfp4_table_kernel(uint8_t* out) {
   const int s = threadIdx.x;   // 256 threads, one scale byte each
   const uint2 r = lut[s];
   uint32_t o[4];
-  dq8(0x76543210u, r, o[0], o[1]);   // codes 0..7 in element order
-  dq8(0xFEDCBA98u, r, o[2], o[3]);   // codes 8..15
+  dq8s(0x76543210u, r, o[0], o[1]);   // codes 0..7 in element order
+  dq8s(0xFEDCBA98u, r, o[2], o[3]);   // codes 8..15
   uint4* dst = reinterpret_cast<uint4*>(out + s * 16);
   *dst = make_uint4(o[0], o[1], o[2], o[3]);
 }

@@ -40,7 +40,8 @@ int ctas_per_sm(const void* kernel, int threads, size_t smem, int tmem_cols);
 
 // Encode a tensor map over `rows` rows of `row_bytes` (64 or 128) bytes with
 // 128-row boxes and the matching shared-memory swizzle.  False on failure.
-bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes);
+bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes,
+                     uint32_t box_rows = kBlock);
 
 // Top-k over block scores of every (b, t, g) row.
 cudaError_t launch_topk(const float* block_scores, const int32_t* seq_lens, int B, int T,
@@ -49,12 +50,14 @@ cudaError_t launch_topk(const float* block_scores, const int32_t* seq_lens, int 
 cudaError_t launch_maxpool(const float* token_scores, const int32_t* seq_lens, int B, int T,
                            int max_pages, float* block_scores, Flags* flags, cudaStream_t st);
 
-constexpr int kAttConsumers = 4;
-constexpr int kAttThreads = (kAttConsumers + 1) * 32;
-constexpr int kAttStages = 2;
+constexpr int kAttThreads = 14 * 32;    // 8 decoders, 4 softmax warps, producer, MMA warp
+constexpr int kAttStages = 3;            // raw K/V blocks in flight per CTA
+constexpr int kAttWorkOffset = 72;       // int[2] in the workspace header (see kWorkOffset)
 constexpr int kPartialFloats = kHpg * kDim + 2 * kHpg;   // O[16][128], m[16], l[16]
 
 struct AttnArgs {
+  CUtensorMap tmap_k, tmap_v;  // K / V code rows [P*4*128][64 B], 64-byte swizzle, 128-row boxes
+  CUtensorMap tmap_q;          // query rows [B*T*64][128 B], 128-byte swizzle, 16-row boxes
   const uint8_t *k_data, *k_scale, *v_data, *v_scale;
   const int32_t* page_table;
   const int32_t* seq_lens;
@@ -64,14 +67,15 @@ struct AttnArgs {
   float* partials;             // [units][splits][kPartialFloats]
   int* counters;               // [units]
   Flags* flags;
+  int* work;                   // [2] in the workspace header: next item, CTAs done (0 on entry)
   float logit_scale_log2;      // softmax_scale * s_q * s_k * log2(e)
   float out_scale;             // s_v
   int B, T, max_pages, num_pages, splits;
 };
 
 size_t attn_smem_bytes();
-int attn_splits(long long units, int num_sms);
-cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
+int attn_splits(long long rows, int num_sms);
+cudaError_t launch_attn(const AttnArgs& a, int num_sms, cudaStream_t st);
 
 // The kernels' NVFP4 -> E4M3 table for all (scale, code) pairs.
 cudaError_t launch_nvfp4_table(uint8_t* out, cudaStream_t st);

@@ -272,8 +272,9 @@ def test_repeat_calls_reuse_workspace():
     o1, s1 = run_decode(w, ws)
     o2, s2 = run_decode(w, ws)
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
-    # the indexer's work counters (workspace header bytes 64..71) are back at 0
-    assert ws[64:72].view(torch.int32).tolist() == [0, 0]
+    # the indexer's and the attention's work counters (workspace header
+    # bytes 64..79) are back at 0
+    assert ws[64:80].view(torch.int32).tolist() == [0, 0, 0, 0]
 
 
 # ---------------------------------------------------------- boundaries -----
