@@ -55,6 +55,7 @@ constexpr int kAttTmemCols = 256;           // A[2] 0..127, S[2] 128..159, O[2] 
 constexpr int kColA = 0, kColS = 128, kColO = 160;
 constexpr float kPExp = 4.f;                // P carries a factor 2^4 (E4M3 normal range)
 constexpr float kLazy = 4.f;                // raise m only when a block max exceeds it by 2^4
+constexpr int kVB = 3;                      // V and P buffers (blocks between decode and O update)
 
 enum : int { kBlkLoad = 0, kBlkEmpty = 1, kBlkEnd = 2 };
 
@@ -71,14 +72,14 @@ __host__ __device__ inline AttLayout att_layout() {
   AttLayout L;
   int off = 0;
   L.raw = off;   off += kAttStages * kAttRawStride;
-  L.vbuf = off;  off += 2 * kBlock * kDim;                 // V rows, E4M3, 128-byte swizzle
+  L.vbuf = off;  off += kVB * kBlock * kDim;               // V rows, E4M3, 128-byte swizzle
   L.qbuf = off;  off += 2 * kHpg * kDim;                   // Q rows, E4M3, 128-byte swizzle
-  L.pbuf = off;  off += 2 * 2 * kBlock * kHpg;             // [2][hi, lo][key][16 heads]
+  L.pbuf = off;  off += kVB * 2 * kBlock * kHpg;           // [kVB][hi, lo][key][16 heads]
   L.lut = off;   off += 256 * 8;
   L.red = off;   off += 2 * 4 * kHpg * 4;                  // block maxima [parity][quarter][16]
   L.bc = off;    off += 4 * 2 * kHpg * 4;                  // per softmax warp: offsets, alphas
   L.lsum = off;  off += 2 * 4 * kHpg * 4;                  // row sums [parity][quarter][16]
-  L.bars = off;  off += (2 * kAttStages + 16) * 8;
+  L.bars = off;  off += (2 * kAttStages + 17) * 8;
   L.meta = off;  off += kAttStages * kInfo * 4;
   L.binfo = off; off += 4 * kInfo * 4;
   L.tslot = off; off += 16;
@@ -173,8 +174,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   uint64_t* kv_full = q_empty + 2;               // [2] decoders -> MMA
   uint64_t* s_full = kv_full + 2;                // [2] MMA -> softmax
   uint64_t* p_full = s_full + 2;                 // [2] softmax -> MMA
-  uint64_t* pv_done = p_full + 2;                // [2] MMA -> decoders, softmax
-  uint64_t* o_free = pv_done + 2;                // [2] softmax -> MMA
+  uint64_t* pv_done = p_full + 2;                // [kVB] MMA -> decoders, softmax
+  uint64_t* o_free = pv_done + kVB;              // [2] softmax -> MMA
   uint64_t* red_full = o_free + 2;               // [1] softmax rendezvous
   uint64_t* misc_bar = red_full + 1;             // [1] softmax rendezvous (item end)
   int* meta = reinterpret_cast<int*>(smem + Ly.meta);
@@ -198,9 +199,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       mbar_init(&kv_full[x], kAttDecoders);
       mbar_init(&s_full[x], 1);
       mbar_init(&p_full[x], 4);
-      mbar_init(&pv_done[x], 1);
       mbar_init(&o_free[x], 4);
     }
+    for (int x = 0; x < kVB; ++x) mbar_init(&pv_done[x], 1);
     mbar_init(red_full, 4);
     mbar_init(misc_bar, 4);
     mbar_fence_init();
@@ -357,15 +358,15 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         tc_fence_after();
         if (kind == kBlkLoad) {
           const uint32_t d = tmem + kColO + 2 * kHpg * ob;
-          const uint32_t va = smem_u32(vbuf + x * kBlock * kDim);
-          const uint32_t pa = smem_u32(pbuf + x * 2 * kBlock * kHpg);
+          const uint32_t va = smem_u32(vbuf + (k % kVB) * kBlock * kDim);
+          const uint32_t pa = smem_u32(pbuf + (k % kVB) * 2 * kBlock * kHpg);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)   // 32 keys per slice
             tc_mma_ss(d, desc_mn_sw128(va + kk * 32 * kDim, 1024),
                       desc_mn_plain(pa + kk * 32 * kHpg, 8 * kHpg, kBlock * kHpg), idesc_o,
                       (first && kk == 0) ? 0u : 1u);
         }
-        tc_commit(&pv_done[x]);
+        tc_commit(&pv_done[k % kVB]);
         return true;
       };
       int kind = issue_s(0);
@@ -396,7 +397,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       const int sp = bi[6], pos = bi[7];
       if (kind == kBlkEnd) break;
       const int ob = ki & 1;
-      if (k >= 2 && !mbar_wait(&pv_done[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 27); break; }
+      const int vb = k % kVB;                          // P buffer (its last reader: block k-3's O)
+      if (k >= kVB && !mbar_wait(&pv_done[vb], ((k / kVB) - 1) & 1)) { report(a.flags, 5, 27); break; }
       if (kind == kBlkLoad) {
         float s[kHpg];
         tmem_ld16(lane_base + kColS + kHpg * x, s);
@@ -437,7 +439,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           const float* al = mybc + kHpg;
 #pragma unroll
           for (int h = 0; h < kHpg; ++h) lt[h] *= al[h];
-          if (!mbar_wait(&pv_done[x ^ 1], ((k - 1) >> 1) & 1)) { report(a.flags, 5, 29); break; }
+          if (!mbar_wait(&pv_done[(k - 1) % kVB], ((k - 1) / kVB) & 1)) { report(a.flags, 5, 29); break; }
           tc_fence_after();
           const uint32_t oa = lane_base + kColO + 2 * kHpg * ob;
 #pragma unroll 1
@@ -468,7 +470,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           if (h2 & 1) { ph[h2 >> 1] |= hw << 16; pl[h2 >> 1] |= lw << 16; }
           else { ph[h2 >> 1] = hw; pl[h2 >> 1] = lw; }
         }
-        uint8_t* pb = pbuf + x * 2 * kBlock * kHpg + (32 * q + lane) * kHpg;
+        uint8_t* pb = pbuf + vb * 2 * kBlock * kHpg + (32 * q + lane) * kHpg;
         *reinterpret_cast<uint4*>(pb) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
         *reinterpret_cast<uint4*>(pb + kBlock * kHpg) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
         fence_async_smem();
@@ -481,7 +483,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       // ---------------------------------------------------- end of the item
       // row sums: this warp's 32 keys, then the four warps
       if (kind == kBlkLoad) {
-        if (!mbar_wait(&pv_done[x], (k >> 1) & 1)) { report(a.flags, 5, 30); break; }
+        if (!mbar_wait(&pv_done[vb], (k / kVB) & 1)) { report(a.flags, 5, 30); break; }
         tc_fence_after();
       }
 #pragma unroll
@@ -599,7 +601,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     for (int k = 0;; ++k) {
       const int s = k % kAttStages, x = k & 1;
       if (!mbar_wait(&raw_full[s], (k / kAttStages) & 1)) { report(a.flags, 5, 33); break; }
-      if (k >= 2 && !mbar_wait(&pv_done[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 34); break; }
+      // A[x] was last read by block k-2's S; V buffer k % kVB by block k-3's O
+      if (k >= 2 && !mbar_wait(&s_full[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 34); break; }
+      if (k >= kVB && !mbar_wait(&pv_done[k % kVB], ((k / kVB) - 1) & 1)) { report(a.flags, 5, 36); break; }
       tc_fence_after();
       const int* m = meta + s * kInfo;
       const int kind = m[0];
@@ -649,7 +653,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         // V: dims 64h..64h+63 signed, as E4M3 into the 128-byte V row of this
         // key (16-byte chunk j at chunk position j ^ (key % 8))
         const uint32_t vscw = *reinterpret_cast<const uint32_t*>(vs + row * kRowScales + 4 * half);
-        uint8_t* vrow = vbuf + x * kBlock * kDim + row * kDim;
+        uint8_t* vrow = vbuf + (k % kVB) * kBlock * kDim + row * kDim;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int cix = 2 * half + cc;
@@ -672,12 +676,14 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&raw_empty[s]);
+        // the block info leaves the stage before the stage is released (the
+        // producer rewrites it for block k + kAttStages right after)
         if (warp == 0) {
           int* bi = binfo + (k & 3) * kInfo;
 #pragma unroll
           for (int i = 0; i < kInfo; ++i) bi[i] = m[i];
         }
+        mbar_arrive(&raw_empty[s]);
         mbar_arrive(&kv_full[x]);
       }
       if (kind == kBlkEnd) break;

@@ -51,7 +51,7 @@ cudaError_t launch_maxpool(const float* token_scores, const int32_t* seq_lens, i
                            int max_pages, float* block_scores, Flags* flags, cudaStream_t st);
 
 constexpr int kAttThreads = 14 * 32;    // 8 decoders, 4 softmax warps, producer, MMA warp
-constexpr int kAttStages = 3;            // raw K/V blocks in flight per CTA
+constexpr int kAttStages = 2;            // raw K/V blocks in flight per CTA
 constexpr int kAttWorkOffset = 72;       // int[2] in the workspace header (see kWorkOffset)
 constexpr int kPartialFloats = kHpg * kDim + 2 * kHpg;   // O[16][128], m[16], l[16]
 
