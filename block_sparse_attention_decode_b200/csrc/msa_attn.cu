@@ -14,8 +14,8 @@
 //     swizzle: the B operand of S); per block, through the page table, two
 //     tiled TMA loads of the K and V codes (64-byte swizzle) and two bulk
 //     copies of their scales into a ring of shared-memory stages;
-//   warps 0-7 (decoders): thread = key row, warp w decoding dims
-//     64(w/4)..64(w/4)+63 of rows 32(w%4)..32(w%4)+31.  K is decoded split
+//   warps 0-3 (decoders): thread = key row, warp w decoding rows
+//     32w..32w+31.  K is decoded split
 //     by sign (K+ and K- magnitudes, as in the indexer) straight into tensor
 //     memory; V is decoded signed into shared memory as E4M3 rows of 128
 //     bytes with the 128-byte swizzle -- the A operand of O^T = V^T P^T in
@@ -26,10 +26,11 @@
 //                                   shared memory, both MN-major),
 //     issuing block k+1's S before block k's O so that the softmax of the
 //     next block overlaps the O update;
-//   warps 8-11 (softmax): warp 8+q reads the S^T lanes of quarter q (thread
-//     = key), masks keys after the query position, takes the per-head block
-//     maximum (warp reduction, then across the four warps through shared
-//     memory), and writes P = 2^(s*c - m + 4) split into two E4M3 terms
+//   warps 4-11 (softmax): warp 4+4j+q reads heads 8j..8j+7 of the S^T lanes
+//     of quarter q (thread = key), masks keys after the query position,
+//     takes the per-head block maximum (warp reduction, then across the four
+//     quarters through shared memory), and writes P = 2^(s*c - m + 4) split
+//     into two E4M3 terms
 //     (P_hi + P_lo holds P to about 2^-8 relative) as 16-byte rows per key.
 //     The running maximum m is raised lazily -- only when a block's maximum
 //     exceeds it by more than 2^4 -- so that P stays below 2^8 (inside E4M3)
@@ -46,8 +47,10 @@
 
 namespace msa {
 
-constexpr int kAttDecoders = 8;
-constexpr int kAttSoftWarp0 = 8;            // softmax warps 8-11
+constexpr int kAttDecoders = 4;             // warps 0-3, one per TMEM lane quarter
+constexpr int kAttSoftWarp0 = 4;            // softmax warps 4-11: two per lane quarter
+constexpr int kAttSoft = 8;
+constexpr int kHh = kHpg / 2;               // heads per softmax warp
 constexpr int kAttProducerWarp = 12;
 constexpr int kAttMmaWarp = 13;
 constexpr int kAttRawStride = 2 * (kPageCodes + kPageScales);   // 18432 = 18 x 1024
@@ -77,7 +80,7 @@ __host__ __device__ inline AttLayout att_layout() {
   L.pbuf = off;  off += kVB * 2 * kBlock * kHpg;           // [kVB][hi, lo][key][16 heads]
   L.lut = off;   off += 256 * 8;
   L.red = off;   off += 2 * 4 * kHpg * 4;                  // block maxima [parity][quarter][16]
-  L.bc = off;    off += 4 * 2 * kHpg * 4;                  // per softmax warp: offsets, alphas
+  L.bc = off;    off += kAttSoft * 2 * kHh * 4;            // per softmax warp: offsets, alphas
   L.lsum = off;  off += 2 * 4 * kHpg * 4;                  // row sums [parity][quarter][16]
   L.bars = off;  off += (2 * kAttStages + 17) * 8;
   L.meta = off;  off += kAttStages * kInfo * 4;
@@ -198,12 +201,12 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       mbar_init(&q_empty[x], 1);
       mbar_init(&kv_full[x], kAttDecoders);
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 4);
-      mbar_init(&o_free[x], 4);
+      mbar_init(&p_full[x], kAttSoft);
+      mbar_init(&o_free[x], kAttSoft);
     }
     for (int x = 0; x < kVB; ++x) mbar_init(&pv_done[x], 1);
-    mbar_init(red_full, 4);
-    mbar_init(misc_bar, 4);
+    mbar_init(red_full, kAttSoft);
+    mbar_init(misc_bar, kAttSoft);
     mbar_fence_init();
   }
   if (warp == kAttMmaWarp) {
@@ -378,14 +381,15 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     }
   } else if (warp >= kAttSoftWarp0) {
     // ------------------------------------------------------------ softmax
-    const int q = warp & 3;
+    // warp 4 + 4*hh + q: keys (TMEM lanes) 32q..32q+31, heads 8hh..8hh+7
+    const int q = warp & 3, hh = (warp - kAttSoftWarp0) >> 2, h0 = kHh * hh;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     const float c = a.logit_scale_log2;               // softmax_scale * s_q * s_k * log2(e)
-    float* mybc = bc + q * 2 * kHpg;                  // this warp's broadcast slot
-    float lt[kHpg];                                   // this key lane's share of the row sums
+    float* mybc = bc + (warp - kAttSoftWarp0) * 2 * kHh;   // this warp's broadcast slot
+    float lt[kHh];                                    // this key lane's share of the row sums
 #pragma unroll
-    for (int h = 0; h < kHpg; ++h) lt[h] = 0.f;
-    float m_used = -INFINITY;                         // lanes 0-15: running max of head `lane`
+    for (int h = 0; h < kHh; ++h) lt[h] = 0.f;
+    float m_used = -INFINITY;                         // lanes 0-7: running max of head h0+lane
     int nred = 0, nmisc = 0, nitem = 0;
     for (int k = 0;; ++k) {
       const int x = k & 1;
@@ -400,17 +404,17 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       const int vb = k % kVB;                          // P buffer (its last reader: block k-3's O)
       if (k >= kVB && !mbar_wait(&pv_done[vb], ((k / kVB) - 1) & 1)) { report(a.flags, 5, 27); break; }
       if (kind == kBlkLoad) {
-        float s[kHpg];
-        tmem_ld16(lane_base + kColS + kHpg * x, s);
+        float s[kHh];
+        tmem_ld8(lane_base + kColS + kHpg * x + h0, s);
         tmem_wait_ld();
         if (blk * kBlock + 32 * q + lane > pos) {      // key after the query position
 #pragma unroll
-          for (int h = 0; h < kHpg; ++h) s[h] = -INFINITY;
+          for (int h = 0; h < kHh; ++h) s[h] = -INFINITY;
         }
-        // block maximum per head: this warp's 32 keys, then the four warps
-        float* rq = red + ((nred & 1) * 4 + q) * kHpg;
+        // block maximum per head: this warp's 32 keys, then the four quarters
+        float* rq = red + ((nred & 1) * 4 + q) * kHpg + h0;
 #pragma unroll
-        for (int h = 0; h < kHpg; ++h) {
+        for (int h = 0; h < kHh; ++h) {
           const float mh = warp_max(s[h]);
           if (lane == h) rq[h] = mh;
         }
@@ -418,8 +422,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         if (lane == 0) mbar_arrive(red_full);
         if (!mbar_wait(red_full, nred & 1)) { report(a.flags, 5, 28); break; }
         int resc = 0;
-        if (lane < kHpg) {
-          const float* rr = red + (nred & 1) * 4 * kHpg + lane;
+        if (lane < kHh) {
+          const float* rr = red + (nred & 1) * 4 * kHpg + h0 + lane;
           const float mb = fmaxf(fmaxf(rr[0], rr[kHpg]), fmaxf(rr[2 * kHpg], rr[3 * kHpg]));
           float alpha = 1.f;
           if (first) {
@@ -429,50 +433,50 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
             m_used = mb;
             resc = 1;
           }
-          mybc[lane] = m_used * c - kPExp;               // exponent offset of head `lane`
-          mybc[kHpg + lane] = alpha;
+          mybc[lane] = m_used * c - kPExp;               // exponent offset of head h0+lane
+          mybc[kHh + lane] = alpha;
         }
         ++nred;
         resc = __any_sync(0xffffffffu, resc);
         __syncwarp();
         if (resc) {   // raise m: rescale the row sums and O^T (after block k-1's update)
-          const float* al = mybc + kHpg;
+          const float* al = mybc + kHh;
 #pragma unroll
-          for (int h = 0; h < kHpg; ++h) lt[h] *= al[h];
+          for (int h = 0; h < kHh; ++h) lt[h] *= al[h];
           if (!mbar_wait(&pv_done[(k - 1) % kVB], ((k - 1) / kVB) & 1)) { report(a.flags, 5, 29); break; }
           tc_fence_after();
-          const uint32_t oa = lane_base + kColO + 2 * kHpg * ob;
+          const uint32_t oa = lane_base + kColO + 2 * kHpg * ob + h0;
 #pragma unroll 1
-          for (int j = 0; j < 4; ++j) {   // columns 8j..8j+7 = heads (8j..8j+7) % 16
+          for (int j = 0; j < 2; ++j) {   // the hi and the lo columns of heads h0..h0+7
             float o8[8];
-            tmem_ld8(oa + 8 * j, o8);
+            tmem_ld8(oa + kHpg * j, o8);
             tmem_wait_ld();
             uint32_t w8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(o8[i] * al[(8 * j + i) & 15]);
-            tmem_st8(oa + 8 * j, w8);
+            for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(o8[i] * al[i]);
+            tmem_st8(oa + kHpg * j, w8);
           }
           tmem_wait_st();
         }
-        // P = 2^(s c - m c + 4) as hi + lo E4M3, one 16-byte row per key
-        uint32_t ph[4], pl[4];
+        // P = 2^(s c - m c + 4) as hi + lo E4M3: bytes h0..h0+7 of the key's rows
+        uint32_t ph[2], pl[2];
 #pragma unroll
-        for (int h2 = 0; h2 < kHpg / 2; ++h2) {
+        for (int h2 = 0; h2 < kHh / 2; ++h2) {
           const float2 mo = *reinterpret_cast<const float2*>(mybc + 2 * h2);   // exponent offsets
           const float p0 = ex2(fmaf(s[2 * h2], c, -mo.x));
           const float p1 = ex2(fmaf(s[2 * h2 + 1], c, -mo.y));
           lt[2 * h2] += p0;
           lt[2 * h2 + 1] += p1;
-          float h0, l0, h1, l1;
-          split4(p0, h0, l0);
-          split4(p1, h1, l1);
-          const uint32_t hw = fp8x2(h0, h1), lw = fp8x2(l0, l1);
+          float a0, b0, a1, b1;
+          split4(p0, a0, b0);
+          split4(p1, a1, b1);
+          const uint32_t hw = fp8x2(a0, a1), lw = fp8x2(b0, b1);
           if (h2 & 1) { ph[h2 >> 1] |= hw << 16; pl[h2 >> 1] |= lw << 16; }
           else { ph[h2 >> 1] = hw; pl[h2 >> 1] = lw; }
         }
-        uint8_t* pb = pbuf + vb * 2 * kBlock * kHpg + (32 * q + lane) * kHpg;
-        *reinterpret_cast<uint4*>(pb) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-        *reinterpret_cast<uint4*>(pb + kBlock * kHpg) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        uint8_t* pb = pbuf + vb * 2 * kBlock * kHpg + (32 * q + lane) * kHpg + h0;
+        *reinterpret_cast<uint2*>(pb) = make_uint2(ph[0], ph[1]);
+        *reinterpret_cast<uint2*>(pb + kBlock * kHpg) = make_uint2(pl[0], pl[1]);
         fence_async_smem();
       }
       tc_fence_before();
@@ -481,55 +485,53 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       if (!last) continue;
 
       // ---------------------------------------------------- end of the item
-      // row sums: this warp's 32 keys, then the four warps
+      // row sums: this warp's 32 keys, then the four quarters
       if (kind == kBlkLoad) {
         if (!mbar_wait(&pv_done[vb], (k / kVB) & 1)) { report(a.flags, 5, 30); break; }
         tc_fence_after();
       }
 #pragma unroll
-      for (int h = 0; h < kHpg; ++h) {
+      for (int h = 0; h < kHh; ++h) {
         float v = lt[h];
         v += __shfl_xor_sync(0xffffffffu, v, 16);
         v += __shfl_xor_sync(0xffffffffu, v, 8);
         v += __shfl_xor_sync(0xffffffffu, v, 4);
         v += __shfl_xor_sync(0xffffffffu, v, 2);
         v += __shfl_xor_sync(0xffffffffu, v, 1);
-        if (lane == h) lsum[((nitem & 1) * 4 + q) * kHpg + h] = v;
+        if (lane == h) lsum[((nitem & 1) * 4 + q) * kHpg + h0 + h] = v;
         lt[h] = 0.f;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(misc_bar);
       if (!mbar_wait(misc_bar, (nmisc++) & 1)) { report(a.flags, 5, 31); break; }
-      const float* ls = lsum + (nitem & 1) * 4 * kHpg;   // [quarter][16] row sums
-      // m of this item (lanes 0-15 hold head `lane`), in log2 units
-      const float mc = m_used * c;
+      const float* ls = lsum + (nitem & 1) * 4 * kHpg + h0;   // [quarter][16] row sums
+      const float mc = m_used * c;                     // lanes 0-7: m of head h0+lane, log2 units
       const int d = 32 * q + lane;                     // this thread's dimension
       const int b = (int)(row / (kG * a.T));
       const int t = (int)((row / kG) % a.T);
       const int g = (int)(row % kG);
-      // O = O_hi + O_lo of heads 8j..8j+7, then release O^T
-      float o[kHpg];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      // O = O_hi + O_lo of heads h0..h0+7, then release O^T
+      float o[kHh];
+      {
         float hi8[8], lo8[8];
         if (kind == kBlkLoad) {
-          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + 8 * j, hi8);
-          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + kHpg + 8 * j, lo8);
+          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + h0, hi8);
+          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + kHpg + h0, lo8);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) hi8[i] = lo8[i] = 0.f;
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[8 * j + i] = hi8[i] + lo8[i];
+        for (int i = 0; i < 8; ++i) o[i] = hi8[i] + lo8[i];
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[ob]);
       if (a.splits == 1) {
-        uint16_t* dst = a.out + (((long long)b * a.T + t) * kHq + kHpg * g) * kDim + d;
+        uint16_t* dst = a.out + (((long long)b * a.T + t) * kHq + kHpg * g + h0) * kDim + d;
 #pragma unroll
-        for (int h = 0; h < kHpg; ++h) {
+        for (int h = 0; h < kHh; ++h) {
           const float l = ls[h] + ls[kHpg + h] + ls[2 * kHpg + h] + ls[3 * kHpg + h];
           const float v = l > 0.f ? o[h] * (a.out_scale / l) : 0.f;
           const __nv_bfloat16 bv = __float2bfloat16_rn(v);
@@ -539,53 +541,52 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         // fp32 partial of this split: O (in units of 2^4 P), m (log2 units), l
         float* part = a.partials + (row * a.splits + sp) * kPartialFloats;
 #pragma unroll
-        for (int h = 0; h < kHpg; ++h) part[h * kDim + d] = o[h];
-        if (q == 0 && lane < kHpg) {
-          part[kHpg * kDim + lane] = kind == kBlkLoad ? mc : -INFINITY;
-          part[kHpg * kDim + kHpg + lane] =
+        for (int h = 0; h < kHh; ++h) part[(h0 + h) * kDim + d] = o[h];
+        if (q == 0 && lane < kHh) {
+          part[kHpg * kDim + h0 + lane] = kind == kBlkLoad ? mc : -INFINITY;
+          part[kHpg * kDim + kHpg + h0 + lane] =
               ls[lane] + ls[kHpg + lane] + ls[2 * kHpg + lane] + ls[3 * kHpg + lane];
         }
-        // all four warps' partials written and fenced, then one thread counts
-        // this split in; the result reaches the four warps through shared memory
+        // all eight warps' partials written and fenced, then one thread counts
+        // this split in; the result reaches the warps through shared memory
         __threadfence();
         __syncwarp();
         if (lane == 0) mbar_arrive(misc_bar);
         if (!mbar_wait(misc_bar, (nmisc++) & 1)) { report(a.flags, 5, 32); break; }
-        if (q == 0 && lane == 0) misc[nitem & 1] = (atomicAdd(&a.counters[row], 1) == a.splits - 1);
+        if (warp == kAttSoftWarp0 && lane == 0)
+          misc[nitem & 1] = (atomicAdd(&a.counters[row], 1) == a.splits - 1);
         __syncwarp();
         if (lane == 0) mbar_arrive(misc_bar);
         if (!mbar_wait(misc_bar, (nmisc++) & 1)) { report(a.flags, 5, 35); break; }
         if (misc[nitem & 1]) {
           __threadfence();
-          // 128 threads: head hr = tid'/8, 16 dims from (tid'%8)*16
-          const int tq = 32 * q + lane, hr = tq >> 3, d0 = (tq & 7) * 16;
+          // 256 threads: head hr = tq/16, 8 dims from (tq%16)*8
+          const int tq = (warp - kAttSoftWarp0) * 32 + lane, hr = tq >> 4, d0 = (tq & 15) * 8;
           const float* base = a.partials + row * a.splits * kPartialFloats;
           float Mx = -INFINITY;
           for (int s2 = 0; s2 < a.splits; ++s2)
             Mx = fmaxf(Mx, __ldcg(base + s2 * kPartialFloats + kHpg * kDim + hr));
           const float Mu = (Mx == -INFINITY) ? 0.f : Mx;
-          float tot[16];
+          float tot[8];
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) tot[cc] = 0.f;
+          for (int cc = 0; cc < 8; ++cc) tot[cc] = 0.f;
           float Lt = 0.f;
           for (int s2 = 0; s2 < a.splits; ++s2) {
             const float* ps2 = base + s2 * kPartialFloats;
             const float f = exp2f(__ldcg(ps2 + kHpg * kDim + hr) - Mu);
             Lt += __ldcg(ps2 + kHpg * kDim + kHpg + hr) * f;
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) tot[cc] += __ldcg(ps2 + hr * kDim + d0 + cc) * f;
+            for (int cc = 0; cc < 8; ++cc) tot[cc] += __ldcg(ps2 + hr * kDim + d0 + cc) * f;
           }
           const float inv = Lt > 0.f ? a.out_scale / Lt : 0.f;
-          uint32_t packed[8];
+          uint32_t packed[4];
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
+          for (int cc = 0; cc < 4; ++cc) {
             const __nv_bfloat162 v = __floats2bfloat162_rn(tot[2 * cc] * inv, tot[2 * cc + 1] * inv);
             packed[cc] = *reinterpret_cast<const uint32_t*>(&v);
           }
-          uint4* dst = reinterpret_cast<uint4*>(
-              a.out + (((long long)b * a.T + t) * kHq + kHpg * g + hr) * kDim + d0);
-          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          *reinterpret_cast<uint4*>(a.out + (((long long)b * a.T + t) * kHq + kHpg * g + hr) * kDim + d0) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
           if (tq == 0) a.counters[row] = 0;   // ready for the next call
         }
       }
@@ -594,9 +595,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------------------ decoders
-    const int quarter = warp & 3, half = warp >> 2;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
-    const int row = 32 * quarter + lane;             // key row of this thread
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    const int row = 32 * warp + lane;                // key row of this thread
     const int sw = (row >> 1) & 3;                   // 64-byte swizzle of the code rows
     for (int k = 0;; ++k) {
       const int s = k % kAttStages, x = k & 1;
@@ -613,15 +613,14 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         const uint8_t* vc = rs + kPageCodes;
         const uint8_t* ks = rs + 2 * kPageCodes;
         const uint8_t* vs = ks + kPageScales;
-        // K: dims 64h..64h+63 split by sign into A[x] (K+ cols 0-31, K- 32-63)
+        // K split by sign into A[x] (K+ cols 0-31, K- 32-63)
         const uint32_t abase = lane_base + kColA + 64 * x;
-        const uint32_t kscw = *reinterpret_cast<const uint32_t*>(ks + row * kRowScales + 4 * half);
-        if (__all_sync(0xffffffffu, (kscw & 0x80808080u) == 0u)) {
+        const uint2 ksc = *reinterpret_cast<const uint2*>(ks + row * kRowScales);
+        if (__all_sync(0xffffffffu, ((ksc.x | ksc.y) & 0x80808080u) == 0u)) {
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int cix = 2 * half + cc;
+          for (int cix = 0; cix < 4; ++cix) {
             const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
-            const uint32_t sb = kscw >> (16 * cc);
+            const uint32_t sb = (cix < 2 ? ksc.x : ksc.y) >> (16 * (cix & 1));
             const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
             uint32_t pw[8], nw[8];
             dq8_split_pos(w4.x, r0, pw[0], pw[1], nw[0], nw[1]);
@@ -633,10 +632,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           }
         } else {
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int cix = 2 * half + cc;
+          for (int cix = 0; cix < 4; ++cix) {
             const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
-            const uint32_t sb = kscw >> (16 * cc);
+            const uint32_t sb = (cix < 2 ? ksc.x : ksc.y) >> (16 * (cix & 1));
             const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
             const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
             const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
@@ -650,15 +648,14 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
             tmem_st8(abase + 32 + 8 * cix, nw);
           }
         }
-        // V: dims 64h..64h+63 signed, as E4M3 into the 128-byte V row of this
-        // key (16-byte chunk j at chunk position j ^ (key % 8))
-        const uint32_t vscw = *reinterpret_cast<const uint32_t*>(vs + row * kRowScales + 4 * half);
+        // V signed, as E4M3 into the 128-byte V row of this key (16-byte
+        // chunk j at chunk position j ^ (key % 8))
+        const uint2 vsc = *reinterpret_cast<const uint2*>(vs + row * kRowScales);
         uint8_t* vrow = vbuf + (k % kVB) * kBlock * kDim + row * kDim;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int cix = 2 * half + cc;
+        for (int cix = 0; cix < 4; ++cix) {
           const uint4 w4 = lds128(vc + row * kRowCodes + ((cix ^ sw) << 4));
-          const uint32_t sb = vscw >> (16 * cc);
+          const uint32_t sb = (cix < 2 ? vsc.x : vsc.y) >> (16 * (cix & 1));
           const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
           uint32_t o[8];
           dq8s(w4.x, r0, o[0], o[1]);
