@@ -220,97 +220,107 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
 
   if (warp == kAttProducerWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int k = 0, ki = 0;            // block slot, item sequence number
-      bool ok = true;
-      auto slot = [&](int kk) -> bool {
-        return kk < kAttStages ||
-               mbar_wait(&raw_empty[kk % kAttStages], ((kk / kAttStages) - 1) & 1);
-      };
-      auto emit = [&](int kind, int blk, int first, int last, long long row, int sp, int pos,
-                      long long page, int g) -> bool {
-        if (!slot(k)) { report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 20); return false; }
-        const int s = k % kAttStages;
-        int* m = meta + s * kInfo;
-        m[0] = kind; m[1] = blk; m[2] = first; m[3] = last;
-        m[4] = ki; m[5] = (int)row; m[6] = sp; m[7] = pos;
-        if (kind == kBlkLoad) {
-          uint8_t* dst = raw + s * kAttRawStride;
-          const long long r0 = (page * kG + g) * kBlock;      // first (page, head, token) row
-          mbar_expect_tx(&raw_full[s], kAttRawStride);
-          tma_load_2d(dst, &a.tmap_k, 0, (int)r0, &raw_full[s]);
-          tma_load_2d(dst + kPageCodes, &a.tmap_v, 0, (int)r0, &raw_full[s]);
-          bulk_g2s(dst + 2 * kPageCodes, a.k_scale + r0 * kRowScales, kPageScales, &raw_full[s]);
-          bulk_g2s(dst + 2 * kPageCodes + kPageScales, a.v_scale + r0 * kRowScales, kPageScales,
-                   &raw_full[s]);
+    // The whole warp sets up an item (lane kk checks selected block kk: its
+    // id and page load in parallel); lane 0 issues the copies.
+    int k = 0, ki = 0;            // block slot, item sequence number
+    bool ok = true;
+    auto emit = [&](int kind, int blk, int first, int last, long long row, int sp, int pos,
+                    long long page, int g) -> bool {
+      bool good = true;
+      if (lane == 0) {
+        if (k >= kAttStages && !mbar_wait(&raw_empty[k % kAttStages], ((k / kAttStages) - 1) & 1)) {
+          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 20);
+          good = false;
         } else {
-          mbar_arrive(&raw_full[s]);
-        }
-        ++k;
-        return true;
-      };
-      long long item = atomicAdd(&a.work[0], 1);
-      while (item < items && ok) {
-        const long long nxt = atomicAdd(&a.work[0], 1);   // claimed early: latency overlaps
-        const long long row = item / a.splits;
-        const int sp = (int)(item % a.splits);
-        const int b = (int)(row / (kG * a.T));
-        const int t = (int)((row / kG) % a.T);
-        const int g = (int)(row % kG);
-        const int L = a.seq_lens[b];
-        const bool len_ok = L >= a.T && L <= a.max_pages * kBlock;
-        const int pos = L - a.T + t;
-        const int nvis = pos / kBlock + 1;
-        const int k0 = kTopk * sp / a.splits, k1 = kTopk * (sp + 1) / a.splits;
-        if (!len_ok && sp == 0 && g == 0 && t == 0) report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
-        // pass 1: the valid blocks of this slice (ids in order, pages)
-        int nval = 0, lastk = -1;
-        if (len_ok) {
-          for (int kk = k0; kk < k1; ++kk) {
-            const int blk = a.sel[row * kTopk + kk];
-            if (blk < 0) continue;
-            if (blk >= nvis) { report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, blk); continue; }
-            const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + blk]
-                                             : (long long)b * a.max_pages + blk;
-            if (p < 0 || p >= a.num_pages) { report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)p); continue; }
-            ++nval;
-            lastk = kk;
+          const int s = k % kAttStages;
+          int* m = meta + s * kInfo;
+          m[0] = kind; m[1] = blk; m[2] = first; m[3] = last;
+          m[4] = ki; m[5] = (int)row; m[6] = sp; m[7] = pos;
+          if (kind == kBlkLoad) {
+            uint8_t* dst = raw + s * kAttRawStride;
+            const long long r0 = (page * kG + g) * kBlock;      // first (page, head, token) row
+            mbar_expect_tx(&raw_full[s], kAttRawStride);
+            tma_load_2d(dst, &a.tmap_k, 0, (int)r0, &raw_full[s]);
+            tma_load_2d(dst + kPageCodes, &a.tmap_v, 0, (int)r0, &raw_full[s]);
+            bulk_g2s(dst + 2 * kPageCodes, a.k_scale + r0 * kRowScales, kPageScales, &raw_full[s]);
+            bulk_g2s(dst + 2 * kPageCodes + kPageScales, a.v_scale + r0 * kRowScales, kPageScales,
+                     &raw_full[s]);
+          } else {
+            mbar_arrive(&raw_full[s]);
           }
         }
-        // the query rows of this item (previous user: item ki-2's last S MMA)
-        const int qs = ki & 1;
+      }
+      good = __shfl_sync(0xffffffffu, good, 0);
+      ++k;
+      return good;
+    };
+    long long item = 0;
+    if (lane == 0) item = atomicAdd(&a.work[0], 1);
+    item = __shfl_sync(0xffffffffu, item, 0);
+    while (item < items && ok) {
+      long long nxt = 0;
+      if (lane == 0) nxt = atomicAdd(&a.work[0], 1);     // claimed early: latency overlaps
+      const long long row = item / a.splits;
+      const int sp = (int)(item % a.splits);
+      const int b = (int)(row / (kG * a.T));
+      const int t = (int)((row / kG) % a.T);
+      const int g = (int)(row % kG);
+      const int L = a.seq_lens[b];
+      const bool len_ok = L >= a.T && L <= a.max_pages * kBlock;
+      const int pos = L - a.T + t;
+      const int nvis = pos / kBlock + 1;
+      const int k0 = kTopk * sp / a.splits, k1 = kTopk * (sp + 1) / a.splits;
+      if (lane == 0 && !len_ok && sp == 0 && g == 0 && t == 0) report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
+      // lane kk: selected block kk of this slice, validated
+      int blk = -1;
+      long long page = -1;
+      bool valid = false;
+      if (len_ok && lane >= k0 && lane < k1) {
+        blk = a.sel[row * kTopk + lane];
+        if (blk >= nvis) {
+          report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, blk);
+        } else if (blk >= 0) {
+          page = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + blk]
+                              : (long long)b * a.max_pages + blk;
+          if (page < 0 || page >= a.num_pages) report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)page);
+          else valid = true;
+        }
+      }
+      const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+      nxt = __shfl_sync(0xffffffffu, nxt, 0);
+      // the query rows of this item (previous user: item ki-2's last S MMA)
+      const int qs = ki & 1;
+      if (lane == 0) {
         if (ki >= 2 && !mbar_wait(&q_empty[qs], ((ki >> 1) - 1) & 1)) {
           report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 21);
           ok = false;
-          break;
-        }
-        if (nval > 0) {
+        } else if (vmask != 0u) {
           mbar_expect_tx(&q_full[qs], kHpg * kDim);
           tma_load_2d(qbuf + qs * kHpg * kDim, &a.tmap_q, 0,
                       (int)(((long long)b * a.T + t) * kHq + kHpg * g), &q_full[qs]);
         } else {
           mbar_arrive(&q_full[qs]);   // keeps the phase count; nothing waits on it
         }
-        // pass 2: emit
-        if (nval == 0) {
-          ok = emit(kBlkEmpty, 0, 1, 1, row, sp, pos, 0, g);
-        } else {
-          int e = 0;
-          for (int kk = k0; kk < k1 && ok; ++kk) {
-            const int blk = a.sel[row * kTopk + kk];
-            if (blk < 0 || blk >= nvis) continue;
-            const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + blk]
-                                             : (long long)b * a.max_pages + blk;
-            if (p < 0 || p >= a.num_pages) continue;
-            ok = emit(kBlkLoad, blk, e == 0, kk == lastk, row, sp, pos, p, g);
-            ++e;
-          }
-        }
-        ++ki;
-        item = nxt;
       }
-      if (ok) emit(kBlkEnd, 0, 0, 0, 0, 0, 0, 0, 0);
-      // every CTA has made its last claim once all have arrived here
+      ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+      if (!ok) break;
+      if (vmask == 0u) {
+        ok = emit(kBlkEmpty, 0, 1, 1, row, sp, pos, 0, g);
+      } else {
+        const int lastk = 31 - __clz(vmask);
+        for (unsigned m = vmask; m != 0u && ok; m &= m - 1u) {
+          const int kk = __ffs(m) - 1;
+          const int bk = __shfl_sync(0xffffffffu, blk, kk);
+          const long long pk = __shfl_sync(0xffffffffu, page, kk);
+          ok = emit(kBlkLoad, bk, m == vmask, kk == lastk, row, sp, pos, pk, g);
+        }
+      }
+      ++ki;
+      item = nxt;
+    }
+    if (ok) emit(kBlkEnd, 0, 0, 0, 0, 0, 0, 0, 0);
+    // every CTA has made its last claim once all have arrived here
+    if (lane == 0) {
       __threadfence();
       if (atomicAdd(&a.work[1], 1) == (int)gridDim.x - 1) {
         atomicExch(&a.work[0], 0);
