@@ -15,13 +15,14 @@
 //     tiled TMA loads of the K and V codes (64-byte swizzle) and two bulk
 //     copies of their scales into a ring of shared-memory stages;
 //   warps 0-3 (decoders): thread = key row, warp w decoding rows
-//     32w..32w+31.  K is decoded split
-//     by sign (K+ and K- magnitudes, as in the indexer) straight into tensor
-//     memory; V is decoded signed into shared memory as E4M3 rows of 128
+//     32w..32w+31.  K is decoded signed (dq8s) straight into tensor memory
+//     (one A operand: 4 MMAs per block rather than 8 for a split by sign --
+//     the MMA-issuing thread is the scarcer resource here); V is decoded
+//     signed into shared memory as E4M3 rows of 128
 //     bytes with the 128-byte swizzle -- the A operand of O^T = V^T P^T in
 //     MN-major form;
 //   warp 13 (MMA, one thread): per block
-//       S^T[128 keys x 16 heads]  = K+ Q^T - K- Q^T   (8 MMAs, A from TMEM)
+//       S^T[128 keys x 16 heads]  = K Q^T   (4 MMAs, A from TMEM)
 //       O^T[128 dims x 32]       += V^T [P_hi | P_lo]^T  (4 MMAs, A and B in
 //                                   shared memory, both MN-major),
 //     issuing block k+1's S before block k's O so that the softmax of the
@@ -54,8 +55,8 @@ constexpr int kHh = kHpg / 2;               // heads per softmax warp
 constexpr int kAttProducerWarp = 12;
 constexpr int kAttMmaWarp = 13;
 constexpr int kAttRawStride = 2 * (kPageCodes + kPageScales);   // 18432 = 18 x 1024
-constexpr int kAttTmemCols = 256;           // A[2] 0..127, S[2] 128..159, O[2] 160..223
-constexpr int kColA = 0, kColS = 128, kColO = 160;
+constexpr int kAttTmemCols = 256;           // A[2] 0..63, S[2] 64..95, O[2] 96..159
+constexpr int kColA = 0, kColS = 64, kColO = 96;
 constexpr float kPExp = 4.f;                // P carries a factor 2^4 (E4M3 normal range)
 constexpr float kLazy = 4.f;                // raise m only when a block max exceeds it by 2^4
 constexpr int kVB = 3;                      // V and P buffers (blocks between decode and O update)
@@ -331,7 +332,6 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_e4m3_f32(128, kHpg);
-      constexpr uint32_t idesc_sn = idesc_s | (1u << 13);                       // negate A
       constexpr uint32_t idesc_o = idesc_e4m3_f32(128, 2 * kHpg) | (1u << 15) | (1u << 16);
       const uint64_t qd[2] = {desc_kmajor_sw128(smem_u32(qbuf)),
                               desc_kmajor_sw128(smem_u32(qbuf + kHpg * kDim))};
@@ -345,12 +345,10 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         if (kind == kBlkLoad) {
           if (first && !mbar_wait(&q_full[ki & 1], (ki >> 1) & 1)) { report(a.flags, 5, 23); return -1; }
           const uint32_t d = tmem + kColS + kHpg * x;
-          const uint32_t ta = tmem + kColA + 64 * x;
+          const uint32_t ta = tmem + kColA + 32 * x;
           const uint64_t bd = qd[ki & 1];
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc_s, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 32 + 8 * kk, bd + 2 * kk, idesc_sn, 1);
         }
         tc_commit(&s_full[x]);
         if (kind != kBlkEnd && last) tc_commit(&q_empty[ki & 1]);
@@ -538,12 +536,15 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[ob]);
+      // lanes 0-7: the row sum of head h0+lane over the four quarters
+      const float lrow = lane < kHh ? ls[lane] + ls[kHpg + lane] + ls[2 * kHpg + lane] + ls[3 * kHpg + lane]
+                                    : 0.f;
       if (a.splits == 1) {
+        const float f = lrow > 0.f ? a.out_scale / lrow : 0.f;   // lanes 0-7
         uint16_t* dst = a.out + (((long long)b * a.T + t) * kHq + kHpg * g + h0) * kDim + d;
 #pragma unroll
         for (int h = 0; h < kHh; ++h) {
-          const float l = ls[h] + ls[kHpg + h] + ls[2 * kHpg + h] + ls[3 * kHpg + h];
-          const float v = l > 0.f ? o[h] * (a.out_scale / l) : 0.f;
+          const float v = o[h] * __shfl_sync(0xffffffffu, f, h);
           const __nv_bfloat16 bv = __float2bfloat16_rn(v);
           dst[(long long)h * kDim] = *reinterpret_cast<const uint16_t*>(&bv);
         }
@@ -554,8 +555,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         for (int h = 0; h < kHh; ++h) part[(h0 + h) * kDim + d] = o[h];
         if (q == 0 && lane < kHh) {
           part[kHpg * kDim + h0 + lane] = kind == kBlkLoad ? mc : -INFINITY;
-          part[kHpg * kDim + kHpg + h0 + lane] =
-              ls[lane] + ls[kHpg + lane] + ls[2 * kHpg + lane] + ls[3 * kHpg + lane];
+          part[kHpg * kDim + kHpg + h0 + lane] = lrow;
         }
         // all eight warps' partials written and fenced, then one thread counts
         // this split in; the result reaches the warps through shared memory
@@ -623,40 +623,20 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         const uint8_t* vc = rs + kPageCodes;
         const uint8_t* ks = rs + 2 * kPageCodes;
         const uint8_t* vs = ks + kPageScales;
-        // K split by sign into A[x] (K+ cols 0-31, K- 32-63)
-        const uint32_t abase = lane_base + kColA + 64 * x;
+        // K signed, as E4M3 into A[x] (row = TMEM lane, 32 columns)
+        const uint32_t abase = lane_base + kColA + 32 * x;
         const uint2 ksc = *reinterpret_cast<const uint2*>(ks + row * kRowScales);
-        if (__all_sync(0xffffffffu, ((ksc.x | ksc.y) & 0x80808080u) == 0u)) {
 #pragma unroll
-          for (int cix = 0; cix < 4; ++cix) {
-            const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
-            const uint32_t sb = (cix < 2 ? ksc.x : ksc.y) >> (16 * (cix & 1));
-            const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
-            uint32_t pw[8], nw[8];
-            dq8_split_pos(w4.x, r0, pw[0], pw[1], nw[0], nw[1]);
-            dq8_split_pos(w4.y, r0, pw[2], pw[3], nw[2], nw[3]);
-            dq8_split_pos(w4.z, r1, pw[4], pw[5], nw[4], nw[5]);
-            dq8_split_pos(w4.w, r1, pw[6], pw[7], nw[6], nw[7]);
-            tmem_st8(abase + 8 * cix, pw);
-            tmem_st8(abase + 32 + 8 * cix, nw);
-          }
-        } else {
-#pragma unroll
-          for (int cix = 0; cix < 4; ++cix) {
-            const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
-            const uint32_t sb = (cix < 2 ? ksc.x : ksc.y) >> (16 * (cix & 1));
-            const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
-            const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
-            const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
-            const uint32_t f1 = (s1 & 0x80u) ? 0x88888888u : 0u;
-            uint32_t pw[8], nw[8];
-            dq8_split(w4.x, r0, f0, pw[0], pw[1], nw[0], nw[1]);
-            dq8_split(w4.y, r0, f0, pw[2], pw[3], nw[2], nw[3]);
-            dq8_split(w4.z, r1, f1, pw[4], pw[5], nw[4], nw[5]);
-            dq8_split(w4.w, r1, f1, pw[6], pw[7], nw[6], nw[7]);
-            tmem_st8(abase + 8 * cix, pw);
-            tmem_st8(abase + 32 + 8 * cix, nw);
-          }
+        for (int cix = 0; cix < 4; ++cix) {
+          const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
+          const uint32_t sb = (cix < 2 ? ksc.x : ksc.y) >> (16 * (cix & 1));
+          const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+          uint32_t o[8];
+          dq8s(w4.x, r0, o[0], o[1]);
+          dq8s(w4.y, r0, o[2], o[3]);
+          dq8s(w4.z, r1, o[4], o[5]);
+          dq8s(w4.w, r1, o[6], o[7]);
+          tmem_st8(abase + 8 * cix, o);
         }
         // V signed, as E4M3 into the 128-byte V row of this key (16-byte
         // chunk j at chunk position j ^ (key % 8))
