@@ -17,38 +17,36 @@
 // do not serve equally -- and ragged batches still finish together; the last
 // CTA to finish resets the counter.  Warp roles inside a CTA, all running a
 // few pages apart:
-//   warp 16 (producer): per page one tiled TMA load of the codes (64-byte
+//   warp 12 (producer): per page one tiled TMA load of the codes (64-byte
 //     swizzle, so that row-per-thread reads are bank-conflict free) and one
 //     bulk copy of the scales into a ring of shared-memory stages;
-//   warps 0-7 (decoders): warps w and w+4 share the TMEM lanes (= key rows)
-//     32(w%4)..32(w%4)+31; thread = key row, warp w decoding dims 0-63 of
-//     its row and warp w+4 dims 64-127.  NVFP4 rows are decoded by sign: K+
-//     holds E4M3(|v|) of the positive elements, K- of the negative ones (one
-//     prmt per 4 codes each, see dq8_split), and both go straight to tensor
-//     memory with tcgen05.st into one of two A buffers -- the A operand never
-//     touches shared memory, and page k+1 is decoded while page k's MMA runs;
-//   warp 17 (MMA): one thread issues per page 4 tcgen05.mma with A = K+ and 4
+//   warps 0-3 (decoders): thread = key row (= TMEM lane).  NVFP4 rows are
+//     decoded by sign: K+ holds E4M3(|v|) of the positive elements, K- of the
+//     negative ones (one prmt per 4 codes each, see dq8_split), and both go
+//     straight to tensor memory with tcgen05.st into one of two A buffers --
+//     the A operand never touches shared memory, and page k+1 is decoded
+//     while page k's MMAs run;
+//   warp 13 (MMA): one thread issues per page 4 tcgen05.mma with A = K+ and 4
 //     with A = K- and the negate-A bit (K = 32 each, A from TMEM, B = the
 //     queries in shared memory) into a double-buffered TMEM accumulator;
-//   warps 8-15 (epilogue, two groups of four taking the even and the odd
-//     pages, so that two pages are reduced at once): warp 8+4j+q reads the
-//     accumulator lanes of quarter q,
-//     masks keys after each query's position, and reduces over keys: in-thread
-//     over the four keys a 16x256b load gives each thread, then xor shuffles
-//     across lane groups; after a rendezvous on an mbarrier each warp
-//     combines the four quarters' partial maxima of a quarter of the columns
-//     and writes those block scores.
+//   warps 4-11 (epilogue, two groups of four taking the even and the odd
+//     pages, so that two pages are reduced at once): warp 4+4j+q reads the
+//     accumulator lanes of quarter q, masks keys after each query's position,
+//     and reduces over keys: in-thread over the four keys a 16x256b load
+//     gives each thread, then xor shuffles across lane groups; after a
+//     rendezvous on an mbarrier each warp combines the four quarters' partial
+//     maxima of a quarter of the columns and writes those block scores.
 // Every wait is a bounded mbarrier wait; on a timeout a thread records
 // MSA_ERR_TIMEOUT and leaves its loop, and TMEM is freed before exit.
 #include "msa_internal.h"
 
 namespace msa {
 
-constexpr int kIdxDecoders = 8;             // two per TMEM lane quarter
+constexpr int kIdxDecoders = 4;             // one per TMEM lane quarter, full rows
 constexpr int kIdxEpilogue = 4;             // per group: one per TMEM lane quarter
-constexpr int kIdxEpiWarp0 = 8;             // two groups: even and odd pages
-constexpr int kIdxProducerWarp = 16;
-constexpr int kIdxMmaWarp = 17;
+constexpr int kIdxEpiWarp0 = 4;             // two groups: even and odd pages
+constexpr int kIdxProducerWarp = 12;
+constexpr int kIdxMmaWarp = 13;
 constexpr int kABufCols = 64;               // TMEM columns of one A buffer (K+ | K-)
 constexpr int kACols = 2 * kABufCols;       // two A buffers
 
@@ -423,7 +421,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     }
   } else {
     // ------------------------------------------------------------ decoders
-    const int quarter = warp & 3, half = warp >> 2;
+    const int quarter = warp;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);   // this warp's TMEM lanes
     const int row = 32 * quarter + lane;                                  // key row of this thread
     int cur_b = -1, cur_y = -1, qsel = 1, L = 0, ends = 0;
@@ -464,10 +462,9 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         const uint32_t abase = lane_base + ab * kABufCols;
         if constexpr (FP8IDX) {
           // 128-byte rows loaded with the 128-byte swizzle: chunk c of row r
-          // sits at chunk position c ^ (r % 8).  This warp: dims 64h..64h+63.
+          // sits at chunk position c ^ (r % 8).
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int c2 = 2 * half + cc;
+          for (int c2 = 0; c2 < 4; ++c2) {
             const uint4 x0 = lds128(rs + row * 128 + (((2 * c2) ^ (row & 7)) << 4));
             const uint4 x1 = lds128(rs + row * 128 + (((2 * c2 + 1) ^ (row & 7)) << 4));
             const uint32_t w8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
@@ -475,19 +472,15 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           }
         } else {
           // 64-byte code rows loaded with the 64-byte swizzle: chunk c of
-          // row r sits at chunk position c ^ ((r / 2) % 4).  This warp:
-          // chunks 2h, 2h+1 (dims 64h..64h+63, block scales 4h..4h+3).
-          const uint32_t scw =
-              *reinterpret_cast<const uint32_t*>(rs + kPageCodes + row * kRowScales + 4 * half);
+          // row r sits at chunk position c ^ ((r / 2) % 4).
+          const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
           const int sw = (row >> 1) & 3;
           // warp-uniform branch: tcgen05.st is a .sync.aligned warp instruction
-          if (__all_sync(0xffffffffu, (scw & 0x80808080u) == 0u)) {
-            // every block scale of the warp's 32 half rows is non-negative
+          if (__all_sync(0xffffffffu, ((sc.x | sc.y) & 0x80808080u) == 0u)) {
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              const int c = 2 * half + cc;
+            for (int c = 0; c < 4; ++c) {
               const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-              const uint32_t sb = scw >> (16 * cc);                     // scales 2c, 2c+1
+              const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));   // scales 2c, 2c+1
               const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
               uint32_t pw[8], nw[8];
               dq8_split_pos(w4.x, r0, pw[0], pw[1], nw[0], nw[1]);
@@ -499,10 +492,9 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
             }
           } else {
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              const int c = 2 * half + cc;
+            for (int c = 0; c < 4; ++c) {
               const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-              const uint32_t sb = scw >> (16 * cc);
+              const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));
               const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
               const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
               const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;

@@ -11,7 +11,7 @@
 
 namespace msa {
 
-constexpr int kIdxThreads = 18 * 32;    // 8 decoders, 8 epilogue warps, producer, MMA warp
+constexpr int kIdxThreads = 14 * 32;    // 4 decoders, 8 epilogue warps, producer, MMA warp
 constexpr int kIdxRawStages = 6;         // raw index-key pages in flight per CTA
 
 struct IdxArgs {
