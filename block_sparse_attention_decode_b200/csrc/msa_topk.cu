@@ -2,7 +2,8 @@
 // the top 16 blocks and the most recent block is always kept).
 // post = vLLM 為 MiniMax-M3.1-Flash 提供 Day-0 支援 (hot.atechcom.net).
 //
-// One CTA per (sequence, token, group) row.  The latest visible block is
+// One warp per (sequence, token, group) row, four rows per CTA, no block-wide
+// synchronisation.  The latest visible block is
 // kept; the other 15 are the best of blocks 0 .. latest-1 ranked by (score
 // descending, block id ascending).  Selection is an exact radix select over
 // order-preserving 32-bit keys of the fp32 scores (4 passes of 8 bits) that
@@ -16,104 +17,120 @@
 
 namespace msa {
 
-constexpr int kTopkThreads = 128;
-constexpr int kTopkCache = 4096;   // rows up to this many candidates are cached in smem
+constexpr int kTopkRows = 4;                  // rows (warps) per CTA
+constexpr int kTopkThreads = 32 * kTopkRows;
+constexpr int kTopkCache = 2048;              // candidates per row cached in shared memory
 
 __global__ void __launch_bounds__(kTopkThreads)
 topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_lens, int B, int T,
             int max_pages, int32_t* __restrict__ sel, Flags* flags) {
-  __shared__ unsigned keys[kTopkCache];
-  __shared__ unsigned hist[256];
-  __shared__ unsigned s_prefix;
-  __shared__ int s_need;
-
-  const long long row = blockIdx.x;          // (b * T + t) * 4 + g
+  __shared__ unsigned keys_all[kTopkRows][kTopkCache];
+  __shared__ unsigned hist_all[kTopkRows][256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * kTopkRows + w;   // (b * T + t) * 4 + g
+  if (row >= (long long)B * T * kG) return;
+  unsigned* keys = keys_all[w];
+  unsigned* hist = hist_all[w];
   const int b = (int)(row / (kG * T));
   const int t = (int)((row / kG) % T);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* out = sel + row * kTopk;
   const int L = seq_lens[b];
   if (L < T || L > max_pages * kBlock) {
-    if (tid == 0 && (row % kG) == 0 && t == 0) report(flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
-    if (tid < kTopk) out[tid] = -1;
+    if (lane == 0 && (row % kG) == 0 && t == 0) report(flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
+    if (lane < kTopk) out[lane] = -1;
     return;
   }
   const int pos = L - T + t;
   const int nb = pos / kBlock + 1;           // visible blocks; the latest is nb-1
   if (nb <= kTopk) {
-    if (tid < kTopk) out[tid] = tid < nb ? tid : -1;
+    if (lane < kTopk) out[lane] = lane < nb ? lane : -1;
     return;
   }
   const float* S = scores + row * max_pages;
   const int n = nb - 1;                      // candidates 0 .. nb-2
   const bool cached = n <= kTopkCache;
-  if (cached)
-    for (int i = tid; i < n; i += kTopkThreads) keys[i] = float_key(S[i]);
+  unsigned kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int i = lane; i < n; i += 32) {
+    const unsigned k = float_key(S[i]);
+    if (cached) keys[i] = k;
+    kmin = min(kmin, k);
+    kmax = max(kmax, k);
+  }
+  __syncwarp();
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
   auto key_at = [&](int i) -> unsigned { return cached ? keys[i] : float_key(S[i]); };
 
   // Radix select, 8 bits per pass from the top: after the passes `prefix`
   // is the key of the 15th best candidate and `need` how many candidates
   // equal to it belong to the selection.
-  unsigned prefix = 0;
+  // Bytes every candidate shares are known already: start at the highest
+  // byte where the smallest and the largest key differ (the scores of a row
+  // usually share their sign and top exponent bits, which would otherwise
+  // send a whole pass's counts into one or two bins).
+  const int top = (31 - __clz(kmin ^ kmax)) >> 3;           // -1 when all keys are equal
+  unsigned prefix = top < 0 ? kmax : (top >= 3 ? 0u : (kmax & ~((1u << (8 * top + 8)) - 1u)));
   int need = kTopk - 1;
-  for (int pass = 3; pass >= 0; --pass) {
+#pragma unroll 1
+  for (int pass = top; pass >= 0; --pass) {
     const int shift = 8 * pass;
-    for (int d = tid; d < 256; d += kTopkThreads) hist[d] = 0;
-    __syncthreads();
-    for (int i = tid; i < n; i += kTopkThreads) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
       const unsigned k = key_at(i);
       if (pass == 3 || (k >> (shift + 8)) == (prefix >> (shift + 8)))
         atomicAdd(&hist[(k >> shift) & 255u], 1u);
     }
-    __syncthreads();
-    if (warp == 0) {   // digit search: lane l owns bins 255-8l .. 248-8l (descending)
-      unsigned c[8], sum = 0;
+    __syncwarp();
+    // digit search: lane l owns bins 255-8l .. 248-8l (descending)
+    unsigned c[8], sum = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) { c[j] = hist[255 - 8 * lane - j]; sum += c[j]; }
-      unsigned incl = sum;
+    for (int j = 0; j < 8; ++j) { c[j] = hist[255 - 8 * lane - j]; sum += c[j]; }
+    unsigned incl = sum;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)need);
-      if (lane == __ffs(hit) - 1) {
-        unsigned above = incl - sum;
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)need);
+    const int src = __ffs(hit) - 1;
+    unsigned np = 0;
+    int nn = 0;
+    if (lane == src) {
+      unsigned above = incl - sum;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (above + c[j] >= (unsigned)need) {
-            s_prefix = prefix | ((unsigned)(255 - 8 * lane - j) << shift);
-            s_need = need - (int)above;
-            break;
-          }
-          above += c[j];
+      for (int j = 0; j < 8; ++j) {
+        if (above + c[j] >= (unsigned)need) {
+          np = prefix | ((unsigned)(255 - 8 * lane - j) << shift);
+          nn = need - (int)above;
+          break;
         }
+        above += c[j];
       }
     }
-    __syncthreads();
-    prefix = s_prefix;
-    need = s_need;
+    prefix = __shfl_sync(0xffffffffu, np, src);
+    need = __shfl_sync(0xffffffffu, nn, src);
+    __syncwarp();   // the histogram is rewritten by the next pass
   }
-  // One warp emits the selection in id order: every candidate above the
-  // threshold key and the `need` lowest ids equal to it, then the latest.
-  if (warp == 0) {
-    int eq_seen = 0, emitted = 0;
-    for (int base = 0; base < n && emitted < kTopk - 1; base += 32) {
-      const int i = base + lane;
-      const unsigned k = i < n ? key_at(i) : 0u;
-      const bool gt = i < n && k > prefix;
-      const bool eq = i < n && k == prefix;
-      const unsigned lt = (1u << lane) - 1u;
-      const unsigned beq = __ballot_sync(0xffffffffu, eq);
-      const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need);
-      const unsigned btake = __ballot_sync(0xffffffffu, take);
-      const int slot = emitted + __popc(btake & lt);
-      if (take && slot < kTopk - 1) out[slot] = i;
-      eq_seen += __popc(beq);
-      emitted += __popc(btake);
-    }
-    if (lane == 0) out[kTopk - 1] = nb - 1;
+  // Emit the selection in id order: every candidate above the threshold key
+  // and the `need` lowest ids equal to it, then the latest.
+  int eq_seen = 0, emitted = 0;
+  for (int base = 0; base < n && emitted < kTopk - 1; base += 32) {
+    const int i = base + lane;
+    const unsigned k = i < n ? key_at(i) : 0u;
+    const bool gt = i < n && k > prefix;
+    const bool eq = i < n && k == prefix;
+    const unsigned lt = (1u << lane) - 1u;
+    const unsigned beq = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need);
+    const unsigned btake = __ballot_sync(0xffffffffu, take);
+    const int slot = emitted + __popc(btake & lt);
+    if (take && slot < kTopk - 1) out[slot] = i;
+    eq_seen += __popc(beq);
+    emitted += __popc(btake);
   }
+  if (lane == 0) out[kTopk - 1] = nb - 1;
 }
 
 __global__ void maxpool_kernel(const float* __restrict__ ts, const int32_t* __restrict__ seq_lens,
@@ -137,8 +154,9 @@ cudaError_t launch_topk(const float* block_scores, const int32_t* seq_lens, int 
                         int max_pages, int32_t* sel, Flags* flags, cudaStream_t st) {
   const long long rows = (long long)B * T * kG;
   if (rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  topk_kernel<<<(unsigned)rows, kTopkThreads, 0, st>>>(block_scores, seq_lens, B, T, max_pages,
-                                                        sel, flags);
+  const long long ctas = (rows + kTopkRows - 1) / kTopkRows;
+  topk_kernel<<<(unsigned)ctas, kTopkThreads, 0, st>>>(block_scores, seq_lens, B, T, max_pages,
+                                                       sel, flags);
   return cudaGetLastError();
 }
 
