@@ -87,6 +87,16 @@ def lib():
         L.orc_attention.argtypes = [ctypes.POINTER(_Cache), ctypes.c_void_p, ctypes.c_double,
                                     ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p,
                                     ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+        L.orc_e2m1_round.restype = ctypes.c_uint
+        L.orc_e2m1_round.argtypes = [ctypes.c_double]
+        L.orc_nvfp4_encode_row.restype = None
+        L.orc_nvfp4_encode_row.argtypes = [ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
+                                           ctypes.c_void_p]
+        L.orc_fp8_encode_row.restype = None
+        L.orc_fp8_encode_row.argtypes = [ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p]
+        L.orc_kv_insert.restype = ctypes.c_int
+        L.orc_kv_insert.argtypes = [ctypes.POINTER(_Cache), ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_float, ctypes.c_float, ctypes.c_float]
         L.orc_set_threads(os.cpu_count() or 1)
         _lib = L
     return _lib
@@ -123,6 +133,29 @@ def decode_nvfp4_row(data64: np.ndarray, scale8: np.ndarray) -> np.ndarray:
     assert data64.size == 64 and scale8.size == 8
     out = np.empty(128, np.float64)
     lib().orc_decode_nvfp4_row(data64.ctypes.data, scale8.ctypes.data, out.ctypes.data)
+    return out
+
+
+def e2m1_round(y: float) -> int:
+    """Nearest E2M1 magnitude code (0..7) of y >= 0, ties to the even code."""
+    return lib().orc_e2m1_round(float(y))
+
+
+def nvfp4_encode_row(x: np.ndarray, s_t: float):
+    """128 fp32 values -> (codes uint8[64], scales uint8[8]) (the insert reading)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    assert x.size == 128
+    data = np.zeros(64, np.uint8)
+    sc = np.zeros(8, np.uint8)
+    lib().orc_nvfp4_encode_row(x.ctypes.data, float(s_t), data.ctypes.data, sc.ctypes.data)
+    return data, sc
+
+
+def fp8_encode_row(x: np.ndarray, s_t: float) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    assert x.size == 128
+    out = np.zeros(128, np.uint8)
+    lib().orc_fp8_encode_row(x.ctypes.data, float(s_t), out.ctypes.data)
     return out
 
 
@@ -228,3 +261,15 @@ def decode(cache: Cache, qi, s_qi, q, s_q, softmax_scale, rows):
     sel = select(cache, rows, bs)
     out = attention(cache, q, s_q, softmax_scale, rows, sel)
     return bs, sel, out
+
+
+def kv_insert(cache: Cache, k_new: np.ndarray, v_new: np.ndarray, idx_new: np.ndarray) -> int:
+    """Quantise the T new tokens of every sequence into `cache` in place.
+    k_new, v_new: fp32 [B][T][4][128]; idx_new: fp32 [B][T][128]."""
+    k_new = np.ascontiguousarray(k_new, dtype=np.float32)
+    v_new = np.ascontiguousarray(v_new, dtype=np.float32)
+    idx_new = np.ascontiguousarray(idx_new, dtype=np.float32)
+    c = cache._c()
+    return int(lib().orc_kv_insert(ctypes.byref(c), k_new.ctypes.data, v_new.ctypes.data,
+                                   idx_new.ctypes.data, np.float32(cache.s_idx),
+                                   np.float32(cache.s_k), np.float32(cache.s_v)))

@@ -458,3 +458,108 @@ void orc_decode_nvfp4_row(const uint8_t* data64, const uint8_t* scale8, double* 
 {
     decode_nvfp4_row(data64, scale8, out128);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Writing new tokens into the cache (NVFP4 / FP8 encode)                    */
+/* ------------------------------------------------------------------------ */
+/* The step before the decode path: the T new tokens' K, V and index key are
+ * quantised into the paged cache ([post, "What is new in the MiniMax-M3.1
+ * architecture"]: NVFP4 KV cache for indexer and attention; [post, "QKV GEMM
+ * + norm + RoPE + KV insert fusion"] names the insertion).  The pages do not
+ * spell out the quantiser; the reading taken (listed in the design notes):
+ *   per 16 elements   r  = amax / (6 * s_t)              (fp32 arithmetic)
+ *                     sb = E4M3 of r, nearest, ties to even, saturating
+ *                     u  = e4m3(sb) * s_t                 (fp32)
+ *   per element       y  = x / u                          (fp32)
+ *                     code = nearest E2M1 magnitude of |y|, ties to the even
+ *                     code, saturating at 6; sign bit set for x < 0 unless
+ *                     the magnitude is 0; u == 0 gives code 0.
+ *   FP8 index keys    E4M3 of x / s_idx (fp32), nearest-even, saturating.
+ * The divisions whose results decide the codes are done in fp32, the
+ * precision a kernel takes them in, so that both sides decide alike. */
+
+/* Nearest E2M1 magnitude code (0..7) of y >= 0: the grid point at the
+ * smallest distance; on a tie the code with mantissa bit 0. */
+unsigned orc_e2m1_round(double y)
+{
+    unsigned best = 0;
+    double bd = INFINITY;
+    if (!(y > 0.0)) return 0u;
+    for (unsigned c = 0; c < 8u; ++c) {
+        const double d = fabs(y - orc_e2m1(c));
+        if (d < bd || (d == bd && (c & 1u) == 0u)) { bd = d; best = c; }
+    }
+    return best;
+}
+
+/* One 128-element row x (fp32 values) -> packed codes [64] + scales [8]. */
+void orc_nvfp4_encode_row(const float* x, float s_t, uint8_t* data64, uint8_t* scale8)
+{
+    volatile float six_st = 6.0f * s_t;       /* volatile: one fp32 rounding each */
+    for (int j = 0; j < ORC_D / 16; ++j) {
+        float amax = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            const float a = fabsf(x[16 * j + i]);
+            if (a > amax) amax = a;
+        }
+        volatile float r = amax / six_st;
+        const unsigned sb = orc_e4m3_round((double)r);
+        volatile float u = (float)orc_e4m3(sb) * s_t;
+        scale8[j] = (uint8_t)sb;
+        for (int i = 0; i < 16; ++i) {
+            const int d = 16 * j + i;
+            unsigned code = 0u;
+            if (u != 0.0f) {
+                volatile float y = x[d] / u;
+                code = orc_e2m1_round(fabs((double)y));
+                if (code != 0u && x[d] < 0.0f) code |= 8u;
+            }
+            if (d & 1) data64[d >> 1] = (uint8_t)((data64[d >> 1] & 0x0Fu) | (code << 4));
+            else data64[d >> 1] = (uint8_t)((data64[d >> 1] & 0xF0u) | code);
+        }
+    }
+}
+
+/* One 128-element row -> FP8 E4M3 bytes. */
+void orc_fp8_encode_row(const float* x, float s_t, uint8_t* out128)
+{
+    for (int d = 0; d < ORC_D; ++d) {
+        volatile float y = x[d] / s_t;
+        out128[d] = (uint8_t)orc_e4m3_round((double)y);
+    }
+}
+
+/* Write the T new tokens of every sequence (positions L-T .. L-1) into the
+ * cache c (whose buffers the caller owns and lets this function write):
+ * k_new, v_new [B][T][4][128], idx_new [B][T][128], fp32 values; s_* are the
+ * cache's fp32 tensor scales.  Returns -1 if a position has no page. */
+int orc_kv_insert(const orc_cache* c, const float* k_new, const float* v_new,
+                  const float* idx_new, float s_idx, float s_k, float s_v)
+{
+    int rc = 0;
+    for (int b = 0; b < c->batch; ++b) {
+        for (int t = 0; t < c->q_tokens; ++t) {
+            const int64_t pos = query_pos(c, b, t);
+            const int64_t p = page_of(c, b, pos / ORC_BLOCK);
+            const int64_t slot = pos % ORC_BLOCK;
+            const int64_t tok = (int64_t)b * c->q_tokens + t;
+            if (p < 0 || !row_ok(c, b, t)) { rc = -1; continue; }
+            for (int g = 0; g < ORC_G; ++g) {
+                const int64_t r = (p * ORC_G + g) * ORC_BLOCK + slot;
+                orc_nvfp4_encode_row(k_new + (tok * ORC_G + g) * ORC_D, s_k,
+                                     (uint8_t*)c->k_data + r * 64, (uint8_t*)c->k_scale + r * 8);
+                orc_nvfp4_encode_row(v_new + (tok * ORC_G + g) * ORC_D, s_v,
+                                     (uint8_t*)c->v_data + r * 64, (uint8_t*)c->v_scale + r * 8);
+            }
+            {
+                const int64_t r = p * ORC_BLOCK + slot;
+                if (c->idx_fp8)
+                    orc_fp8_encode_row(idx_new + tok * ORC_D, s_idx, (uint8_t*)c->idx_data + r * 128);
+                else
+                    orc_nvfp4_encode_row(idx_new + tok * ORC_D, s_idx, (uint8_t*)c->idx_data + r * 64,
+                                         (uint8_t*)c->idx_scale + r * 8);
+            }
+        }
+    }
+    return rc;
+}
