@@ -485,6 +485,7 @@ unsigned orc_e2m1_round(double y)
     unsigned best = 0;
     double bd = INFINITY;
     if (!(y > 0.0)) return 0u;
+    if (y >= 6.0) return 7u;                  /* saturates at the largest value */
     for (unsigned c = 0; c < 8u; ++c) {
         const double d = fabs(y - orc_e2m1(c));
         if (d < bd || (d == bd && (c & 1u) == 0u)) { bd = d; best = c; }

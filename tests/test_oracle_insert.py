@@ -28,6 +28,7 @@ def test_e2m1_round_hand_cases():
     for y, c in ties.items():
         assert oracle.e2m1_round(y) == c, y
     assert oracle.e2m1_round(6.5) == 7 and oracle.e2m1_round(1e9) == 7     # saturates
+    assert oracle.e2m1_round(1e30) == 7      # beyond where y - 4 and y - 6 are equal in f64
     assert oracle.e2m1_round(0.2499) == 0 and oracle.e2m1_round(0.2501) == 1
 
 
@@ -92,10 +93,12 @@ def test_fp8_rows_equal_torch_cast():
 def test_saturation_and_zero_blocks():
     x = np.zeros(128, np.float32)
     x[16:32] = 1e6                                    # far above 448 * 6 * s_t
+    x[32:48] = 1e30                                   # quotients far beyond f64 resolution of 6
     data, sc = oracle.nvfp4_encode_row(x, 6.0 / 448.0)
     assert sc[0] == 0 and np.all(data[:8] == 0)          # all-zero block
     assert sc[1] == 0x7E                               # scale saturates at 448
-    assert np.all(data[8:16] == 0x77)                  # codes saturate at 6
+    assert np.all(data[8:24] == 0x77)                  # codes saturate at 6
+    assert sc[2] == 0x7E
     # a small negative value that rounds to magnitude 0 gets code 0, not -0
     x = np.zeros(128, np.float32)
     x[0], x[1] = 6.0, -0.1                            # scale 1, y(-0.1) -> 0
