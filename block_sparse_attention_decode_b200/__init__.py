@@ -23,7 +23,7 @@ BLOCK, TOPK, HEAD_DIM, KV_HEADS, Q_HEADS = 128, 16, 128, 4, 64
 EXPORTED = [
     "msa_workspace_size", "msa_workspace_init", "msa_indexer_score", "msa_block_maxpool_topk",
     "msa_sparse_attn_decode", "msa_decode", "msa_get_last_error", "msa_debug_nvfp4_table",
-    "msa_status_string", "msa_decode_static",
+    "msa_status_string", "msa_decode_static", "msa_kv_insert",
 ]
 STATIC_WORKSPACE_BYTES = 16 << 20
 
@@ -78,6 +78,8 @@ def load() -> ctypes.CDLL:
     L.msa_decode.argtypes = [P(msa_cache), P(msa_seqs), vp, f32, vp, f32, f32, vp, vp, vp, sz, vp]
     L.msa_decode_static.restype = ctypes.c_int
     L.msa_decode_static.argtypes = [P(msa_cache), P(msa_seqs), vp, f32, vp, f32, f32, vp, vp, vp]
+    L.msa_kv_insert.restype = ctypes.c_int
+    L.msa_kv_insert.argtypes = [P(msa_cache), P(msa_seqs), vp, vp, vp, vp, sz, vp]
     L.msa_get_last_error.restype = ctypes.c_int
     L.msa_get_last_error.argtypes = [vp, vp, P(i32)]
     L.msa_debug_nvfp4_table.restype = ctypes.c_int
@@ -93,6 +95,8 @@ def status_string(status: int) -> str:
 
 
 def _ptr(t):
+    if t is not None and not t.is_cuda:
+        raise ValueError("libmsa takes CUDA tensors; got a tensor on %s" % t.device)
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
@@ -107,12 +111,21 @@ def _check(status: int, what: str):
         raise MsaError(status, what)
 
 
+def _device_tensors(ts):
+    """The library takes device pointers only: refuse host tensors here rather
+    than hand a kernel an address it cannot read."""
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libmsa takes CUDA tensors; got a tensor on %s" % t.device)
+
+
 class Cache:
     """Holds the cache tensors (keeps them alive) and their C description."""
 
     def __init__(self, idx_data, idx_scale, k_data, k_scale, v_data, v_scale,
                  s_idx: float, s_k: float, s_v: float):
         self.tensors = (idx_data, idx_scale, k_data, k_scale, v_data, v_scale)
+        _device_tensors(self.tensors)
         self.c = msa_cache(
             idx_data=idx_data.data_ptr(),
             idx_scale=idx_scale.data_ptr() if idx_scale is not None else None,
@@ -127,6 +140,7 @@ class Seqs:
 
     def __init__(self, seq_lens, q_tokens: int, max_pages: int, page_table=None):
         self.tensors = (seq_lens, page_table)
+        _device_tensors(self.tensors)
         self.c = msa_seqs(page_table=page_table.data_ptr() if page_table is not None else None,
                           seq_lens=seq_lens.data_ptr(), batch=int(seq_lens.shape[0]),
                           q_tokens=int(q_tokens), max_pages=int(max_pages))
@@ -198,6 +212,15 @@ def msa_decode_static(cache: Cache, seqs: Seqs, qi, s_qi: float, q, s_q: float,
     _check(load().msa_decode_static(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi), s_qi,
                                     _ptr(q), s_q, softmax_scale, _ptr(out), _ptr(sel_out),
                                     _stream(stream)), "msa_decode_static")
+
+
+def msa_kv_insert(cache: Cache, seqs: Seqs, k_new, v_new, idx_new, ws, stream=None):
+    """Quantise the new tokens (bf16 tensors [B][T][4][128], [B][T][4][128],
+    [B][T][128]) into the cache the descriptor points to."""
+    for x in (k_new, v_new, idx_new):
+        assert x.dtype == torch.bfloat16 and x.is_contiguous()
+    _check(load().msa_kv_insert(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(k_new), _ptr(v_new),
+                                _ptr(idx_new), _ptr(ws), ws.numel(), _stream(stream)), "msa_kv_insert")
 
 
 def msa_get_last_error(ws, stream=None):

@@ -16,7 +16,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmsa.so")
-SOURCES = ["msa_api.cu", "msa_indexer.cu", "msa_topk.cu", "msa_attn.cu", "msa_static.cu"]
+SOURCES = ["msa_api.cu", "msa_indexer.cu", "msa_topk.cu", "msa_attn.cu", "msa_static.cu",
+           "msa_insert.cu"]
 HEADERS = ["msa_device.cuh", "msa_internal.h"]
 
 NVCC_FLAGS = [

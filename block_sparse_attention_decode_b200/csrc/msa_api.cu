@@ -294,6 +294,40 @@ msa_status msa_decode(const msa_cache* cache, const msa_seqs* seqs, const uint8_
   return run_attn(cache, seqs, q, s_q, sel, softmax_scale, out, ws, L, s);
 }
 
+msa_status msa_kv_insert(const msa_cache* cache, const msa_seqs* seqs, const uint16_t* k_new,
+                         const uint16_t* v_new, const uint16_t* idx_new, void* ws, size_t ws_bytes,
+                         msa_stream_t stream) {
+  if (!seqs_ok(seqs)) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_cache(cache, true, true);
+  if (st != MSA_OK) return st;
+  if (!k_new || !aligned16(k_new) || !v_new || !aligned16(v_new) || !idx_new || !aligned16(idx_new))
+    return MSA_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  InsArgs a{};
+  a.idx_data = const_cast<uint8_t*>(cache->idx_data);
+  a.idx_scale = const_cast<uint8_t*>(cache->idx_scale);
+  a.k_data = const_cast<uint8_t*>(cache->k_data);
+  a.k_scale = const_cast<uint8_t*>(cache->k_scale);
+  a.v_data = const_cast<uint8_t*>(cache->v_data);
+  a.v_scale = const_cast<uint8_t*>(cache->v_scale);
+  a.page_table = seqs->page_table;
+  a.seq_lens = seqs->seq_lens;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.idx_new = idx_new;
+  a.flags = at<Flags>(ws, L.flags);
+  a.s_idx = cache->s_idx;
+  a.s_k = cache->s_k;
+  a.s_v = cache->s_v;
+  a.B = seqs->batch;
+  a.T = seqs->q_tokens;
+  a.max_pages = seqs->max_pages;
+  a.num_pages = cache->num_pages;
+  a.idx_fp8 = cache->idx_dtype == MSA_IDX_FP8;
+  return cuda_status(launch_insert(a, (cudaStream_t)stream));
+}
+
 msa_status msa_get_last_error(void* ws, msa_stream_t stream, int32_t* detail) {
   if (!ws) return MSA_ERR_WORKSPACE;
   const cudaStream_t s = (cudaStream_t)stream;

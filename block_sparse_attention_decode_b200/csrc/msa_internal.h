@@ -77,6 +77,19 @@ size_t attn_smem_bytes();
 int attn_splits(long long rows, int num_sms);
 cudaError_t launch_attn(const AttnArgs& a, int num_sms, cudaStream_t st);
 
+// Quantise the new tokens into the cache (msa_kv_insert).
+struct InsArgs {
+  uint8_t *idx_data, *idx_scale, *k_data, *k_scale, *v_data, *v_scale;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const uint16_t *k_new, *v_new;   // bf16 [B][T][4][128]
+  const uint16_t* idx_new;         // bf16 [B][T][128]
+  Flags* flags;
+  float s_idx, s_k, s_v;
+  int B, T, max_pages, num_pages, idx_fp8;
+};
+cudaError_t launch_insert(const InsArgs& a, cudaStream_t st);
+
 // The kernels' NVFP4 -> E4M3 table for all (scale, code) pairs.
 cudaError_t launch_nvfp4_table(uint8_t* out, cudaStream_t st);
 

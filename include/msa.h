@@ -169,6 +169,28 @@ MSA_API msa_status msa_decode(const msa_cache* cache, const msa_seqs* seqs,
                       float softmax_scale, uint16_t* out, int32_t* sel_out,
                       void* ws, size_t ws_bytes, msa_stream_t stream);
 
+/* Write the new tokens into the cache: for every sequence b, the q_tokens
+ * tokens at positions seq_lens[b]-q_tokens .. seq_lens[b]-1 (the same
+ * tokens msa_decode treats as the queries' own) are quantised and stored at
+ * their page (page_table, or b*max_pages + block when it is NULL) and slot
+ * ([post, "What is new in the MiniMax-M3.1 architecture"]: NVFP4 KV cache
+ * for the indexer and the attention; [post, "QKV GEMM + norm + RoPE + KV
+ * insert fusion"] names the insertion).
+ *   k_new, v_new: device bf16 [B][T][4][128] (per KV head); idx_new: device
+ *   bf16 [B][T][128] (the shared index-key head); all 16-byte aligned.
+ *   NVFP4 rows: per 16 elements the scale byte is E4M3 (nearest-even,
+ *   saturating) of amax/(6*s_t), each code the nearest E2M1 value of
+ *   x/(scale*s_t) (ties to the even code, saturating at 6), s_t = the
+ *   cache's s_k, s_v or s_idx; FP8 index keys are E4M3 of x/s_idx.
+ * The cache buffers are written through the descriptor's pointers (they
+ * must be writable device memory); nothing else in the cache changes.
+ * Pages outside the pool or invalid lengths are reported in the workspace
+ * (MSA_ERR_DEVICE_BOUNDS via msa_get_last_error) and those rows skipped. */
+MSA_API msa_status msa_kv_insert(const msa_cache* cache, const msa_seqs* seqs,
+                                 const uint16_t* k_new, const uint16_t* v_new,
+                                 const uint16_t* idx_new, void* ws, size_t ws_bytes,
+                                 msa_stream_t stream);
+
 /* Synchronise `stream`, return the first device-side error recorded in the
  * workspace since the last call (MSA_OK if none) and clear it.
  * detail (optional) receives the offending value (page id, block id, ...). */

@@ -124,3 +124,27 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(msa, "_lib", None)
     with pytest.raises(ImportError):
         msa.load()
+
+
+def test_kv_insert_host_checks(lib):
+    s = _seqs()
+    c = _cache()
+    ws = FAKE
+    # null inputs, then a workspace that is too small: rejected before any launch
+    st = lib.msa_kv_insert(ctypes.byref(c), ctypes.byref(s), None, ctypes.c_void_p(FAKE),
+                           ctypes.c_void_p(FAKE), ctypes.c_void_p(ws), 1 << 30, None)
+    assert st == msa.MSA_ERR_INVALID_ARG
+    st = lib.msa_kv_insert(ctypes.byref(c), ctypes.byref(s), ctypes.c_void_p(FAKE + 8),
+                           ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(ws), 1 << 30, None)
+    assert st == msa.MSA_ERR_INVALID_ARG     # misaligned
+    st = lib.msa_kv_insert(ctypes.byref(c), ctypes.byref(s), ctypes.c_void_p(FAKE),
+                           ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(ws), 16, None)
+    assert st == msa.MSA_ERR_WORKSPACE
+
+
+def test_binding_refuses_host_tensors(lib):
+    t = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        msa.Cache(t, t, t, t, t, t, 1.0, 1.0, 1.0)
+    with pytest.raises(ValueError):
+        msa.Seqs(torch.zeros(2, dtype=torch.int32), 1, 4)
