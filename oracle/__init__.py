@@ -51,7 +51,7 @@ class _Cache(ctypes.Structure):
         ("k_data", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
         ("v_data", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
         ("s_idx", ctypes.c_double), ("s_k", ctypes.c_double), ("s_v", ctypes.c_double),
-        ("num_pages", ctypes.c_int64), ("idx_fp8", ctypes.c_int),
+        ("num_pages", ctypes.c_int64), ("idx_mode", ctypes.c_int),
         ("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int64),
         ("seq_lens", ctypes.c_void_p), ("batch", ctypes.c_int), ("q_tokens", ctypes.c_int),
     ]
@@ -176,6 +176,7 @@ class Cache:
     max_pages: int
     seq_lens: np.ndarray           # int32 [B]
     q_tokens: int
+    idx_exact: bool = False        # NVFP4 index keys scored at their exact value (no E4M3 re-rounding)
 
     def _c(self) -> _Cache:
         arrs = [self.idx_data, self.k_data, self.k_scale, self.v_data, self.v_scale, self.seq_lens]
@@ -188,7 +189,7 @@ class Cache:
         c.v_data, c.v_scale = self.v_data.ctypes.data, self.v_scale.ctypes.data
         c.s_idx, c.s_k, c.s_v = float(self.s_idx), float(self.s_k), float(self.s_v)
         c.num_pages = int(self.k_data.shape[0])
-        c.idx_fp8 = 1 if self.idx_scale is None else 0
+        c.idx_mode = 1 if self.idx_scale is None else (2 if self.idx_exact else 0)
         c.page_table = self.page_table.ctypes.data if self.page_table is not None else None
         c.max_pages = int(self.max_pages)
         c.seq_lens = self.seq_lens.ctypes.data

@@ -134,7 +134,8 @@ typedef struct {
     const uint8_t *k_data, *k_scale, *v_data, *v_scale;
     double s_idx, s_k, s_v;
     int64_t num_pages;
-    int idx_fp8;                             /* 0: NVFP4 index keys, 1: FP8 */
+    int idx_mode;                            /* 0: NVFP4 index keys, 1: FP8,
+                                                2: NVFP4 scored at exact value */
     const int32_t* page_table;               /* [B][max_pages] or NULL */
     int64_t max_pages;
     const int32_t* seq_lens;                 /* [B] */
@@ -152,15 +153,23 @@ static int64_t page_of(const orc_cache* c, int b, int64_t blk)
     return p;
 }
 
-/* Index key of logical token j of sequence b (no tensor scale). */
+/* Index key of logical token j of sequence b (no tensor scale).
+ * Mode 2 is the exact variant of [post, "NVIDIA Rubin optimized MSA"]: the
+ * NVFP4 keys are converted to FP16 and scored with an FP16 MMA, so the scores
+ * carry no E4M3 re-rounding; e2m1 * e4m3 is exact in FP16 (at most 5
+ * significant bits, magnitude 2^-10 .. 2688), hence the key is that product. */
 static int index_key(const orc_cache* c, int b, int64_t j, double* v)
 {
     int64_t p = page_of(c, b, j / ORC_BLOCK);
     int64_t r = j % ORC_BLOCK;
     if (p < 0) return -1;
-    if (c->idx_fp8) {
+    if (c->idx_mode == 1) {
         const uint8_t* row = c->idx_data + (p * ORC_BLOCK + r) * ORC_D;
         for (int d = 0; d < ORC_D; ++d) v[d] = orc_e4m3(row[d]);
+    } else if (c->idx_mode == 2) {
+        const uint8_t* row = c->idx_data + (p * ORC_BLOCK + r) * 64;
+        const uint8_t* sc = c->idx_scale + (p * ORC_BLOCK + r) * 8;
+        for (int d = 0; d < ORC_D; ++d) v[d] = orc_e2m1(nib(row, d)) * orc_e4m3(sc[d / 16]);
     } else {
         decode_nvfp4_row(c->idx_data + (p * ORC_BLOCK + r) * 64,
                          c->idx_scale + (p * ORC_BLOCK + r) * 8, v);
@@ -554,7 +563,7 @@ int orc_kv_insert(const orc_cache* c, const float* k_new, const float* v_new,
             }
             {
                 const int64_t r = p * ORC_BLOCK + slot;
-                if (c->idx_fp8)
+                if (c->idx_mode == 1)
                     orc_fp8_encode_row(idx_new + tok * ORC_D, s_idx, (uint8_t*)c->idx_data + r * 128);
                 else
                     orc_nvfp4_encode_row(idx_new + tok * ORC_D, s_idx, (uint8_t*)c->idx_data + r * 64,
