@@ -88,6 +88,8 @@ KERNEL_SOURCES = {
     "attention": ["block_sparse_attention_decode_b200/csrc/msa_attn.cu",
                   "block_sparse_attention_decode_b200/csrc/msa_device.cuh"],
     "topk": ["block_sparse_attention_decode_b200/csrc/msa_topk.cu"],
+    "indexer_exact": ["block_sparse_attention_decode_b200/csrc/msa_indexer.cu",
+                      "block_sparse_attention_decode_b200/csrc/msa_device.cuh"],
 }
 
 
@@ -338,6 +340,34 @@ def run_gpu(args, rank, world, local_rank):
     achieved = kernel_bytes[dom] / (per[dom] * 1e-3) / 1e9
     traffic = dram_traffic(dom, name)
 
+    # ---- the exact index-score variant (MSA_IDX_NVFP4_EXACT: the same NVFP4
+    # index keys scored at their exact value with FP16 MMA), timed like the
+    # indexer above on the same cache
+    idx_exact = None
+    if not w.idx_fp8:
+        cache_x = msa.Cache(w.idx_data, w.idx_scale, w.k_data, w.k_scale, w.v_data, w.v_scale,
+                            w.s_idx, w.s_k, w.s_v, idx_exact=True)
+        for _ in range(3):
+            msa.msa_indexer_score(cache_x, seqs, w.qi, w.s_qi, None, bscores, ws, stream)
+        evx = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for e0, e1 in evx:
+            flush.fill_(1)
+            e0.record(stream)
+            msa.msa_indexer_score(cache_x, seqs, w.qi, w.s_qi, None, bscores, ws, stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        st, detail = msa.msa_get_last_error(ws)
+        if st != msa.MSA_OK:
+            raise RuntimeError("device error %d (%d) in the exact indexer" % (st, detail))
+        x_ms = sum(a.elapsed_time(b) for a, b in evx) / args.steps
+        x_gbs = kernel_bytes["indexer"] / (x_ms * 1e-3) / 1e9
+        idx_exact = {"ms": x_ms, "achieved_gbs": x_gbs, "frac": x_gbs / peak,
+                     "bytes_per_launch": kernel_bytes["indexer"],
+                     "traffic": dram_traffic("indexer_exact", name),
+                     "note": "NVFP4 index keys decoded exactly to FP16 and scored with FP16 "
+                             "MMA (no E4M3 re-rounding); not part of the timed step"}
+
     # ---- the step before the path: writing the step's B*T new tokens into
     # the cache (their K, V and index key, from bf16), timed on its own into
     # a scratch copy of the pages it writes so the benchmark cache is unchanged
@@ -448,6 +478,7 @@ def run_gpu(args, rank, world, local_rank):
                          "algorithmic_bytes_per_launch": kernel_bytes[dom],
                          "peak_source": peak_src},
             "kernel_ms": per,
+            "indexer_exact": idx_exact,
             "kv_insert": {"ms": ins_ms, "tokens": B * T, "bytes": ins_bytes,
                           "gbs": ins_bytes / (ins_ms * 1e-3) / 1e9,
                           "note": "writing the step's new tokens into the cache (not part of the "

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA = 0, 1, 2, 3
 MSA_ERR_DEVICE_BOUNDS, MSA_ERR_TIMEOUT, MSA_ERR_WORKSPACE = 4, 5, 6
-MSA_IDX_NVFP4, MSA_IDX_FP8 = 0, 1
+MSA_IDX_NVFP4, MSA_IDX_FP8, MSA_IDX_NVFP4_EXACT = 0, 1, 2
 BLOCK, TOPK, HEAD_DIM, KV_HEADS, Q_HEADS = 128, 16, 128, 4, 64
 
 EXPORTED = [
@@ -123,16 +123,22 @@ class Cache:
     """Holds the cache tensors (keeps them alive) and their C description."""
 
     def __init__(self, idx_data, idx_scale, k_data, k_scale, v_data, v_scale,
-                 s_idx: float, s_k: float, s_v: float):
+                 s_idx: float, s_k: float, s_v: float, idx_exact: bool = False):
+        """idx_scale None = FP8 index keys; idx_exact = score NVFP4 index keys
+        at their exact value (MSA_IDX_NVFP4_EXACT)."""
         self.tensors = (idx_data, idx_scale, k_data, k_scale, v_data, v_scale)
         _device_tensors(self.tensors)
+        if idx_scale is None:
+            dtype = MSA_IDX_FP8
+        else:
+            dtype = MSA_IDX_NVFP4_EXACT if idx_exact else MSA_IDX_NVFP4
         self.c = msa_cache(
             idx_data=idx_data.data_ptr(),
             idx_scale=idx_scale.data_ptr() if idx_scale is not None else None,
             k_data=k_data.data_ptr(), k_scale=k_scale.data_ptr(),
             v_data=v_data.data_ptr(), v_scale=v_scale.data_ptr(),
             s_idx=s_idx, s_k=s_k, s_v=s_v, num_pages=int(k_data.shape[0]),
-            idx_dtype=MSA_IDX_FP8 if idx_scale is None else MSA_IDX_NVFP4)
+            idx_dtype=dtype)
 
 
 class Seqs:
@@ -152,7 +158,7 @@ class Seqs:
 
 def cache_of(w) -> Cache:
     return Cache(w.idx_data, w.idx_scale, w.k_data, w.k_scale, w.v_data, w.v_scale,
-                 w.s_idx, w.s_k, w.s_v)
+                 w.s_idx, w.s_k, w.s_v, idx_exact=w.idx_exact)
 
 
 def seqs_of(w) -> Seqs:

@@ -62,9 +62,11 @@ msa_status check_cache(const msa_cache* c, bool need_index, bool need_kv) {
   if (!c) return MSA_ERR_INVALID_ARG;
   if (c->num_pages < 1) return MSA_ERR_INVALID_ARG;
   if (need_index) {
-    if (c->idx_dtype != MSA_IDX_NVFP4 && c->idx_dtype != MSA_IDX_FP8) return MSA_ERR_INVALID_ARG;
+    if (c->idx_dtype != MSA_IDX_NVFP4 && c->idx_dtype != MSA_IDX_FP8 &&
+        c->idx_dtype != MSA_IDX_NVFP4_EXACT)
+      return MSA_ERR_INVALID_ARG;
     if (!c->idx_data || !aligned16(c->idx_data)) return MSA_ERR_INVALID_ARG;
-    if (c->idx_dtype == MSA_IDX_NVFP4 && (!c->idx_scale || !aligned16(c->idx_scale)))
+    if (c->idx_dtype != MSA_IDX_FP8 && (!c->idx_scale || !aligned16(c->idx_scale)))
       return MSA_ERR_INVALID_ARG;
     if (!good_scale(c->s_idx)) return MSA_ERR_INVALID_ARG;
   }
@@ -110,7 +112,8 @@ msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi,
   a.T = s->q_tokens;
   a.max_pages = s->max_pages;
   a.num_pages = c->num_pages;
-  return cuda_status(launch_indexer(a, c->idx_dtype == MSA_IDX_FP8, device_sms(), st));
+  const int mode = fp8 ? kIdxFp8 : (c->idx_dtype == MSA_IDX_NVFP4_EXACT ? kIdxF16 : kIdxNvfp4);
+  return cuda_status(launch_indexer(a, mode, device_sms(), st));
 }
 
 msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, float s_q,

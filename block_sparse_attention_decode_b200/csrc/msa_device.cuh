@@ -66,76 +66,6 @@ __device__ __forceinline__ void build_nvfp4_lut(uint2* lut, int tid, int nthread
   }
 }
 
-// Decode 8 codes (one 32-bit word: element n in nibble n) with table row r.
-// o0 = elements 0..3, o1 = elements 4..7 (E4M3 bytes, element order kept).
-__device__ __forceinline__ void dq8(uint32_t w, uint2 r, uint32_t& o0, uint32_t& o1) {
-  const uint32_t mag = w & 0x77777777u;
-  const uint32_t sgn = (w >> 3) & 0x11111111u;
-  o0 = __byte_perm(r.x, r.y, mag) ^ __byte_perm(0x00008000u, 0u, sgn);
-  o1 = __byte_perm(r.x, r.y, mag >> 16) ^ __byte_perm(0x00008000u, 0u, sgn >> 16);
-}
-
-// Decode 32 consecutive elements (16 code bytes, 2 scale bytes) into 8 words:
-// out[m] = elements 4m..4m+3.
-__device__ __forceinline__ void dq32(const uint2* lut, uint4 c, uint32_t sc2, uint32_t (&out)[8]) {
-  const uint2 r0 = lut[sc2 & 0xFFu];
-  const uint2 r1 = lut[(sc2 >> 8) & 0xFFu];
-  dq8(c.x, r0, out[0], out[1]);
-  dq8(c.y, r0, out[2], out[3]);
-  dq8(c.z, r1, out[4], out[5]);
-  dq8(c.w, r1, out[6], out[7]);
-}
-
-// ------------------------------------------------------------ FP8 MMA -----
-// D(16x8 f32) += A(16x32 e4m3, row) * B(32x8 e4m3, col).
-//   a0:(row g, k 4t..4t+3) a1:(row g+8, same k) a2:(row g, k 16+4t..) a3:(row g+8, ..)
-//   b0:(k 4t..4t+3, col g)  b1:(k 16+4t.., col g)
-//   d0:(row g, col 2t) d1:(row g, col 2t+1) d2:(row g+8, col 2t) d3:(row g+8, col 2t+1)
-// with g = lane/4, t = lane%4.
-__device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Two fp32 -> packed E4M3x2 (lo in the low byte), RNE, satfinite.
-__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
-  return pack_e4m3x2(a, b) | (pack_e4m3x2(c, d) << 16);
-}
-
-// Two fp32 values as a sum of two E4M3 terms: hi = E4M3(v), lo = E4M3(v - hi)
-// with the remainder formed in f16 (v and hi are exact in f16 to 2^-11).
-// hi + lo carries v to about 8 significant bits instead of E4M3's 4.
-__device__ __forceinline__ void split_e4m3x2(float lo_v, float hi_v, uint32_t& h, uint32_t& l) {
-  uint16_t hh, ll;
-  uint32_t p16, h16, r16;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(hh) : "f"(hi_v), "f"(lo_v));
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(p16) : "f"(hi_v), "f"(lo_v));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(h16) : "h"(hh));
-  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(r16) : "r"(p16), "r"(h16));
-  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;\n" : "=h"(ll) : "r"(r16));
-  h = hh;
-  l = ll;
-}
-
-__device__ __forceinline__ void split_e4m3x4(float a, float b, float c, float d, uint32_t& h,
-                                             uint32_t& l) {
-  uint32_t h0, l0, h1, l1;
-  split_e4m3x2(a, b, h0, l0);
-  split_e4m3x2(c, d, h1, l1);
-  h = h0 | (h1 << 16);
-  l = l0 | (l1 << 16);
-}
-
 // -------------------------------------------- mbarrier + bulk async copy --
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -195,19 +125,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 
 __device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
-__device__ __forceinline__ uint32_t lds16(const void* p) {
-  return *reinterpret_cast<const uint16_t*>(p);
-}
-
 // Order-preserving map float -> uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ float key_float(uint32_t k) {
-  const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
-  return __uint_as_float(u);
 }
 
 }  // namespace msa
@@ -257,16 +178,6 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, one K = 32 slice (E4M3).
-__device__ __forceinline__ void tc_mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrive on *bar once every tcgen05 operation issued so far by this thread completes.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
@@ -278,24 +189,6 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 }
 
-// Warp-wide: lane l reads TMEM lane (taddr.lane + l), 32 consecutive columns.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   uint32_t r[8];
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
@@ -305,20 +198,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
                : "memory");
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Max of a float over the 32 lanes of the warp (result in every lane).
@@ -364,12 +243,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
-// NVFP4 -> E4M3 split by sign for 8 codes (element n in nibble n):
-// pos = E4M3(|value|) of the positive elements (0 elsewhere), neg likewise for
-// the negative ones, so value = pos - neg.  `r` is the table row of |scale|
-// (all bytes < 0x80); a selector nibble with its top bit set makes prmt
-// return 0x00 (the sign of a non-negative byte), which drops the elements of
-// the other sign.  flip = 0x88888888 when the block scale is negative.
 // PTX prmt in its default mode (the top bit of each selector nibble
 // replicates the sign of the selected byte, unlike __byte_perm).
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -403,6 +276,12 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// NVFP4 -> E4M3 split by sign for 8 codes (element n in nibble n):
+// pos = E4M3(|value|) of the positive elements (0 elsewhere), neg likewise for
+// the negative ones, so value = pos - neg.  `r` is the table row of |scale|
+// (all bytes < 0x80); a selector nibble with its top bit set makes prmt
+// return 0x00 (the sign of a non-negative byte), which drops the elements of
+// the other sign.  flip = 0x88888888 when the block scale is negative.
 __device__ __forceinline__ void dq8_split(uint32_t w, uint2 r, uint32_t flip, uint32_t& p0,
                                           uint32_t& p1, uint32_t& n0, uint32_t& n1) {
   const uint32_t wp = w ^ flip;
@@ -424,34 +303,66 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
   return d;
 }
 
-// fp32 pair -> f16x2, lo in the low half (round to nearest even).
-__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+// ----------------------------------------------- NVFP4 -> FP16 (exact) ----
+// e2m1 x e4m3 has at most 5 significant bits and lies in [2^-10, 2688], so
+// it is exact in FP16: no re-rounding ([post, "NVIDIA Rubin optimized MSA"]
+// scores the index keys this way).
+
+// Two E2M1 codes (the low byte of b, element 0 in the low nibble) -> f16x2
+// (element 0 in the low half), unscaled.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t b) {
   uint32_t d;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(d) : "f"(hi), "f"(lo));
+  asm("{\n.reg .b8 c, z;\nmov.b16 {c, z}, %1;\ncvt.rn.f16x2.e2m1x2 %0, c;\n}\n"
+      : "=r"(d)
+      : "h"((uint16_t)(b & 0xFFFFu)));
   return d;
 }
 
-// D(16x8 f32) += A(16x16 f16, row) * B(16x8 f16, col).
-//   a0:(row g, k 2t..2t+1) a1:(row g+8, same) a2:(row g, k 2t+8..) a3:(row g+8, k 2t+8..)
-//   b0:(k 2t..2t+1, col g) b1:(k 2t+8..2t+9, col g); d as in mma_e4m3.
-__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                        uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+// The 8 codes of w (element n in nibble n) -> 4 f16x2 words o[0..3], o[m] =
+// elements 2m (low half) and 2m+1, unscaled.
+// Each byte is first moved to the bottom of a register of its own (prmt):
+// unpacking the four bytes of one register through nested vector moves
+// (32 -> 2 x 16 -> 4 x 8 bits) gave byte 0 in place of byte 2 on sm_100a.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t* o) {
+  o[0] = e2m1x2_to_f16x2(prmt(w, 0u, 0x4440u));
+  o[1] = e2m1x2_to_f16x2(prmt(w, 0u, 0x4441u));
+  o[2] = e2m1x2_to_f16x2(prmt(w, 0u, 0x4442u));
+  o[3] = e2m1x2_to_f16x2(prmt(w, 0u, 0x4443u));
 }
 
-// Four 8x8 b16 matrices, transposed: lane 8i+j gives the address of row j of
-// matrix i; register i receives matrix i with thread (g, t) holding column g,
-// rows 2t and 2t+1.
-__device__ __forceinline__ void ldsm_x4_trans(const void* row_addr, uint32_t& r0, uint32_t& r1,
-                                              uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(smem_u32(row_addr))
-               : "memory");
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Warp-wide: lane l writes 16 consecutive 32-bit columns of TMEM lane (taddr.lane + l).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+// Instruction descriptor: kind::f16, A = B = f16 (format code 0), fp32
+// accumulate, both operands K-major, shape M x N.  The fields sit where they
+// do for kind::f8f6f4, where format code 0 names E4M3.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, one K = 16 slice of FP16.  A: 8
+// consecutive 32-bit TMEM columns = 16 K-elements of each row.
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // Warp-wide 16x256b TMEM load, R = 1, 2 or 4 repetitions along columns:

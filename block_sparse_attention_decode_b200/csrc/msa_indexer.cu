@@ -7,8 +7,8 @@
 // Per page (= one 128-token block) the scores are one dense FP8 contraction
 //   D[128 keys x NQ queries] = K_page[128 x 128] * Qi[NQ x 128]^T
 // with the keys as the M side (the block max is a reduction over TMEM
-// lanes) and a chunk of NQ index queries (T tokens x 4 groups, padded to a
-// multiple of 8) as the N side.
+// lanes) and a chunk of NQ index queries (T tokens x 4 groups, padded to
+// 16, 32, 64, 128 or 256) as the N side.
 //
 // Work split: the pages of all sequences form one flat list, cut into chunks
 // of kChunkPages; a work item is (query tile of NQ index queries, chunk).
@@ -38,6 +38,16 @@
 //     maxima of a quarter of the columns and writes those block scores.
 // Every wait is a bounded mbarrier wait; on a timeout a thread records
 // MSA_ERR_TIMEOUT and leaves its loop, and TMEM is freed before exit.
+//
+// Modes (the template parameter MODE):
+//   kIdxNvfp4  NVFP4 keys re-rounded to E4M3, FP8 MMA (the sign split above);
+//   kIdxFp8    E4M3 keys, copied to TMEM as they are;
+//   kIdxF16    NVFP4 keys decoded exactly to FP16 (e2m1 x scale needs no
+//              rounding in FP16) and scored with FP16 MMA against the index
+//              queries widened to FP16 -- the exact scores of [post, "NVIDIA
+//              Rubin optimized MSA"].  One A buffer holds the 128 FP16 values
+//              of each row in 64 columns; the queries take two 128-byte
+//              swizzled K-halves in shared memory; 8 MMAs of K = 16 per page.
 #include "msa_internal.h"
 
 namespace msa {
@@ -47,7 +57,7 @@ constexpr int kIdxEpilogue = 4;             // per group: one per TMEM lane quar
 constexpr int kIdxEpiWarp0 = 4;             // two groups: even and odd pages
 constexpr int kIdxProducerWarp = 12;
 constexpr int kIdxMmaWarp = 13;
-constexpr int kABufCols = 64;               // TMEM columns of one A buffer (K+ | K-)
+constexpr int kABufCols = 64;               // TMEM columns of one A buffer (K+ | K-, or FP16)
 constexpr int kACols = 2 * kABufCols;       // two A buffers
 
 enum : int { kPageLoad = 0, kPageMasked = 1, kPageBad = 2, kPageEnd = 3 };
@@ -62,11 +72,14 @@ __host__ __device__ inline int raw_stage_stride(bool fp8idx) {
   return fp8idx ? kBlock * kDim : ((kPageCodes + kPageScales + 1023) / 1024) * 1024;
 }
 
-__host__ __device__ inline IdxLayout idx_layout(int nq, bool fp8idx, int batch) {
+// Bytes of one query row in shared memory: E4M3, or two 128-byte K-halves of FP16.
+__host__ __device__ constexpr int q_row_bytes(int mode) { return mode == kIdxF16 ? 256 : 128; }
+
+__host__ __device__ inline IdxLayout idx_layout(int nq, int mode, int batch) {
   IdxLayout L;
   int off = 0;
-  L.qbuf = off;    off += 2 * nq * 128;                   // nq % 8 == 0 -> 1024-aligned
-  L.raw_stride = raw_stage_stride(fp8idx);
+  L.qbuf = off;    off += 2 * nq * q_row_bytes(mode);     // nq % 8 == 0 -> 1024-aligned
+  L.raw_stride = raw_stage_stride(mode == kIdxFp8);
   L.raw = off;     off += kIdxRawStages * L.raw_stride;
   L.lut = off;     off += 256 * 8;
   L.red = off;     off += 2 * kIdxEpilogue * nq * 4;          // [group][quarter][nq]
@@ -81,9 +94,11 @@ __host__ __device__ inline IdxLayout idx_layout(int nq, bool fp8idx, int batch) 
   return L;
 }
 
+// N of the MMA: with A in tensor memory and M = 128, N is a multiple of 16
+// from 16 to 256 (the tcgen05.mma shape table), so one query token's 4 index
+// queries are padded to 16.
 int idx_nq(int T) {
   const int nq = kG * T;
-  if (nq <= 8) return 8;
   if (nq <= 16) return 16;
   if (nq <= 32) return 32;
   if (nq <= 64) return 64;
@@ -91,8 +106,8 @@ int idx_nq(int T) {
   return 256;
 }
 
-size_t indexer_smem_bytes(bool fp8idx, int batch, int T) {
-  return (size_t)idx_layout(idx_nq(T), fp8idx, batch).total;
+size_t indexer_smem_bytes(int mode, int batch, int T) {
+  return (size_t)idx_layout(idx_nq(T), mode, batch).total;
 }
 
 __host__ __device__ constexpr int pow2_at_least(int x) {
@@ -138,14 +153,17 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
 
 __device__ __forceinline__ void sts128(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
-template <int NQ, bool FP8IDX>
+template <int NQ, int MODE>
 __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_constant__ IdxArgs a) {
+  constexpr bool FP8IDX = MODE == kIdxFp8;
+  constexpr bool F16 = MODE == kIdxF16;
+  constexpr int kQRow = q_row_bytes(MODE);
   constexpr int kND = NQ <= 64 ? 2 : 1;                      // accumulator buffers
   constexpr int kCols = pow2_at_least(kACols + kND * NQ);    // TMEM columns
   constexpr int kChunk = NQ < 32 ? NQ : (NQ >= 128 ? 16 : 32);   // columns per TMEM load
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
-  const IdxLayout Ly = idx_layout(NQ, FP8IDX, a.B);
+  const IdxLayout Ly = idx_layout(NQ, MODE, a.B);
   uint8_t* qbuf = smem + Ly.qbuf;
   uint8_t* raw = smem + Ly.raw;
   uint2* lut = reinterpret_cast<uint2*>(smem + Ly.lut);
@@ -166,7 +184,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  if (!FP8IDX) build_nvfp4_lut(lut, tid, blockDim.x);
+  if (MODE == kIdxNvfp4) build_nvfp4_lut(lut, tid, blockDim.x);
   if (tid == 0) {
     for (int s = 0; s < kIdxRawStages; ++s) {
       mbar_init(&raw_full[s], 1);
@@ -269,12 +287,15 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   } else if (warp == kIdxMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(128, NQ);
+      constexpr uint32_t idesc = F16 ? idesc_f16_f32(128, NQ) : idesc_e4m3_f32(128, NQ);
       constexpr uint32_t idesc_neg = idesc | (1u << 13);     // negate A
-      // B descriptors of the two query buffers; a K = 32 slice starts 32
-      // bytes further (2 in the descriptor's 16-byte address units)
+      // B descriptors of the two query buffers; a K slice (32 E4M3 or 16
+      // FP16 values) starts 32 bytes further (2 in the descriptor's 16-byte
+      // address units); FP16 queries continue in a second 128-byte-wide tile
+      // NQ rows further for K >= 64.
       const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(qbuf));
-      const uint64_t bdesc1 = desc_kmajor_sw128(smem_u32(qbuf + NQ * 128));
+      const uint64_t bdesc1 = desc_kmajor_sw128(smem_u32(qbuf + NQ * kQRow));
+      constexpr uint64_t kHalf = (uint64_t)(NQ * 128 / 16);    // second K-half, descriptor units
       // Page k uses A buffer k % 2 and accumulator k % kND; with two
       // accumulators one commit (to acc_full[k % 2]) releases both.
       auto issue = [&](int k, int ab, int x, int& ends) -> bool {
@@ -287,9 +308,15 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           const uint32_t d = tmem + kACols + x * NQ;
           const uint32_t ta = tmem + ab * kABufCols;
           const uint64_t bd = tinfo[2 * ab + 1] ? bdesc1 : bdesc0;
+          if constexpr (F16) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc, kk > 0);
-          if (!FP8IDX) {
+            for (int kk = 0; kk < 8; ++kk)
+              tc_mma_f16_ts(d, ta + 8 * kk, bd + (kk >> 2) * kHalf + 2 * (kk & 3), idesc, kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc, kk > 0);
+          }
+          if (MODE == kIdxNvfp4) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 32 + 8 * kk, bd + 2 * kk, idesc_neg, 1);
           }
@@ -444,7 +471,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         // B operand: the index queries of tile ny of sequence nb, swizzled
         // (its previous user, an MMA of page k-2 or earlier, has completed:
         // the wait above).
-        uint8_t* qb = qbuf + qsel * NQ * 128;
+        uint8_t* qb = qbuf + qsel * NQ * kQRow;
         const int qbase = ny * NQ;
         for (int idx = warp * 32 + lane; idx < NQ * 8; idx += kIdxDecoders * 32) {
           const int nrow = idx / 8, c = idx % 8;
@@ -453,7 +480,20 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           if (t < a.T)
             v = *reinterpret_cast<const uint4*>(
                 a.qi + (((long long)nb * a.T + t) * kG + (qg & 3)) * kDim + 16 * c);
-          sts128(qb + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
+          if constexpr (F16) {
+            // dims 16c..16c+15 -> FP16 chunks 2c, 2c+1 of 8 dims: K-half c / 4,
+            // chunk positions (2c % 8, 2c % 8 + 1) ^ (row % 8) in its 128-byte row
+            const uint4 lo = make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
+                                        e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
+            const uint4 hi = make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
+                                        e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
+            uint8_t* rowp = qb + (c >> 2) * NQ * 128 + nrow * 128;
+            const int j = (2 * c) & 7;
+            sts128(rowp + ((j ^ (nrow & 7)) << 4), lo);
+            sts128(rowp + (((j + 1) ^ (nrow & 7)) << 4), hi);
+          } else {
+            sts128(qb + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
+          }
         }
         fence_async_smem();
       }
@@ -469,6 +509,25 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
             const uint4 x1 = lds128(rs + row * 128 + (((2 * c2 + 1) ^ (row & 7)) << 4));
             const uint32_t w8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
             tmem_st8(abase + 8 * c2, w8);
+          }
+        } else if constexpr (F16) {
+          // 64-byte code rows (64-byte swizzle, as below); chunk c = elements
+          // 32c..32c+31 under scale bytes 2c and 2c+1 -> FP16 columns 16c..16c+15
+          const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
+          const int sw = (row >> 1) & 3;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
+            const uint32_t s2 = e4m3x2_to_f16x2((c < 2 ? sc.x : sc.y) >> (16 * (c & 1)));
+            const uint32_t s_lo = prmt(s2, 0u, 0x1010u), s_hi = prmt(s2, 0u, 0x3232u);
+            uint32_t o[16];
+            e2m1x8_to_f16x2(w4.x, o + 0);
+            e2m1x8_to_f16x2(w4.y, o + 4);
+            e2m1x8_to_f16x2(w4.z, o + 8);
+            e2m1x8_to_f16x2(w4.w, o + 12);
+#pragma unroll
+            for (int m = 0; m < 16; ++m) o[m] = hmul2(o[m], m < 8 ? s_lo : s_hi);
+            tmem_st16(abase + 16 * c, o);
           }
         } else {
           // 64-byte code rows loaded with the 64-byte swizzle: chunk c of
@@ -533,10 +592,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   if (warp == kIdxMmaWarp) tmem_dealloc(tmem, kCols);
 }
 
-template <int NQ, bool FP8IDX>
+template <int NQ, int MODE>
 static cudaError_t launch_nq(const IdxArgs& a, int num_sms, cudaStream_t st) {
-  auto kern = indexer_kernel<NQ, FP8IDX>;
-  const size_t smem = (size_t)idx_layout(NQ, FP8IDX, a.B).total;
+  auto kern = indexer_kernel<NQ, MODE>;
+  const size_t smem = (size_t)idx_layout(NQ, MODE, a.B).total;
   static size_t configured = 0;
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -550,12 +609,14 @@ static cudaError_t launch_nq(const IdxArgs& a, int num_sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_indexer(const IdxArgs& a, bool fp8idx, int num_sms, cudaStream_t st) {
+cudaError_t launch_indexer(const IdxArgs& a, int mode, int num_sms, cudaStream_t st) {
   const int nq = idx_nq(a.T);
 #define MSA_IDX_CASE(NQV)                                                     \
-  if (nq == NQV)                                                              \
-    return fp8idx ? launch_nq<NQV, true>(a, num_sms, st) : launch_nq<NQV, false>(a, num_sms, st);
-  MSA_IDX_CASE(8)
+  if (nq == NQV) {                                                            \
+    if (mode == kIdxFp8) return launch_nq<NQV, kIdxFp8>(a, num_sms, st);      \
+    if (mode == kIdxF16) return launch_nq<NQV, kIdxF16>(a, num_sms, st);      \
+    return launch_nq<NQV, kIdxNvfp4>(a, num_sms, st);                         \
+  }
   MSA_IDX_CASE(16)
   MSA_IDX_CASE(32)
   MSA_IDX_CASE(64)

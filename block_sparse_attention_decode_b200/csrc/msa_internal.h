@@ -12,12 +12,15 @@
 namespace msa {
 
 constexpr int kIdxThreads = 14 * 32;    // 4 decoders, 8 epilogue warps, producer, MMA warp
+// Indexer arithmetic: NVFP4 keys re-rounded to E4M3 (FP8 MMA), E4M3 keys, or
+// NVFP4 keys decoded exactly to FP16 (FP16 MMA).
+enum : int { kIdxNvfp4 = 0, kIdxFp8 = 1, kIdxF16 = 2 };
 constexpr int kIdxRawStages = 6;         // raw index-key pages in flight per CTA
 
 struct IdxArgs {
   CUtensorMap tmap_idx;        // rows of idx_data: 64-byte rows (64B swizzle) or 128 (128B swizzle)
   const uint8_t* idx_data;     // NVFP4 codes [P][128][64] or FP8 keys [P][128][128]
-  const uint8_t* idx_scale;    // [P][128][8] (NVFP4 only)
+  const uint8_t* idx_scale;    // [P][128][8] (NVFP4 keys only)
   const int32_t* page_table;   // [B][max_pages] or null
   const int32_t* seq_lens;     // [B]
   const uint8_t* qi;           // [B][T][4][128] E4M3
@@ -29,9 +32,9 @@ struct IdxArgs {
   int B, T, max_pages, num_pages;
 };
 
-size_t indexer_smem_bytes(bool fp8idx, int batch, int T);
+size_t indexer_smem_bytes(int mode, int batch, int T);
 int idx_nq(int T);
-cudaError_t launch_indexer(const IdxArgs& a, bool fp8idx, int num_sms, cudaStream_t st);
+cudaError_t launch_indexer(const IdxArgs& a, int mode, int num_sms, cudaStream_t st);
 
 // CTAs of `kernel` resident per SM for `threads` threads and `smem` dynamic
 // shared memory (registers, shared memory, and `tmem_cols` of the 512 TMEM

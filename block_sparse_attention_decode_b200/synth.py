@@ -103,6 +103,7 @@ class Workload:
     s_qi: float = S_Q
     s_q: float = S_Q
     softmax_scale: float = D ** -0.5
+    idx_exact: bool = False         # score NVFP4 index keys exactly (no E4M3 re-rounding)
     meta: dict = field(default_factory=dict)
 
     @property
@@ -127,7 +128,8 @@ def _page_map(batch, nblk, max_pages, paged, seed, device):
 def make_workload(name: str, batch: int, seq_lens, q_tokens: int, *, paged: bool,
                   seed: int, device="cpu", idx_fp8: bool = False, max_pages: int | None = None,
                   plant_every: int = 0, scale_floor_byte: int = 0,
-                  neg_scale_frac: float = 0.0, chunk_pages: int = 2048) -> Workload:
+                  neg_scale_frac: float = 0.0, chunk_pages: int = 2048,
+                  idx_exact: bool = False) -> Workload:
     """Build a workload.  seq_lens counts the q_tokens new tokens (which are the
     last q_tokens positions of each sequence).
 
@@ -210,6 +212,8 @@ def make_workload(name: str, batch: int, seq_lens, q_tokens: int, *, paged: bool
             flip = torch.rand(t.shape, generator=gn, device=device) < neg_scale_frac
             t |= flip.to(torch.uint8) << 7
 
+    if idx_exact and idx_fp8:
+        raise ValueError("idx_exact applies to NVFP4 index keys")
     s_idx = S_Q if idx_fp8 else S_NVFP4
     return Workload(
         name=name, batch=batch, q_tokens=q_tokens,
@@ -218,7 +222,7 @@ def make_workload(name: str, batch: int, seq_lens, q_tokens: int, *, paged: bool
         idx_data=idx_data, idx_scale=idx_scale, k_data=k_data, k_scale=k_scale,
         v_data=v_data, v_scale=v_scale,
         qi=encode_fp8(qi_f, S_Q), q=encode_fp8(q_f, S_Q),
-        s_idx=s_idx, meta={"seed": seed, "paged": paged, "plant_every": plant_every,
+        s_idx=s_idx, idx_exact=idx_exact, meta={"seed": seed, "paged": paged, "plant_every": plant_every,
                            "scale_floor_byte": scale_floor_byte,
                            "neg_scale_frac": neg_scale_frac},
     )

@@ -43,6 +43,10 @@
  *   idx_data  [P][128][64]     NVFP4 index-key codes        (idx_dtype NVFP4)
  *   idx_scale [P][128][8]      NVFP4 index-key block scales
  *   idx_data  [P][128][128]    E4M3 index keys, idx_scale NULL (idx_dtype FP8)
+ *   (idx_dtype NVFP4_EXACT: the NVFP4 layout above, but the indexer scores
+ *   the keys at their exact value e2m1(code) * e4m3(scale) * s_idx, without
+ *   the E4M3 re-rounding -- the FP16 scoring of [post, "NVIDIA Rubin
+ *   optimized MSA"]; K and V are always decoded as above.)
  *   k_data, v_data   [P][4][128][64]  NVFP4 codes  (page, kv head, token)
  *   k_scale, v_scale [P][4][128][8]   E4M3 block scales
  * Sequences: sequence b holds seq_lens[b] tokens, which INCLUDE its q_tokens
@@ -90,19 +94,25 @@ typedef enum {
     MSA_ERR_WORKSPACE = 6       /* workspace NULL or smaller than required       */
 } msa_status;
 
-enum { MSA_IDX_NVFP4 = 0, MSA_IDX_FP8 = 1 };
+/* Index-key format and scoring arithmetic (msa_cache.idx_dtype):
+ *   MSA_IDX_NVFP4        NVFP4 keys, re-rounded to E4M3, FP8 tensor-core MMA;
+ *   MSA_IDX_FP8          E4M3 keys, FP8 MMA;
+ *   MSA_IDX_NVFP4_EXACT  NVFP4 keys decoded exactly to FP16 and scored with
+ *                        FP16 MMA against the index queries widened to FP16
+ *                        (exact products, fp32 accumulation). */
+enum { MSA_IDX_NVFP4 = 0, MSA_IDX_FP8 = 1, MSA_IDX_NVFP4_EXACT = 2 };
 
 /* One layer's cache (device pointers, caller-owned). */
 typedef struct {
     const uint8_t* idx_data;
-    const uint8_t* idx_scale;   /* NULL for MSA_IDX_FP8 */
+    const uint8_t* idx_scale;   /* NULL for MSA_IDX_FP8, required otherwise */
     const uint8_t* k_data;
     const uint8_t* k_scale;
     const uint8_t* v_data;
     const uint8_t* v_scale;
     float s_idx, s_k, s_v;      /* per-tensor fp32 scales (> 0) */
     int32_t num_pages;          /* pages in each pool */
-    int32_t idx_dtype;          /* MSA_IDX_NVFP4 or MSA_IDX_FP8 */
+    int32_t idx_dtype;          /* MSA_IDX_NVFP4, MSA_IDX_FP8 or MSA_IDX_NVFP4_EXACT */
 } msa_cache;
 
 /* The batch of sequences of one decode step. */
@@ -132,7 +142,7 @@ MSA_API msa_status msa_workspace_init(void* ws, size_t ws_bytes, msa_stream_t st
  *   j > pos; entries of blocks i >= ceil(len/128) untouched.
  * block_scores: [B][T][4][max_pages] fp32; written for i < ceil(len/128);
  *   -inf where block i has no key visible to the query.
- * Index keys are NVFP4 or FP8 per cache->idx_dtype. */
+ * Index keys are NVFP4 or FP8, scored as cache->idx_dtype says. */
 MSA_API msa_status msa_indexer_score(const msa_cache* cache, const msa_seqs* seqs,
                              const uint8_t* qi, float s_qi,
                              float* token_scores, float* block_scores,

@@ -48,7 +48,7 @@ def host_cache(w, seq_ids=None) -> tuple[oracle.Cache, list[int]]:
                      v_scale=take(w.v_scale), s_idx=w.s_idx, s_k=w.s_k, s_v=w.s_v,
                      page_table=new_pt, max_pages=max(nblk),
                      seq_lens=np.ascontiguousarray(lens[seq_ids], dtype=np.int32),
-                     q_tokens=w.q_tokens)
+                     q_tokens=w.q_tokens, idx_exact=w.idx_exact)
     return c, seq_ids
 
 

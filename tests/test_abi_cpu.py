@@ -73,7 +73,8 @@ def _decode(lib, cache, seqs, ws=FAKE, ws_bytes=1 << 40, s_qi=1.0, s_q=1.0, scal
 
 
 @pytest.mark.parametrize("case", [
-    "null_cache", "null_seqs", "misaligned_k", "null_idx_scale_nvfp4", "bad_dtype", "zero_pages",
+    "null_cache", "null_seqs", "misaligned_k", "null_idx_scale_nvfp4", "null_idx_scale_exact",
+    "misaligned_idx_scale_exact", "bad_dtype", "zero_pages",
     "neg_scale", "nan_scale", "inf_softmax", "misaligned_q", "null_out", "misaligned_sel",
 ])
 def test_host_checks_reject(lib, case):
@@ -83,6 +84,10 @@ def test_host_checks_reject(lib, case):
     if case == "null_seqs": seqs = None
     if case == "misaligned_k": cache = _cache(k_data=FAKE + 8)
     if case == "null_idx_scale_nvfp4": cache = _cache(idx_scale=None)
+    if case == "null_idx_scale_exact":
+        cache = _cache(idx_scale=None, idx_dtype=msa.MSA_IDX_NVFP4_EXACT)
+    if case == "misaligned_idx_scale_exact":
+        cache = _cache(idx_scale=FAKE + 8, idx_dtype=msa.MSA_IDX_NVFP4_EXACT)
     if case == "bad_dtype": cache = _cache(idx_dtype=7)
     if case == "zero_pages": cache = _cache(num_pages=0)
     if case == "neg_scale": cache = _cache(s_v=-1.0)

@@ -9,6 +9,7 @@ Workloads (seeded, synthetic, N(0,1) before quantisation):
   ctx128k_b64_t8       64 x 131,072, 8 query tokens (causal), shuffled pages
   ragged_b16_t1        16 ragged lengths in [2,048, 262,144], shuffled pages
   prefill_67584_t2048  1 x (65,536 cached + 2,048 new), 2,048 query tokens
+and the 128K workload once more with exactly scored index keys.
 """
 import numpy as np
 import pytest
@@ -49,5 +50,17 @@ def test_full_size_sampled(name):
         seq_ids = sorted(set(seq_ids + [int(np.argmax(lens))]))
     swaps, mx, mean = compare_decode(w, seq_ids, tokens, what=name)
     print("%s: near-tie swaps %d, max-abs %.3g, mean-abs %.3g" % (name, swaps, mx, mean))
+    del w
+    torch.cuda.empty_cache()
+
+
+def test_full_size_exact_indexer_sampled():
+    """The benchmark workload with the index keys scored at their exact value
+    (MSA_IDX_NVFP4_EXACT), sampled like the rest."""
+    torch.cuda.empty_cache()
+    w = synth.workload("ctx128k_b64_t8", device="cuda")
+    w = synth.Workload(**{**w.__dict__, "idx_exact": True})
+    swaps, mx, mean = compare_decode(w, [11], None, what="ctx128k_b64_t8 exact")
+    print("ctx128k_b64_t8 exact: near-tie swaps %d, max-abs %.3g, mean-abs %.3g" % (swaps, mx, mean))
     del w
     torch.cuda.empty_cache()

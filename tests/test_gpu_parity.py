@@ -109,8 +109,21 @@ SMALL = [
                         neg_scale_frac=0.05)),
 ]
 
+# NVFP4 index keys scored at their exact value (MSA_IDX_NVFP4_EXACT): query
+# tiles of 8, 32 and 256 index queries, signed scales, ragged tails.
+EXACT = [
+    ("t1_exact", dict(batch=3, seq_lens=[300, 2049, 5000], q_tokens=1, paged=True, seed=32,
+                      idx_exact=True)),
+    ("t8_exact", dict(batch=2, seq_lens=[3000, 9000], q_tokens=8, paged=True, seed=33,
+                      idx_exact=True)),
+    ("neg_scales_exact", dict(batch=2, seq_lens=[5000, 2600], q_tokens=4, paged=True, seed=34,
+                              neg_scale_frac=0.05, idx_exact=True)),
+    ("t64_exact", dict(batch=1, seq_lens=[4000], q_tokens=64, paged=True, seed=35,
+                       idx_exact=True)),
+]
 
-@pytest.mark.parametrize("name,kw", SMALL, ids=[s[0] for s in SMALL])
+
+@pytest.mark.parametrize("name,kw", SMALL + EXACT, ids=[s[0] for s in SMALL + EXACT])
 def test_indexer_scores(name, kw):
     w = dev_workload(name, **kw)
     ts, bs = run_indexer(w)
@@ -128,6 +141,24 @@ def test_indexer_scores(name, kw):
         ref_t[:, :pos + 1] = rts[r, :, :pos + 1]
         parity.check_scores(gts[r, :, :nblk * 128], ref_t, "%s token scores row %d" % (name, r))
         parity.check_scores(gbs[r, :, :nblk], rbs[r, :, :nblk], "%s block scores row %d" % (name, r))
+
+
+def test_exact_mode_is_not_rerounded():
+    """The exact-mode scores sit on the unrounded oracle, far (relative to the
+    score tolerance) from the E4M3 re-rounded one, and the two GPU modes differ."""
+    w = dev_workload("exact_vs_rr", 2, [3000, 9000], 8, paged=True, seed=33, idx_exact=True)
+    ts, _ = run_indexer(w)
+    ts_rr, _ = run_indexer(synth.Workload(**{**w.__dict__, "idx_exact": False}))
+    c, _ = parity.host_cache(w)
+    rows = oracle.all_rows(c)
+    c.idx_exact = False
+    rts_rr, _ = oracle.indexer(c, w.qi.cpu().numpy(), w.s_qi, rows, ctx_cap=w.max_pages * 128)
+    g = ts.cpu().numpy().reshape(len(rows), 4, -1)
+    b, t = rows[0]
+    pos = int(c.seq_lens[b]) - w.q_tokens + t
+    with pytest.raises(AssertionError):
+        parity.check_scores(g[0, :, :pos + 1], rts_rr[0, :, :pos + 1], "exact vs re-rounded")
+    assert not torch.equal(ts, ts_rr)
 
 
 def test_block_scores_independent_of_batch_composition():
@@ -232,7 +263,7 @@ def test_attention_given_oracle_selection(name, kw):
 
 
 # ------------------------------------------------------------- decode ------
-@pytest.mark.parametrize("name,kw", SMALL, ids=[s[0] for s in SMALL])
+@pytest.mark.parametrize("name,kw", SMALL + EXACT, ids=[s[0] for s in SMALL + EXACT])
 def test_decode_small(name, kw):
     w = dev_workload(name, **kw)
     compare_decode(w, what=name)
