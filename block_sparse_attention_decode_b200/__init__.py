@@ -23,8 +23,9 @@ BLOCK, TOPK, HEAD_DIM, KV_HEADS, Q_HEADS = 128, 16, 128, 4, 64
 EXPORTED = [
     "msa_workspace_size", "msa_workspace_init", "msa_indexer_score", "msa_block_maxpool_topk",
     "msa_sparse_attn_decode", "msa_decode", "msa_get_last_error", "msa_debug_nvfp4_table",
-    "msa_status_string", "msa_decode_static", "msa_kv_insert",
+    "msa_status_string", "msa_decode_static", "msa_kv_insert", "msa_indexer_score_part",
 ]
+MAX_PARTS = 64
 STATIC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -70,6 +71,9 @@ def load() -> ctypes.CDLL:
     L.msa_workspace_init.argtypes = [vp, sz, vp]
     L.msa_indexer_score.restype = ctypes.c_int
     L.msa_indexer_score.argtypes = [P(msa_cache), P(msa_seqs), vp, f32, vp, vp, vp, sz, vp]
+    L.msa_indexer_score_part.restype = ctypes.c_int
+    L.msa_indexer_score_part.argtypes = [P(msa_cache), P(msa_seqs), vp, f32, vp, vp, i32, i32, vp,
+                                         sz, vp]
     L.msa_block_maxpool_topk.restype = ctypes.c_int
     L.msa_block_maxpool_topk.argtypes = [vp, i32, P(msa_seqs), vp, vp, sz, vp]
     L.msa_sparse_attn_decode.restype = ctypes.c_int
@@ -189,6 +193,14 @@ def msa_indexer_score(cache: Cache, seqs: Seqs, qi, s_qi: float, token_scores, b
     _check(load().msa_indexer_score(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi), s_qi,
                                     _ptr(token_scores), _ptr(block_scores), _ptr(ws),
                                     ws.numel(), _stream(stream)), "msa_indexer_score")
+
+
+def msa_indexer_score_part(cache: Cache, seqs: Seqs, qi, s_qi: float, token_scores, block_scores,
+                           part: int, nparts: int, ws, stream=None):
+    _check(load().msa_indexer_score_part(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi),
+                                         s_qi, _ptr(token_scores), _ptr(block_scores), int(part),
+                                         int(nparts), _ptr(ws), ws.numel(), _stream(stream)),
+           "msa_indexer_score_part")
 
 
 def msa_block_maxpool_topk(scores, is_token_level: bool, seqs: Seqs, sel, ws, stream=None):

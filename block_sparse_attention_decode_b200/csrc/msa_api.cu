@@ -92,7 +92,7 @@ msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_E
 
 msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi, float s_qi,
                        float* token_scores, float* block_scores, void* ws, const Layout& L,
-                       cudaStream_t st) {
+                       cudaStream_t st, int part = 0, int nparts = 1) {
   IdxArgs a{};
   const bool fp8 = c->idx_dtype == MSA_IDX_FP8;
   if (!encode_row_tmap(&a.tmap_idx, c->idx_data, (uint64_t)c->num_pages * MSA_BLOCK_TOKENS,
@@ -112,6 +112,8 @@ msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi,
   a.T = s->q_tokens;
   a.max_pages = s->max_pages;
   a.num_pages = c->num_pages;
+  a.part = part;
+  a.nparts = nparts;
   const int mode = fp8 ? kIdxFp8 : (c->idx_dtype == MSA_IDX_NVFP4_EXACT ? kIdxF16 : kIdxNvfp4);
   return cuda_status(launch_indexer(a, mode, device_sms(), st));
 }
@@ -227,7 +229,16 @@ msa_status msa_workspace_init(void* ws, size_t ws_bytes, msa_stream_t stream) {
 msa_status msa_indexer_score(const msa_cache* cache, const msa_seqs* seqs, const uint8_t* qi,
                              float s_qi, float* token_scores, float* block_scores, void* ws,
                              size_t ws_bytes, msa_stream_t stream) {
+  return msa_indexer_score_part(cache, seqs, qi, s_qi, token_scores, block_scores, 0, 1, ws,
+                                ws_bytes, stream);
+}
+
+msa_status msa_indexer_score_part(const msa_cache* cache, const msa_seqs* seqs, const uint8_t* qi,
+                                  float s_qi, float* token_scores, float* block_scores,
+                                  int32_t part, int32_t nparts, void* ws, size_t ws_bytes,
+                                  msa_stream_t stream) {
   if (!seqs_ok(seqs)) return MSA_ERR_INVALID_ARG;
+  if (nparts < 1 || nparts > MSA_MAX_PARTS || part < 0 || part >= nparts) return MSA_ERR_INVALID_ARG;
   msa_status st = check_cache(cache, true, false);
   if (st != MSA_OK) return st;
   if (!qi || !aligned16(qi) || !block_scores || !aligned16(block_scores) || !good_scale(s_qi))
@@ -236,7 +247,7 @@ msa_status msa_indexer_score(const msa_cache* cache, const msa_seqs* seqs, const
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
   return run_indexer(cache, seqs, qi, s_qi, token_scores, block_scores, ws, L,
-                     (cudaStream_t)stream);
+                     (cudaStream_t)stream, part, nparts);
 }
 
 msa_status msa_block_maxpool_topk(const float* scores, int32_t is_token_level, const msa_seqs* seqs,

@@ -12,6 +12,9 @@
 //
 // Work split: the pages of all sequences form one flat list, cut into chunks
 // of kChunkPages; a work item is (query tile of NQ index queries, chunk).
+// A launch may score only part `part` of `nparts` of every sequence's blocks
+// (the context split of [post, "NVFP4 indexer DCP"]); the flat list then
+// holds only those blocks.
 // Persistent CTAs (two per SM) take items from a counter in the workspace
 // header as they go, so that CTAs sharing an SM -- which the warp schedulers
 // do not serve equally -- and ragged batches still finish together; the last
@@ -116,9 +119,22 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
   return p;
 }
 
-// Exclusive prefix over the number of blocks of each sequence, in shared
-// memory (prefix[B] = total pages).  Invalid lengths count as 0 blocks and
-// are reported once (by CTA (0,0)).
+// The part of a sequence of length L this launch scores: logical blocks
+// [first, first + count) with first = floor(nblk * part / nparts) -- the
+// context split of [post, "NVFP4 indexer DCP"] (parts 0 of 1: every block).
+// Invalid lengths give 0 blocks.
+__device__ __forceinline__ int part_blocks(const IdxArgs& a, int L, int* first) {
+  if (L < a.T || L > a.max_pages * kBlock) { *first = 0; return 0; }
+  const int nblk = (L + kBlock - 1) / kBlock;
+  const int lo = (int)((long long)nblk * a.part / a.nparts);
+  const int hi = (int)((long long)nblk * (a.part + 1) / a.nparts);
+  *first = lo;
+  return hi - lo;
+}
+
+// Exclusive prefix over the number of blocks this launch scores in each
+// sequence, in shared memory (prefix[B] = total pages).  Invalid lengths
+// count as 0 blocks and are reported once (by CTA (0,0)).
 __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (a.B + nt - 1) / nt;
@@ -126,12 +142,10 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
   int sum = 0;
   for (int b = lo; b < hi; ++b) {
     const int L = a.seq_lens[b];
-    int nb = 0;
-    if (L >= a.T && L <= a.max_pages * kBlock) {
-      nb = (L + kBlock - 1) / kBlock;
-    } else if (blockIdx.x == 0 && blockIdx.y == 0) {
+    int first;
+    const int nb = part_blocks(a, L, &first);
+    if ((L < a.T || L > a.max_pages * kBlock) && blockIdx.x == 0 && blockIdx.y == 0)
       report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
-    }
     sum += nb;
   }
   scratch[tid] = sum;
@@ -145,8 +159,8 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
   int run = scratch[tid];
   for (int b = lo; b < hi; ++b) {
     prefix[b] = run;
-    const int L = a.seq_lens[b];
-    run += (L >= a.T && L <= a.max_pages * kBlock) ? (L + kBlock - 1) / kBlock : 0;
+    int first;
+    run += part_blocks(a, a.seq_lens[b], &first);
   }
   __syncthreads();
 }
@@ -223,6 +237,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         return kk < kIdxRawStages ||
                mbar_wait(&raw_empty[kk % kIdxRawStages], ((kk / kIdxRawStages) - 1) & 1);
       };
+      int first_b = -1, first = 0;                // part_blocks of sequence first_b
       int item = atomicAdd(&a.work[0], 1);
       while (item < items && ok) {
         const int nxt = atomicAdd(&a.work[0], 1);  // claimed early: its latency overlaps this item
@@ -235,12 +250,17 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           while (r - l > 1) { const int m = (l + r) >> 1; if (prefix[m] <= p0) l = m; else r = m; }
           b = l;
         }
-        int i = p0 - prefix[b];
-        for (int pg = p0; pg < p1; ++pg, ++k) {
+        int li = p0 - prefix[b];                    // index among this part's blocks of b
+        for (int pg = p0; pg < p1; ++pg, ++k, ++li) {
           if (!slot(k)) { report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1); ok = false; break; }
           const int s = k % kIdxRawStages;
-          while (i >= prefix[b + 1] - prefix[b]) { i -= prefix[b + 1] - prefix[b]; ++b; }
+          while (li >= prefix[b + 1] - prefix[b]) { li -= prefix[b + 1] - prefix[b]; ++b; }
           const int L = a.seq_lens[b];
+          if (b != first_b) {                       // first block of b's part
+            first_b = b;
+            part_blocks(a, L, &first);
+          }
+          const int i = first + li;                 // logical block
           int kind = kPageLoad;
           const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + i]
                                            : (long long)b * a.max_pages + i;
@@ -267,7 +287,6 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           } else {
             mbar_arrive(&raw_full[s]);
           }
-          ++i;
         }
         item = nxt;
       }

@@ -30,6 +30,7 @@ struct IdxArgs {
   int* work;                   // [2] in the workspace header: next item, CTAs done (0 on entry)
   float score_scale;           // s_qi * s_idx
   int B, T, max_pages, num_pages;
+  int part, nparts;            // score blocks [nblk*part/nparts, nblk*(part+1)/nparts) of each sequence
 };
 
 size_t indexer_smem_bytes(int mode, int batch, int T);

@@ -80,6 +80,7 @@ extern "C" {
 #define MSA_KV_HEADS 4
 #define MSA_Q_HEADS 64
 #define MSA_MAX_BATCH 4096
+#define MSA_MAX_PARTS 64        /* context parts of msa_indexer_score_part */
 
 /* A cudaStream_t, declared without the CUDA headers. */
 typedef struct CUstream_st* msa_stream_t;
@@ -146,6 +147,26 @@ MSA_API msa_status msa_workspace_init(void* ws, size_t ws_bytes, msa_stream_t st
 MSA_API msa_status msa_indexer_score(const msa_cache* cache, const msa_seqs* seqs,
                              const uint8_t* qi, float s_qi,
                              float* token_scores, float* block_scores,
+                             void* ws, size_t ws_bytes, msa_stream_t stream);
+
+/* msa_indexer_score restricted to one part of every sequence's context: the
+ * context split of [post, "NVFP4 indexer DCP"], where each GPU scores all
+ * four index heads over its share of the pages and the shares' results are
+ * combined into one exact selection.  Part `part` of `nparts` of a sequence
+ * with nblk = ceil(len/128) blocks is the logical blocks
+ *     [floor(nblk*part/nparts), floor(nblk*(part+1)/nparts))
+ * (the parts tile 0..nblk-1; a part may be empty).  Only those blocks are
+ * read (so the page table entries and pages of other parts are never
+ * touched) and only their entries of token_scores / block_scores are
+ * written, with exactly the values msa_indexer_score writes for them; the
+ * element-wise max of all parts' block_scores, each pre-filled with -inf,
+ * is msa_indexer_score's block_scores.  Causal masking uses each block's
+ * absolute position.  1 <= nparts <= MSA_MAX_PARTS, 0 <= part < nparts,
+ * else MSA_ERR_INVALID_ARG; other arguments as msa_indexer_score. */
+MSA_API msa_status msa_indexer_score_part(const msa_cache* cache, const msa_seqs* seqs,
+                             const uint8_t* qi, float s_qi,
+                             float* token_scores, float* block_scores,
+                             int32_t part, int32_t nparts,
                              void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /* Step (3) of [post, "MSA primer"]: per (b, t, g) select the top 16 blocks

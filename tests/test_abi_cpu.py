@@ -118,6 +118,10 @@ def test_stage_entry_points_check_args(lib):
                                    0.1, FAKE, FAKE, 1 << 40, None)
     assert r == msa.MSA_ERR_INVALID_ARG           # sel required
     assert lib.msa_debug_nvfp4_table(None, None) == msa.MSA_ERR_INVALID_ARG
+    for part, nparts in ((0, 0), (1, 1), (-1, 2), (0, 65)):     # context parts out of range
+        r = lib.msa_indexer_score_part(ctypes.byref(cache), ctypes.byref(seqs), FAKE, 1.0, None,
+                                       FAKE, part, nparts, FAKE, 1 << 40, None)
+        assert r == msa.MSA_ERR_INVALID_ARG, (part, nparts)
     fp8 = _cache(idx_scale=None, idx_dtype=msa.MSA_IDX_FP8, s_idx=-2.0)
     r = lib.msa_indexer_score(ctypes.byref(fp8), ctypes.byref(seqs), FAKE, 1.0, None, FAKE,
                               FAKE, 1 << 40, None)
