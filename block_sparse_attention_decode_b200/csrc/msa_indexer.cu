@@ -124,10 +124,13 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
 // context split of [post, "NVFP4 indexer DCP"] (parts 0 of 1: every block).
 // Invalid lengths give 0 blocks.
 __device__ __forceinline__ int part_blocks(const IdxArgs& a, int L, int* first) {
-  if (L < a.T || L > a.max_pages * kBlock) { *first = 0; return 0; }
+  *first = 0;
+  if (L < a.T || L > a.max_pages * kBlock) return 0;
   const int nblk = (L + kBlock - 1) / kBlock;
-  const int lo = (int)((long long)nblk * a.part / a.nparts);
-  const int hi = (int)((long long)nblk * (a.part + 1) / a.nparts);
+  if (a.nparts == 1) return nblk;
+  // nblk * nparts fits in 32 bits: nblk < 2^24 (L <= max_pages * 128 < 2^31), nparts <= 64
+  const int lo = nblk * a.part / a.nparts;
+  const int hi = nblk * (a.part + 1) / a.nparts;
   *first = lo;
   return hi - lo;
 }
