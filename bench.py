@@ -93,6 +93,21 @@ KERNEL_SOURCES = {
 }
 
 
+L2_BYTES = 126 * 1000 * 1000
+
+
+def l2_notes(cache_bytes: int):
+    """How the timed regions treat L2 for a cache of cache_bytes: the note of
+    the device-timed steps and the note of the end-to-end loop."""
+    gb = cache_bytes / 1e9
+    if cache_bytes > L2_BYTES:
+        return ("256 MiB written before each timed step (outside the events); "
+                "inputs %.1f GB > 126 MB L2" % gb, "no L2 flush (inputs > L2)")
+    return ("256 MiB written before each timed step (outside the events); inputs %.3f GB "
+            "fit in the 126 MB L2, so the flush is what sends them back to HBM" % gb,
+            "no L2 flush: the inputs (%.3f GB) fit in L2 and stay there from step to step" % gb)
+
+
 def dram_traffic(kernel: str, workload: str):
     """Per-launch DRAM bytes from the committed ncu summary, or None when the
     kernel source changed since the counters were taken."""
@@ -451,6 +466,9 @@ def run_gpu(args, rank, world, local_rank):
     h2d = h_qi.numel() + h_q.numel() + h_lens.numel() * 4
     d2h = h_out[0].numel() * 2
 
+    cache_bytes = (w.idx_data.numel() + 2 * (w.k_data.numel() + w.k_scale.numel())
+                   + (w.idx_scale.numel() if w.idx_scale is not None else 0))
+    l2_note, e2e_l2_note = l2_notes(cache_bytes)
     result = None
     if rank == 0:
         q_total = B * T * world
@@ -466,10 +484,7 @@ def run_gpu(args, rank, world, local_rank):
                        "kv_cache": "nvfp4, 128-token pages" + (", shuffled page table"
                                                                  if w.page_table is not None else ""),
                        "global_batch": B * world, "parallelism": "dp%d" % world,
-                       "l2": "256 MiB written before each timed step (outside the events); "
-                             "inputs %.1f GB > 126 MB L2" % (
-                                 (w.idx_data.numel() + 2 * (w.k_data.numel() + w.k_scale.numel())
-                                  + (w.idx_scale.numel() if w.idx_scale is not None else 0)) / 1e9)},
+                       "l2": l2_note},
             "hbm": {"algorithmic_bytes_per_step": bytes_["total"], "achieved_gbs": gbs,
                     "frac_of_measured": gbs / peak, "frac_of_spec_8000": gbs / SPEC_HBM_GBS,
                     "peak_source": peak_src, "bytes": bytes_},
@@ -489,8 +504,7 @@ def run_gpu(args, rank, world, local_rank):
             "e2e": {"value": q_total / (ms_e2e * 1e-3), "unit": "queries/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                     "mode": "pipelined: each step's queries copied in and output copied out on "
-                            "copy streams, overlapping other steps' decodes; no L2 flush "
-                            "(inputs > L2)"},
+                            "copy streams, overlapping other steps' decodes; " + e2e_l2_note},
             "wall_s_timed_region": t_wall,
         }
     return result
