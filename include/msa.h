@@ -185,7 +185,8 @@ MSA_API msa_status msa_block_maxpool_topk(const float* scores, int32_t is_token_
  * softmax over the keys j <= pos of the selected blocks of
  *   softmax_scale * s_q * s_k * (q_h . k_j),
  * output s_v * sum_j p_j v_j rounded to bf16.  K and V are NVFP4, decoded to
- * E4M3 in the kernel and contracted with FP8 MMA (P is rounded to E4M3).
+ * E4M3 in the kernel and contracted with FP8 MMA; the probabilities P enter
+ * the P.V product as the sum of two E4M3 terms (P to about 2^-8 relative).
  * sel entries -1 are skipped; ids outside 0..pos/128 are a device error. */
 MSA_API msa_status msa_sparse_attn_decode(const msa_cache* cache, const msa_seqs* seqs,
                                   const uint8_t* q, float s_q, const int32_t* sel,
