@@ -110,6 +110,10 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
 def _check(status: int, what: str):
     if status != MSA_OK:
         raise MsaError(status, what)
@@ -178,7 +182,7 @@ def msa_workspace_size(seqs: Seqs) -> int:
 
 
 def msa_workspace_init(ws: torch.Tensor, stream=None):
-    _check(load().msa_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+    _check(load().msa_workspace_init(_ptr(ws), _nbytes(ws), _stream(stream)),
            "msa_workspace_init")
 
 
@@ -190,36 +194,48 @@ def alloc_workspace(seqs: Seqs, device=None) -> torch.Tensor:
 
 def msa_indexer_score(cache: Cache, seqs: Seqs, qi, s_qi: float, token_scores, block_scores,
                       ws, stream=None):
+    """Indexer scores and block max-pool.  qi: uint8 E4M3 [B][T][4][128];
+    token_scores: float32 [B][T][4][max_pages*128] or None; block_scores:
+    float32 [B][T][4][max_pages]."""
     _check(load().msa_indexer_score(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi), s_qi,
                                     _ptr(token_scores), _ptr(block_scores), _ptr(ws),
-                                    ws.numel(), _stream(stream)), "msa_indexer_score")
+                                    _nbytes(ws), _stream(stream)), "msa_indexer_score")
 
 
 def msa_indexer_score_part(cache: Cache, seqs: Seqs, qi, s_qi: float, token_scores, block_scores,
                            part: int, nparts: int, ws, stream=None):
+    """msa_indexer_score over part `part` of `nparts` of every sequence's
+    blocks only (context parallelism); the other entries are not written."""
     _check(load().msa_indexer_score_part(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi),
                                          s_qi, _ptr(token_scores), _ptr(block_scores), int(part),
-                                         int(nparts), _ptr(ws), ws.numel(), _stream(stream)),
+                                         int(nparts), _ptr(ws), _nbytes(ws), _stream(stream)),
            "msa_indexer_score_part")
 
 
 def msa_block_maxpool_topk(scores, is_token_level: bool, seqs: Seqs, sel, ws, stream=None):
+    """Top-16 blocks per (b, t, g), the latest always kept: sel int32
+    [B][T][4][16], ascending, -1 padded.  scores: block scores, or token
+    scores (max-pooled first) when is_token_level."""
     _check(load().msa_block_maxpool_topk(_ptr(scores), int(bool(is_token_level)),
-                                         ctypes.byref(seqs.c), _ptr(sel), _ptr(ws), ws.numel(),
+                                         ctypes.byref(seqs.c), _ptr(sel), _ptr(ws), _nbytes(ws),
                                          _stream(stream)), "msa_block_maxpool_topk")
 
 
 def msa_sparse_attn_decode(cache: Cache, seqs: Seqs, q, s_q: float, sel, softmax_scale: float,
                            out, ws, stream=None):
+    """Attention over the selected blocks.  q: uint8 E4M3 [B][T][64][128];
+    sel: int32 [B][T][4][16]; out: bfloat16 [B][T][64][128]."""
     _check(load().msa_sparse_attn_decode(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(q), s_q,
-                                         _ptr(sel), softmax_scale, _ptr(out), _ptr(ws), ws.numel(),
+                                         _ptr(sel), softmax_scale, _ptr(out), _ptr(ws), _nbytes(ws),
                                          _stream(stream)), "msa_sparse_attn_decode")
 
 
 def msa_decode(cache: Cache, seqs: Seqs, qi, s_qi: float, q, s_q: float, softmax_scale: float,
                out, sel_out, ws, stream=None):
+    """The whole decode step (indexer, top-16, attention) on `stream`;
+    sel_out (int32 [B][T][4][16]) optional."""
     _check(load().msa_decode(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi), s_qi, _ptr(q),
-                             s_q, softmax_scale, _ptr(out), _ptr(sel_out), _ptr(ws), ws.numel(),
+                             s_q, softmax_scale, _ptr(out), _ptr(sel_out), _ptr(ws), _nbytes(ws),
                              _stream(stream)), "msa_decode")
 
 
@@ -236,12 +252,15 @@ def msa_kv_insert(cache: Cache, seqs: Seqs, k_new, v_new, idx_new, ws, stream=No
     """Quantise the new tokens (bf16 tensors [B][T][4][128], [B][T][4][128],
     [B][T][128]) into the cache the descriptor points to."""
     for x in (k_new, v_new, idx_new):
-        assert x.dtype == torch.bfloat16 and x.is_contiguous()
+        if x.dtype != torch.bfloat16 or not x.is_contiguous():
+            raise ValueError("msa_kv_insert takes contiguous bfloat16 tensors")
     _check(load().msa_kv_insert(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(k_new), _ptr(v_new),
-                                _ptr(idx_new), _ptr(ws), ws.numel(), _stream(stream)), "msa_kv_insert")
+                                _ptr(idx_new), _ptr(ws), _nbytes(ws), _stream(stream)), "msa_kv_insert")
 
 
 def msa_get_last_error(ws, stream=None):
+    """(status, detail) of the first device-side error since the last call;
+    synchronises the stream and clears the record."""
     detail = ctypes.c_int32(0)
     st = load().msa_get_last_error(_ptr(ws), _stream(stream), ctypes.byref(detail))
     return int(st), int(detail.value)
