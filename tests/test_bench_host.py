@@ -49,3 +49,22 @@ def test_measured_peaks_come_from_the_file():
     peak, src = bench.measured_peaks()
     d = json.load(open(bench.os.path.join(bench.ROOT, "MEASURED_PEAKS.json")))
     assert src == "measured" and peak == float(d["hbm_gbs"])
+
+
+def test_reference_arm_prints_the_contract_line():
+    """bench.py --impl reference (the oracle on the host cores) prints one JSON
+    line with the contract's keys; a small workload keeps it quick."""
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload",
+                        "ctx4k_b1_t1", "--steps", "1", "--warmup", "0"],
+                       cwd=bench.ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["warmup"] >= 3
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
