@@ -221,21 +221,22 @@ def algorithmic_bytes(w, sel):
 
 
 # --------------------------------------------------------- CPU baseline --
-def cpu_sample_workload(name: str, seed_offset: int = 0):
-    """One sequence with the shapes of `name` (its full context, all of its
-    query tokens), generated on the host: a bounded sample of the workload."""
+def cpu_sample_workload(name: str, seed_offset: int = 0, nseq: int = 1):
+    """nseq sequences with the shapes of `name` (the longest context of the
+    workload, all of its query tokens), generated on the host: a bounded
+    sample of the workload."""
     from block_sparse_attention_decode_b200 import synth
     kw = dict(synth.WORKLOADS[name])
     if kw["seq_lens"] is None:
         kw["seq_lens"] = synth.ragged_lengths(kw["batch"], 2048, 262144, kw["seed"])
     L = max(kw["seq_lens"])
-    kw.update(batch=1, seq_lens=[L], seed=kw["seed"] + 100 + seed_offset)
-    if kw.get("plant_every"):
-        kw["plant_every"] = kw["plant_every"]
+    kw.update(batch=nseq, seq_lens=[L] * nseq, seed=kw["seed"] + 100 + seed_offset)
     return synth.make_workload(name + "_cpu_sample", device="cpu", **kw)
 
 
-def oracle_step(w, tokens, threads):
+def oracle_step(w, rows, threads):
+    """The float64 oracle's whole path (index scan, top-16, attention) for the
+    (sequence, token) rows of w on `threads` host threads; seconds."""
     import numpy as np
     import oracle
     oracle.set_threads(threads)
@@ -244,27 +245,35 @@ def oracle_step(w, tokens, threads):
                      k_scale=n(w.k_scale), v_data=n(w.v_data), v_scale=n(w.v_scale),
                      s_idx=w.s_idx, s_k=w.s_k, s_v=w.s_v, page_table=n(w.page_table),
                      max_pages=w.max_pages, seq_lens=n(w.seq_lens), q_tokens=w.q_tokens)
-    rows = [(0, t) for t in tokens]
     t0 = time.perf_counter()
     oracle.decode(c, np.ascontiguousarray(n(w.qi)), w.s_qi, np.ascontiguousarray(n(w.q)), w.s_q,
-                  w.softmax_scale, rows)
+                  w.softmax_scale, list(rows))
     return time.perf_counter() - t0
 
 
+def host_threads() -> int:
+    """Threads both oracle arms use: every host core."""
+    return max(1, os.cpu_count() or 1)
+
+
 def cpu_baseline(name: str, budget_s: float = 20.0):
-    w = cpu_sample_workload(name)
-    threads = max(1, min(os.cpu_count() or 1, w.q_tokens))
-    tokens = list(range(w.q_tokens))
-    dt = oracle_step(w, tokens, threads)
+    import math
+    from block_sparse_attention_decode_b200 import synth
+    threads = host_threads()
+    T = synth.WORKLOADS[name]["q_tokens"]
+    nseq = max(1, math.ceil(threads / T))          # enough (sequence, token) rows for every thread
+    w = cpu_sample_workload(name, nseq=nseq)
+    rows = [(b, t) for b in range(nseq) for t in range(T)]
+    dt = oracle_step(w, rows, threads)
     reps = 1
     while dt * (reps + 1) / reps < budget_s and reps < 3:
-        dt += oracle_step(w, tokens, threads)
+        dt += oracle_step(w, rows, threads)
         reps += 1
-    qps = reps * len(tokens) / dt
+    qps = reps * len(rows) / dt
     return {"value": qps, "unit": "queries/s", "cores": threads, "kind": "oracle",
-            "sample": "%d x (1 sequence of %d tokens, its %d query tokens: full index scan, "
-                      "top-16, attention) of %s, float64 C oracle" % (reps, int(w.seq_lens[0]),
-                                                                    w.q_tokens, name)}
+            "sample": "%d x (%d sequences of %d tokens, all %d query tokens of each: full index "
+                      "scan, top-16, attention) of %s, float64 C oracle on %d host threads"
+                      % (reps, nseq, int(w.seq_lens[0]), T, name, threads)}
 
 
 # ------------------------------------------------------------- GPU arm ----
@@ -529,12 +538,12 @@ def main():
         if rank != 0:
             return 0
         w = cpu_sample_workload(args.workload)
-        threads = max(1, os.cpu_count() or 1)
+        threads = host_threads()
         # K steps of one query each (token k % T of the sampled sequence: full
         # index scan, top-16, attention), evaluated together on all host cores;
         # the W warm-up queries likewise.
-        oracle_step(w, [k % w.q_tokens for k in range(args.warmup)], threads)
-        t = oracle_step(w, [k % w.q_tokens for k in range(args.steps)], threads)
+        oracle_step(w, [(0, k % w.q_tokens) for k in range(args.warmup)], threads)
+        t = oracle_step(w, [(0, k % w.q_tokens) for k in range(args.steps)], threads)
         qps = args.steps / t
         sample = ("per step: one query token of 1 sequence of %d tokens (shapes of %s): full "
                   "index scan, top-16 and attention in the float64 C oracle; the %d steps run "

@@ -3,6 +3,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "msa.h"
 #include "msa_internal.h"
@@ -14,15 +15,12 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-int device_sms() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 148; }
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
-    cudaGetLastError();
-    return 148;
-  }
-  return sms;
-}
+// SM count the attention's split heuristic is planned for (B200: 148 SMs).
+// The workspace layout depends on it, so it is a constant of the library
+// rather than a property queried from whatever device is current: the size
+// msa_workspace_size reports is then the same on every machine.  The
+// persistent grids themselves use the device's real SM count.
+constexpr int kPlanSms = 148;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool good_scale(float s) { return std::isfinite(s) && s > 0.f; }
@@ -43,10 +41,10 @@ bool seqs_ok(const msa_seqs* s) {
   return rows <= 0x7FFFFFFFLL / MSA_TOPK;
 }
 
-Layout layout_for(const msa_seqs* s, int sms) {
+Layout layout_for(const msa_seqs* s) {
   Layout L{};
   const long long rows = (long long)s->batch * s->q_tokens * kG;
-  L.splits = attn_splits(rows, sms);
+  L.splits = attn_splits(rows, kPlanSms);
   size_t off = 0;
   L.flags = off;    off += align_up(sizeof(Flags));
   L.bscores = off;  off += align_up((size_t)rows * s->max_pages * sizeof(float));
@@ -80,10 +78,68 @@ msa_status check_cache(const msa_cache* c, bool need_index, bool need_kv) {
 }
 
 msa_status check_ws(const msa_seqs* s, void* ws, size_t ws_bytes, Layout* L) {
-  *L = layout_for(s, device_sms());
+  *L = layout_for(s);
   if (!ws || !aligned16(ws) || ws_bytes < L->total) return MSA_ERR_WORKSPACE;
   return MSA_OK;
 }
+
+// Memory check before any launch: the first and the last byte of
+// [p, p + bytes) must be device memory of the current device (or managed
+// memory).  Pageable or pinned host memory, another device's memory and
+// addresses CUDA does not know are rejected with `bad`, so that a wrong
+// pointer from a C caller returns an error instead of faulting the GPU.
+// A buffer that ends inside another allocation is not detected.  NULL
+// pointers pass (whether a pointer may be NULL is checked before).
+msa_status check_buf(const void* p, size_t bytes, msa_status bad = MSA_ERR_INVALID_ARG) {
+  if (p == nullptr || bytes == 0) return MSA_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MSA_ERR_CUDA; }
+  const uint8_t* ends[2] = {static_cast<const uint8_t*>(p), static_cast<const uint8_t*>(p) + bytes - 1};
+  for (const uint8_t* x : ends) {
+    cudaPointerAttributes at{};
+    const cudaError_t e = cudaPointerGetAttributes(&at, x);
+    if (e == cudaErrorInvalidValue) { cudaGetLastError(); return bad; }
+    if (e != cudaSuccess) { cudaGetLastError(); return MSA_ERR_CUDA; }
+    if (at.type == cudaMemoryTypeManaged) continue;
+    if (at.type != cudaMemoryTypeDevice || at.device != dev) return bad;
+  }
+  return MSA_OK;
+}
+
+// The cache pools and the sequence descriptors, sized by num_pages / batch.
+msa_status check_cache_mem(const msa_cache* c, bool need_index, bool need_kv) {
+  const size_t P = (size_t)c->num_pages;
+  msa_status st;
+  if (need_index) {
+    const size_t row = c->idx_dtype == MSA_IDX_FP8 ? MSA_HEAD_DIM : MSA_HEAD_DIM / 2;
+    if ((st = check_buf(c->idx_data, P * MSA_BLOCK_TOKENS * row)) != MSA_OK) return st;
+    if (c->idx_dtype != MSA_IDX_FP8 &&
+        (st = check_buf(c->idx_scale, P * MSA_BLOCK_TOKENS * 8)) != MSA_OK)
+      return st;
+  }
+  if (need_kv) {
+    const size_t codes = P * MSA_KV_HEADS * MSA_BLOCK_TOKENS * (MSA_HEAD_DIM / 2);
+    const size_t scales = P * MSA_KV_HEADS * MSA_BLOCK_TOKENS * 8;
+    if ((st = check_buf(c->k_data, codes)) != MSA_OK || (st = check_buf(c->v_data, codes)) != MSA_OK ||
+        (st = check_buf(c->k_scale, scales)) != MSA_OK || (st = check_buf(c->v_scale, scales)) != MSA_OK)
+      return st;
+  }
+  return MSA_OK;
+}
+
+msa_status check_seqs_mem(const msa_seqs* s) {
+  msa_status st = check_buf(s->seq_lens, (size_t)s->batch * 4);
+  if (st != MSA_OK) return st;
+  return check_buf(s->page_table, (size_t)s->batch * s->max_pages * 4);
+}
+
+// Rows (sequence, token) of the step and the per-row byte counts of the
+// query, output and selection buffers.
+size_t n_tok(const msa_seqs* s) { return (size_t)s->batch * s->q_tokens; }
+constexpr size_t kQiBytes = MSA_KV_HEADS * MSA_HEAD_DIM;            // per token
+constexpr size_t kQBytes = MSA_Q_HEADS * MSA_HEAD_DIM;              // per token
+constexpr size_t kOutBytes = MSA_Q_HEADS * MSA_HEAD_DIM * 2;        // per token
+constexpr size_t kSelBytes = MSA_KV_HEADS * MSA_TOPK * 4;           // per token
 
 template <typename T>
 T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off); }
@@ -115,7 +171,7 @@ msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi,
   a.part = part;
   a.nparts = nparts;
   const int mode = fp8 ? kIdxFp8 : (c->idx_dtype == MSA_IDX_NVFP4_EXACT ? kIdxF16 : kIdxNvfp4);
-  return cuda_status(launch_indexer(a, mode, device_sms(), st));
+  return cuda_status(launch_indexer(a, mode, st));
 }
 
 msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, float s_q,
@@ -155,7 +211,7 @@ msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, flo
   a.max_pages = s->max_pages;
   a.num_pages = c->num_pages;
   a.splits = L.splits;
-  return cuda_status(launch_attn(a, device_sms(), st));
+  return cuda_status(launch_attn(a, st));
 }
 
 }  // namespace
@@ -191,24 +247,86 @@ bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int ctas_per_sm(const void* kernel, int threads, size_t smem, int tmem_cols) {
-  int dev = 0, smem_sm = 0, regs_sm = 0, max_threads = 0;
+namespace {
+
+// CTAs of a kernel resident per SM (registers, shared memory, threads, TMEM).
+cudaError_t ctas_per_sm(const void* kernel, int dev, int threads, size_t smem, int tmem_cols,
+                        int* n_out) {
+  int smem_sm = 0, regs_sm = 0, max_threads = 0;
   cudaFuncAttributes fa{};
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaFuncGetAttributes(&fa, kernel) != cudaSuccess ||
-      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&max_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess) {
-    cudaGetLastError();
-    return 1;
-  }
+  cudaError_t e;
+  if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&max_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev)) != cudaSuccess)
+    return e;
   const int warps = (threads + 31) / 32;
   const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;      // allocation granularity
-  int n = regs_warp > 0 ? regs_sm / (regs_warp * warps) : 1;
+  int n = regs_warp > 0 ? regs_sm / (regs_warp * warps) : max_threads / (warps * 32);
   const size_t per_cta_smem = smem + fa.sharedSizeBytes + 1024;      // 1 KB reserved per CTA
-  n = std::min<long long>(n, (long long)(smem_sm / per_cta_smem));
+  n = (int)std::min<long long>(n, (long long)(smem_sm / per_cta_smem));
   n = std::min(n, max_threads / (warps * 32));
   if (tmem_cols > 0) n = std::min(n, 512 / tmem_cols);
-  return n < 1 ? 1 : n;
+  if (n < 1) return cudaErrorInvalidConfiguration;
+  *n_out = n;
+  return cudaSuccess;
+}
+
+// Per (kernel, device): the dynamic shared-memory limit set so far (only
+// ever raised: a smaller launch after a larger one keeps the larger limit)
+// and the grid computed for the last size seen.
+struct GridEntry {
+  const void* kernel;
+  int dev;
+  size_t smem_limit;
+  size_t smem;
+  int grid;
+};
+std::mutex g_grid_mu;
+GridEntry g_grid[64];
+int g_grid_n = 0;
+
+}  // namespace
+
+cudaError_t persistent_grid(const void* kernel, int threads, size_t smem, int tmem_cols, int* grid) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_grid_mu);
+  GridEntry* ent = nullptr;
+  for (int i = 0; i < g_grid_n; ++i)
+    if (g_grid[i].kernel == kernel && g_grid[i].dev == dev) ent = &g_grid[i];
+  if (ent != nullptr && ent->smem == smem && ent->smem_limit >= smem) {
+    *grid = ent->grid;
+    return cudaSuccess;
+  }
+  if (ent == nullptr || ent->smem_limit < smem) {
+    // with the table full (more kernels x devices than it holds), the limit
+    // goes straight to the device maximum so that no later call lowers it
+    int limit = (int)smem;
+    if (ent == nullptr && g_grid_n == (int)(sizeof(g_grid) / sizeof(g_grid[0])) &&
+        (e = cudaDeviceGetAttribute(&limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, limit)) !=
+        cudaSuccess)
+      return e;
+  }
+  int sms = 0, per_sm = 0;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = ctas_per_sm(kernel, dev, threads, smem, tmem_cols, &per_sm)) != cudaSuccess) return e;
+  *grid = sms * per_sm;
+  if (ent == nullptr && g_grid_n < (int)(sizeof(g_grid) / sizeof(g_grid[0]))) {
+    ent = &g_grid[g_grid_n++];
+    ent->kernel = kernel;
+    ent->dev = dev;
+    ent->smem_limit = 0;
+  }
+  if (ent != nullptr) {
+    ent->smem_limit = std::max(ent->smem_limit, smem);
+    ent->smem = smem;
+    ent->grid = *grid;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace msa
@@ -217,11 +335,13 @@ extern "C" {
 
 size_t msa_workspace_size(const msa_seqs* seqs) {
   if (!seqs_ok(seqs)) return 0;
-  return layout_for(seqs, device_sms()).total;
+  return layout_for(seqs).total;
 }
 
 msa_status msa_workspace_init(void* ws, size_t ws_bytes, msa_stream_t stream) {
   if (!ws || ws_bytes < sizeof(Flags)) return MSA_ERR_WORKSPACE;
+  const msa_status st = check_buf(ws, sizeof(Flags), MSA_ERR_WORKSPACE);
+  if (st != MSA_OK) return st;
   return cuda_status(cudaMemsetAsync(ws, 0, align_up(sizeof(Flags)) <= ws_bytes ? align_up(sizeof(Flags)) : ws_bytes,
                                      (cudaStream_t)stream));
 }
@@ -246,6 +366,12 @@ msa_status msa_indexer_score_part(const msa_cache* cache, const msa_seqs* seqs, 
   if (token_scores && !aligned16(token_scores)) return MSA_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  const size_t nt = n_tok(seqs), bs_bytes = nt * MSA_KV_HEADS * seqs->max_pages * 4;
+  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+      (st = check_cache_mem(cache, true, false)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
+      (st = check_buf(qi, nt * kQiBytes)) != MSA_OK || (st = check_buf(block_scores, bs_bytes)) != MSA_OK ||
+      (st = check_buf(token_scores, bs_bytes * MSA_BLOCK_TOKENS)) != MSA_OK)
+    return st;
   return run_indexer(cache, seqs, qi, s_qi, token_scores, block_scores, ws, L,
                      (cudaStream_t)stream, part, nparts);
 }
@@ -258,6 +384,11 @@ msa_status msa_block_maxpool_topk(const float* scores, int32_t is_token_level, c
   Layout L;
   msa_status st = check_ws(seqs, ws, ws_bytes, &L);
   if (st != MSA_OK) return st;
+  const size_t nt = n_tok(seqs), bs_bytes = nt * MSA_KV_HEADS * seqs->max_pages * 4;
+  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
+      (st = check_buf(scores, is_token_level ? bs_bytes * MSA_BLOCK_TOKENS : bs_bytes)) != MSA_OK ||
+      (st = check_buf(sel, nt * kSelBytes)) != MSA_OK)
+    return st;
   const cudaStream_t s = (cudaStream_t)stream;
   const float* bs = scores;
   if (is_token_level) {
@@ -282,6 +413,12 @@ msa_status msa_sparse_attn_decode(const msa_cache* cache, const msa_seqs* seqs, 
   if (!good_scale(s_q) || !good_scale(softmax_scale)) return MSA_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  const size_t nt = n_tok(seqs);
+  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+      (st = check_cache_mem(cache, false, true)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
+      (st = check_buf(q, nt * kQBytes)) != MSA_OK || (st = check_buf(sel, nt * kSelBytes)) != MSA_OK ||
+      (st = check_buf(out, nt * kOutBytes)) != MSA_OK)
+    return st;
   return run_attn(cache, seqs, q, s_q, sel, softmax_scale, out, ws, L, (cudaStream_t)stream);
 }
 
@@ -298,6 +435,12 @@ msa_status msa_decode(const msa_cache* cache, const msa_seqs* seqs, const uint8_
     return MSA_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  const size_t nt = n_tok(seqs);
+  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+      (st = check_cache_mem(cache, true, true)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
+      (st = check_buf(qi, nt * kQiBytes)) != MSA_OK || (st = check_buf(q, nt * kQBytes)) != MSA_OK ||
+      (st = check_buf(out, nt * kOutBytes)) != MSA_OK || (st = check_buf(sel_out, nt * kSelBytes)) != MSA_OK)
+    return st;
   const cudaStream_t s = (cudaStream_t)stream;
   float* bs = at<float>(ws, L.bscores);
   int32_t* sel = sel_out ? sel_out : at<int32_t>(ws, L.sel);
@@ -318,6 +461,13 @@ msa_status msa_kv_insert(const msa_cache* cache, const msa_seqs* seqs, const uin
     return MSA_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  const size_t nt = n_tok(seqs);
+  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+      (st = check_cache_mem(cache, true, true)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
+      (st = check_buf(k_new, nt * MSA_KV_HEADS * MSA_HEAD_DIM * 2)) != MSA_OK ||
+      (st = check_buf(v_new, nt * MSA_KV_HEADS * MSA_HEAD_DIM * 2)) != MSA_OK ||
+      (st = check_buf(idx_new, nt * MSA_HEAD_DIM * 2)) != MSA_OK)
+    return st;
   InsArgs a{};
   a.idx_data = const_cast<uint8_t*>(cache->idx_data);
   a.idx_scale = const_cast<uint8_t*>(cache->idx_scale);
@@ -344,6 +494,8 @@ msa_status msa_kv_insert(const msa_cache* cache, const msa_seqs* seqs, const uin
 
 msa_status msa_get_last_error(void* ws, msa_stream_t stream, int32_t* detail) {
   if (!ws) return MSA_ERR_WORKSPACE;
+  const msa_status st = check_buf(ws, sizeof(Flags), MSA_ERR_WORKSPACE);
+  if (st != MSA_OK) return st;
   const cudaStream_t s = (cudaStream_t)stream;
   Flags h{};
   if (cudaMemcpyAsync(&h, ws, sizeof(Flags), cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -361,6 +513,8 @@ msa_status msa_get_last_error(void* ws, msa_stream_t stream, int32_t* detail) {
 
 msa_status msa_debug_nvfp4_table(uint8_t* out, msa_stream_t stream) {
   if (!out || !aligned16(out)) return MSA_ERR_INVALID_ARG;
+  const msa_status st = check_buf(out, 256 * 16);
+  if (st != MSA_OK) return st;
   return cuda_status(launch_nvfp4_table(out, (cudaStream_t)stream));
 }
 

@@ -15,8 +15,8 @@
 //     tiled TMA loads of the K and V codes (64-byte swizzle) and two bulk
 //     copies of their scales into a ring of shared-memory stages;
 //   warps 0-3 (decoders): thread = key row, warp w decoding rows
-//     32w..32w+31.  K is decoded signed (dq8s) straight into tensor memory
-//     (one A operand: 4 MMAs per block rather than 8 for a split by sign --
+//     32w..32w+31.  K is decoded signed (dq8) straight into tensor memory
+//     (dq8; one A operand: 4 MMAs per block rather than 8 for a split by sign --
 //     the MMA-issuing thread is the scarcer resource here); V is decoded
 //     signed into shared memory as E4M3 rows of 128
 //     bytes with the 128-byte swizzle -- the A operand of O^T = V^T P^T in
@@ -31,8 +31,8 @@
 //     of quarter q (thread = key), masks keys after the query position,
 //     takes the per-head block maximum (warp reduction, then across the four
 //     quarters through shared memory), and writes P = 2^(s*c - m + 4) split
-//     into two E4M3 terms
-//     (P_hi + P_lo holds P to about 2^-8 relative) as 16-byte rows per key.
+//     into two E4M3 terms through FP16 (P_hi + P_lo holds P to about 2^-8
+//     relative) as 16-byte rows per key.
 //     The running maximum m is raised lazily -- only when a block's maximum
 //     exceeds it by more than 2^4 -- so that P stays below 2^8 (inside E4M3)
 //     and O^T in tensor memory is rescaled rarely.  At the end of an item
@@ -100,20 +100,6 @@ int attn_splits(long long rows, int num_sms) {
   return s;
 }
 
-// Signed NVFP4 -> E4M3 decode of 8 codes (element n in nibble n) with table
-// row r = lut[scale byte] (signed scales included): o0 = elements 0..3, o1 =
-// 4..7.  The magnitudes come from one prmt per 4 codes; the sign byte 0x80
-// of a negative code comes from a prmt with sign replication on a table of
-// 0x7F bytes (0x7F for a non-negative code, 0x00 for a negative one), plus 1
-// and inverted, and is xor-ed in (so a negative scale flips it back).
-__device__ __forceinline__ void dq8s(uint32_t w, uint2 r, uint32_t& o0, uint32_t& o1) {
-  const uint32_t mag = w & 0x77777777u;
-  const uint32_t s0 = prmt(0x7F7F7F7Fu, 0x7F7F7F7Fu, w);
-  const uint32_t s1 = prmt(0x7F7F7F7Fu, 0x7F7F7F7Fu, hi16(w));
-  o0 = prmt(r.x, r.y, mag) ^ (~(s0 + 0x01010101u) & 0x80808080u);
-  o1 = prmt(r.x, r.y, hi16(mag)) ^ (~(s1 + 0x01010101u) & 0x80808080u);
-}
-
 // Shared-memory descriptor, MN-major operand with the 128-byte swizzle: rows
 // of 128 bytes (128 M elements) per K index, 8-row atoms `sbo` bytes apart.
 __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t addr, uint32_t sbo) {
@@ -129,23 +115,20 @@ __device__ __forceinline__ uint64_t desc_mn_plain(uint32_t addr, uint32_t lbo, u
          ((uint64_t)(sbo >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
-// D[tmem] (+)= A[smem] * B[smem] (E4M3), one K = 32 slice.
-__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-      "l"(ad), "l"(bd), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Split x (0 <= x <= 256) into hi + lo with hi holding 4 significant bits
-// (Veltkamp's splitting with the factor 2^20 + 1 for a 24-bit significand);
-// both are then exact or rounded once as E4M3.
-__device__ __forceinline__ void split4(float x, float& hi, float& lo) {
-  const float c = __fmul_rn(1048577.f, x);
-  hi = __fsub_rn(c, __fsub_rn(c, x));
-  lo = __fsub_rn(x, hi);
+// P (two values, 0 <= p <= 256) as the sum of two E4M3 terms, each pair
+// packed in 16 bits (low byte = first value): P is rounded to FP16 (relative
+// error 2^-11), hi = E4M3(P16); P16 - hi is exact in FP16 (hi lies within
+// 2^-4 of P16) and lo = E4M3(P16 - hi), so hi + lo holds P to about 2^-8.
+__device__ __forceinline__ void p_split_e4m3x2(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  uint32_t p16, back, r16;
+  uint16_t h8, l8;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(p16) : "f"(p1), "f"(p0));
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;\n" : "=h"(h8) : "r"(p16));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(back) : "h"(h8));
+  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(r16) : "r"(p16), "r"(back));
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;\n" : "=h"(l8) : "r"(r16));
+  hi = h8;
+  lo = l8;
 }
 
 // 2^x with the SFU's approximate exp2 (relative error below 2^-22).
@@ -155,9 +138,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t fp8x2(float a, float b) {
-  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-}
 
 __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_dyn[];
@@ -475,10 +455,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           const float p1 = ex2(fmaf(s[2 * h2 + 1], c, -mo.y));
           lt[2 * h2] += p0;
           lt[2 * h2 + 1] += p1;
-          float a0, b0, a1, b1;
-          split4(p0, a0, b0);
-          split4(p1, a1, b1);
-          const uint32_t hw = fp8x2(a0, a1), lw = fp8x2(b0, b1);
+          uint32_t hw, lw;
+          p_split_e4m3x2(p0, p1, hw, lw);
           if (h2 & 1) { ph[h2 >> 1] |= hw << 16; pl[h2 >> 1] |= lw << 16; }
           else { ph[h2 >> 1] = hw; pl[h2 >> 1] = lw; }
         }
@@ -632,10 +610,10 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           const uint32_t sb = (cix < 2 ? ksc.x : ksc.y) >> (16 * (cix & 1));
           const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
           uint32_t o[8];
-          dq8s(w4.x, r0, o[0], o[1]);
-          dq8s(w4.y, r0, o[2], o[3]);
-          dq8s(w4.z, r1, o[4], o[5]);
-          dq8s(w4.w, r1, o[6], o[7]);
+          dq8(w4.x, r0, o[0], o[1]);
+          dq8(w4.y, r0, o[2], o[3]);
+          dq8(w4.z, r1, o[4], o[5]);
+          dq8(w4.w, r1, o[6], o[7]);
           tmem_st8(abase + 8 * cix, o);
         }
         // V signed, as E4M3 into the 128-byte V row of this key (16-byte
@@ -648,10 +626,10 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           const uint32_t sb = (cix < 2 ? vsc.x : vsc.y) >> (16 * (cix & 1));
           const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
           uint32_t o[8];
-          dq8s(w4.x, r0, o[0], o[1]);
-          dq8s(w4.y, r0, o[2], o[3]);
-          dq8s(w4.z, r1, o[4], o[5]);
-          dq8s(w4.w, r1, o[6], o[7]);
+          dq8(w4.x, r0, o[0], o[1]);
+          dq8(w4.y, r0, o[2], o[3]);
+          dq8(w4.z, r1, o[4], o[5]);
+          dq8(w4.w, r1, o[6], o[7]);
           // code chunk cix = dims 32cix..32cix+31 = V chunks 2cix, 2cix+1
           *reinterpret_cast<uint4*>(vrow + (((2 * cix) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<uint4*>(vrow + (((2 * cix + 1) ^ (row & 7)) << 4)) =
@@ -684,24 +662,19 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   if (warp == kAttMmaWarp) tmem_dealloc(tmem, kAttTmemCols);
 }
 
-cudaError_t launch_attn(const AttnArgs& a, int num_sms, cudaStream_t st) {
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   const size_t smem = attn_smem_bytes();
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(attn_kernel), kAttThreads, smem,
-                                 kAttTmemCols);
-  attn_kernel<<<num_sms * per_sm, kAttThreads, smem, st>>>(a);
+  int grid = 0;
+  cudaError_t e = persistent_grid(reinterpret_cast<const void*>(attn_kernel), kAttThreads, smem,
+                                  kAttTmemCols, &grid);
+  if (e != cudaSuccess) return e;
+  attn_kernel<<<grid, kAttThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 // ----------------------------------------------------- parity debug hook --
-// The kernels' NVFP4 -> E4M3 table through the signed decode the V operand
-// uses (dq8s): out[s*16 + c] for scale byte s and code c.
+// The kernels' NVFP4 -> E4M3 table through the signed decode every kernel
+// uses (dq8): out[s*16 + c] for scale byte s and code c.
 __global__ void nvfp4_table_kernel(uint8_t* out) {
   __shared__ uint2 lut[256];
   build_nvfp4_lut(lut, threadIdx.x, blockDim.x);
@@ -709,8 +682,8 @@ __global__ void nvfp4_table_kernel(uint8_t* out) {
   const int s = threadIdx.x;   // 256 threads, one scale byte each
   const uint2 r = lut[s];
   uint32_t o[4];
-  dq8s(0x76543210u, r, o[0], o[1]);   // codes 0..7 in element order
-  dq8s(0xFEDCBA98u, r, o[2], o[3]);   // codes 8..15
+  dq8(0x76543210u, r, o[0], o[1]);   // codes 0..7 in element order
+  dq8(0xFEDCBA98u, r, o[2], o[3]);   // codes 8..15
   uint4* dst = reinterpret_cast<uint4*>(out + s * 16);
   *dst = make_uint4(o[0], o[1], o[2], o[3]);
 }

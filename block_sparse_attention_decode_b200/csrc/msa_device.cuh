@@ -401,3 +401,93 @@ __device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, float (&v)[4 * R
 }
 
 }  // namespace msa
+
+namespace msa {
+
+// D[tmem] (+)= A[smem] * B[smem]^T (E4M3, kind::f8f6f4), one K = 32 slice.
+__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T (FP16, kind::f16), one K = 16 slice.
+__device__ __forceinline__ void tc_mma_ss_f16(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Signed NVFP4 -> E4M3 decode of 8 codes w (element n in nibble n) with the
+// table row r = lut[scale byte] (E4M3 of the 8 E2M1 magnitudes times the
+// scale, sign of the scale included): o0 = elements 0..3, o1 = 4..7, low
+// byte first.  The magnitudes come from one prmt per four codes.  The code
+// signs sit in bit 3 of each nibble: those of the odd elements are already
+// bit 7 of the bytes of w, those of the even elements bit 7 of the bytes of
+// w << 4, and one byte permute per four codes interleaves them into bit 7 of
+// the output bytes, where an xor applies them.  Nine operations per 8 codes.
+__device__ __forceinline__ void dq8(uint32_t w, uint2 r, uint32_t& o0, uint32_t& o1) {
+  const uint32_t mag = w & 0x77777777u;
+  const uint32_t u = w << 4;
+  const uint32_t s0 = prmt(u, w, 0x5140u);    // bytes: signs of elements 0, 1, 2, 3
+  const uint32_t s1 = prmt(u, w, 0x7362u);    // elements 4, 5, 6, 7
+  o0 = prmt(r.x, r.y, mag) ^ (s0 & 0x80808080u);
+  o1 = prmt(r.x, r.y, mag >> 16) ^ (s1 & 0x80808080u);
+}
+
+// Warp-wide 16x256b TMEM load, 8 repetitions (64 columns): thread (g =
+// lane/4, t = lane%4) receives for c < 8: v[4c+0] = (lane g, col 8c+2t),
+// v[4c+1] = (lane g, col 8c+2t+1), v[4c+2] = (lane g+8, col 8c+2t),
+// v[4c+3] = (lane g+8, col 8c+2t+1), lanes relative to taddr's lane.
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Warp-wide 32x32b TMEM load of 32 consecutive columns: lane l receives
+// columns c..c+31 of TMEM lane (taddr.lane + l).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Max of n floats (n a multiple of 2) with three-input max instructions.
+template <int N>
+__device__ __forceinline__ float max_of(const float* v) {
+  float m = fmaxf(v[0], v[1]);
+#pragma unroll
+  for (int i = 2; i + 1 < N; i += 2) m = fmax3(m, v[i], v[i + 1]);
+  return m;
+}
+
+}  // namespace msa

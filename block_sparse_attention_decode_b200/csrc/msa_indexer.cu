@@ -4,92 +4,93 @@
 // max-pooled to one score per 128-token block).
 // post = vLLM 為 MiniMax-M3.1-Flash 提供 Day-0 支援 (hot.atechcom.net).
 //
-// Per page (= one 128-token block) the scores are one dense FP8 contraction
-//   D[128 keys x NQ queries] = K_page[128 x 128] * Qi[NQ x 128]^T
-// with the keys as the M side (the block max is a reduction over TMEM
-// lanes) and a chunk of NQ index queries (T tokens x 4 groups, padded to
-// 16, 32, 64, 128 or 256) as the N side.
+// Per page (= one 128-token block) the scores are one dense contraction
+//   D[M queries x 128 keys] = Qi[M x 128] * K_page[128 keys x 128]^T
+// with a tile of index queries as the M side (T tokens x 4 groups; M = 64
+// when the tile holds at most 64 index queries, else tiles of 128) and the
+// page's keys as the N side.  Each query's row of D then sits in one TMEM
+// lane, so the block max is a reduction along the lane's columns: inside the
+// thread, plus two shuffles when a 16x256b load spreads a row over four
+// threads.  With M = 64 the accumulator occupies lanes 0-15 of each 32-lane
+// quarter (rows 16q..16q+15 in quarter q).
 //
 // Work split: the pages of all sequences form one flat list, cut into chunks
-// of kChunkPages; a work item is (query tile of NQ index queries, chunk).
-// A launch may score only part `part` of `nparts` of every sequence's blocks
-// (the context split of [post, "NVFP4 indexer DCP"]); the flat list then
-// holds only those blocks.
-// Persistent CTAs (two per SM) take items from a counter in the workspace
-// header as they go, so that CTAs sharing an SM -- which the warp schedulers
-// do not serve equally -- and ragged batches still finish together; the last
-// CTA to finish resets the counter.  Warp roles inside a CTA, all running a
-// few pages apart:
-//   warp 12 (producer): per page one tiled TMA load of the codes (64-byte
+// of kChunkPages; a work item is (query tile, chunk).  A launch may score
+// only part `part` of `nparts` of every sequence's blocks (the context split
+// of [post, "NVFP4 indexer DCP"]); the flat list then holds only those
+// blocks.  Persistent CTAs take items from a counter in the workspace header
+// as they go (ragged batches and CTAs sharing an SM still finish together);
+// the last CTA to finish resets the counter.  Warp roles, a few pages apart:
+//   warp 8 (producer): per page one tiled TMA load of the codes (64-byte
 //     swizzle, so that row-per-thread reads are bank-conflict free) and one
-//     bulk copy of the scales into a ring of shared-memory stages;
-//   warps 0-3 (decoders): thread = key row (= TMEM lane).  NVFP4 rows are
-//     decoded by sign: K+ holds E4M3(|v|) of the positive elements, K- of the
-//     negative ones (one prmt per 4 codes each, see dq8_split), and both go
-//     straight to tensor memory with tcgen05.st into one of two A buffers --
-//     the A operand never touches shared memory, and page k+1 is decoded
-//     while page k's MMAs run;
-//   warp 13 (MMA): one thread issues per page 4 tcgen05.mma with A = K+ and 4
-//     with A = K- and the negate-A bit (K = 32 each, A from TMEM, B = the
-//     queries in shared memory) into a double-buffered TMEM accumulator;
-//   warps 4-11 (epilogue, two groups of four taking the even and the odd
-//     pages, so that two pages are reduced at once): warp 4+4j+q reads the
-//     accumulator lanes of quarter q, masks keys after each query's position,
-//     and reduces over keys: in-thread over the four keys a 16x256b load
-//     gives each thread, then xor shuffles across lane groups; after a
-//     rendezvous on an mbarrier each warp combines the four quarters' partial
-//     maxima of a quarter of the columns and writes those block scores.
+//     bulk copy of the scales into a ring of shared-memory stages (FP8 index
+//     keys: one TMA load with the 128-byte swizzle, which is already the
+//     MMA's B operand);
+//   warps 0-3 (decoders): thread = key row.  NVFP4 rows are decoded to signed
+//     E4M3 (dq8: a table row per scale byte, byte permutes for magnitudes
+//     and signs) and stored as 128-byte rows with the 128-byte swizzle -- the
+//     K-major B operand -- into one of two buffers, so page k+1 is decoded
+//     while page k's MMAs run.  When the query tile changes they also stage
+//     the tile's index queries (the A operand) into one of two buffers;
+//   warp 9 (MMA): one thread issues per page 4 tcgen05.mma of K = 32 (E4M3;
+//     8 of K = 16 for FP16) into one of two TMEM accumulators;
+//   warps 4-7 (epilogue): warp 4+q reads the accumulator lanes of quarter q,
+//     masks keys after each query's position, takes each query's maximum
+//     over the page's keys and writes the block score.
 // Every wait is a bounded mbarrier wait; on a timeout a thread records
 // MSA_ERR_TIMEOUT and leaves its loop, and TMEM is freed before exit.
 //
 // Modes (the template parameter MODE):
-//   kIdxNvfp4  NVFP4 keys re-rounded to E4M3, FP8 MMA (the sign split above);
-//   kIdxFp8    E4M3 keys, copied to TMEM as they are;
+//   kIdxNvfp4  NVFP4 keys re-rounded to E4M3, FP8 MMA (the decode above);
+//   kIdxFp8    E4M3 keys, scored from the TMA buffer as they are;
 //   kIdxF16    NVFP4 keys decoded exactly to FP16 (e2m1 x scale needs no
 //              rounding in FP16) and scored with FP16 MMA against the index
 //              queries widened to FP16 -- the exact scores of [post, "NVIDIA
-//              Rubin optimized MSA"].  One A buffer holds the 128 FP16 values
-//              of each row in 64 columns; the queries take two 128-byte
-//              swizzled K-halves in shared memory; 8 MMAs of K = 16 per page.
+//              Rubin optimized MSA"].  Query and key rows are 256 bytes, held
+//              as two 128-byte K-halves; 8 MMAs of K = 16 per page.
 #include "msa_internal.h"
 
 namespace msa {
 
-constexpr int kIdxDecoders = 4;             // one per TMEM lane quarter, full rows
-constexpr int kIdxEpilogue = 4;             // per group: one per TMEM lane quarter
-constexpr int kIdxEpiWarp0 = 4;             // two groups: even and odd pages
-constexpr int kIdxProducerWarp = 12;
-constexpr int kIdxMmaWarp = 13;
-constexpr int kABufCols = 64;               // TMEM columns of one A buffer (K+ | K-, or FP16)
-constexpr int kACols = 2 * kABufCols;       // two A buffers
+constexpr int kIdxDecWarps = 4;             // warps 0-3: one key row per thread
+constexpr int kIdxEpiWarp0 = 4;             // warps 4-7: one per TMEM lane quarter
+constexpr int kIdxProducerWarp = 8;
+constexpr int kIdxMmaWarp = 9;
+static_assert(kIdxThreads == 10 * 32, "warp roles");
 
 enum : int { kPageLoad = 0, kPageMasked = 1, kPageBad = 2, kPageEnd = 3 };
 constexpr int kChunkPages = 8;              // pages per work item
+constexpr int kInfoRing = 8;                // per-page info slots (decoders -> MMA, epilogue)
+constexpr int kIdxTmemCols = 256;           // two accumulators of 128 columns
 
-struct IdxLayout {
-  int qbuf, raw, raw_stride, lut, red, bars, meta, tinfo, pinfo, tslot, prefix, scratch, total;
+template <int MODE>
+struct IdxCfg {
+  static constexpr bool kFp8 = MODE == kIdxFp8;
+  static constexpr bool kF16 = MODE == kIdxF16;
+  static constexpr int kRow = kF16 ? 256 : 128;            // bytes per query / key row
+  static constexpr int kRaw = kFp8 ? kBlock * kDim : kPageCodes + kPageScales;
+  static constexpr int kRawStride = (kRaw + 1023) / 1024 * 1024;
+  static constexpr int kStages = kFp8 ? 5 : (kF16 ? 3 : 4);   // raw pages in flight
+  static constexpr int kNB = kFp8 ? 0 : 2;                 // decoded key pages (B operand), page k in k % 2
+  static constexpr int kBBytes = kBlock * kRow;
 };
 
-// Bytes of one raw page in shared memory (codes [+ scales]), 1024-aligned.
-__host__ __device__ inline int raw_stage_stride(bool fp8idx) {
-  return fp8idx ? kBlock * kDim : ((kPageCodes + kPageScales + 1023) / 1024) * 1024;
-}
+struct IdxLayout {
+  int qbuf, raw, bbuf, lut, bars, meta, pinfo, tslot, prefix, scratch, total;
+};
 
-// Bytes of one query row in shared memory: E4M3, or two 128-byte K-halves of FP16.
-__host__ __device__ constexpr int q_row_bytes(int mode) { return mode == kIdxF16 ? 256 : 128; }
-
-__host__ __device__ inline IdxLayout idx_layout(int nq, int mode, int batch) {
+template <int MODE, int M>
+__host__ __device__ inline IdxLayout idx_layout(int batch) {
+  using C = IdxCfg<MODE>;
   IdxLayout L;
   int off = 0;
-  L.qbuf = off;    off += 2 * nq * q_row_bytes(mode);     // nq % 8 == 0 -> 1024-aligned
-  L.raw_stride = raw_stage_stride(mode == kIdxFp8);
-  L.raw = off;     off += kIdxRawStages * L.raw_stride;
-  L.lut = off;     off += 256 * 8;
-  L.red = off;     off += 2 * kIdxEpilogue * nq * 4;          // [group][quarter][nq]
-  L.bars = off;    off += (2 * kIdxRawStages + 10) * 8;
-  L.meta = off;    off += 4 * kIdxRawStages * 4;           // per stage: b, i, kind, tile
-  L.tinfo = off;   off += 2 * 2 * 4;                       // per A buffer: what, qsel
-  L.pinfo = off;   off += 4 * 8 * 4;                       // ring of 4: b, i, kind, L, tile
+  L.qbuf = off;    off += 2 * M * C::kRow;                 // two query tiles (multiples of 1024)
+  L.raw = off;     off += C::kStages * C::kRawStride;
+  L.bbuf = off;    off += C::kNB * C::kBBytes;
+  L.lut = off;     off += MODE == kIdxNvfp4 ? 256 * 8 : 0;
+  L.bars = off;    off += (2 * C::kStages + 8) * 8;
+  L.meta = off;    off += C::kStages * 8 * 4;              // per stage: b, i, kind, tile, L
+  L.pinfo = off;   off += kInfoRing * 8 * 4;               // per page: b, i, kind, tile, L, qsel
   L.tslot = off;   off += 16;
   L.prefix = off;  off += (batch + 1) * 4;
   L.scratch = off; off += kIdxThreads * 4;
@@ -97,26 +98,14 @@ __host__ __device__ inline IdxLayout idx_layout(int nq, int mode, int batch) {
   return L;
 }
 
-// N of the MMA: with A in tensor memory and M = 128, N is a multiple of 16
-// from 16 to 256 (the tcgen05.mma shape table), so one query token's 4 index
-// queries are padded to 16.
-int idx_nq(int T) {
-  const int nq = kG * T;
-  if (nq <= 16) return 16;
-  if (nq <= 32) return 32;
-  if (nq <= 64) return 64;
-  if (nq <= 128) return 128;
-  return 256;
-}
+// Index queries per tile: a tile is the M side of the MMA.
+int idx_tile_queries(int T) { return kG * T <= 64 ? 64 : 128; }
 
 size_t indexer_smem_bytes(int mode, int batch, int T) {
-  return (size_t)idx_layout(idx_nq(T), mode, batch).total;
-}
-
-__host__ __device__ constexpr int pow2_at_least(int x) {
-  int p = 32;
-  while (p < x) p *= 2;
-  return p;
+  const bool m64 = idx_tile_queries(T) == 64;
+  if (mode == kIdxFp8) return (size_t)(m64 ? idx_layout<kIdxFp8, 64>(batch) : idx_layout<kIdxFp8, 128>(batch)).total;
+  if (mode == kIdxF16) return (size_t)(m64 ? idx_layout<kIdxF16, 64>(batch) : idx_layout<kIdxF16, 128>(batch)).total;
+  return (size_t)(m64 ? idx_layout<kIdxNvfp4, 64>(batch) : idx_layout<kIdxNvfp4, 128>(batch)).total;
 }
 
 // The part of a sequence of length L this launch scores: logical blocks
@@ -137,7 +126,7 @@ __device__ __forceinline__ int part_blocks(const IdxArgs& a, int L, int* first) 
 
 // Exclusive prefix over the number of blocks this launch scores in each
 // sequence, in shared memory (prefix[B] = total pages).  Invalid lengths
-// count as 0 blocks and are reported once (by CTA (0,0)).
+// count as 0 blocks and are reported once (by CTA 0).
 __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (a.B + nt - 1) / nt;
@@ -147,7 +136,7 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
     const int L = a.seq_lens[b];
     int first;
     const int nb = part_blocks(a, L, &first);
-    if ((L < a.T || L > a.max_pages * kBlock) && blockIdx.x == 0 && blockIdx.y == 0)
+    if ((L < a.T || L > a.max_pages * kBlock) && blockIdx.x == 0)
       report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
     sum += nb;
   }
@@ -170,31 +159,32 @@ __device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
 
 __device__ __forceinline__ void sts128(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
-template <int NQ, int MODE>
+// Instruction descriptor of the page MMA: M x 128, fp32 accumulate, both
+// operands K-major; E4M3 (kind::f8f6f4) or FP16 (kind::f16), whose format
+// fields both read 0.
+template <int M>
+__host__ __device__ constexpr uint32_t idx_idesc() { return idesc_e4m3_f32(M, kBlock); }
+
+template <int MODE, int M>
 __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_constant__ IdxArgs a) {
-  constexpr bool FP8IDX = MODE == kIdxFp8;
-  constexpr bool F16 = MODE == kIdxF16;
-  constexpr int kQRow = q_row_bytes(MODE);
-  constexpr int kND = NQ <= 64 ? 2 : 1;                      // accumulator buffers
-  constexpr int kCols = pow2_at_least(kACols + kND * NQ);    // TMEM columns
-  constexpr int kChunk = NQ < 32 ? NQ : (NQ >= 128 ? 16 : 32);   // columns per TMEM load
+  using C = IdxCfg<MODE>;
+  constexpr bool FP8 = C::kFp8, F16 = C::kF16;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
-  const IdxLayout Ly = idx_layout(NQ, MODE, a.B);
+  const IdxLayout Ly = idx_layout<MODE, M>(a.B);
   uint8_t* qbuf = smem + Ly.qbuf;
   uint8_t* raw = smem + Ly.raw;
+  uint8_t* bbuf = smem + Ly.bbuf;
   uint2* lut = reinterpret_cast<uint2*>(smem + Ly.lut);
-  float* red = reinterpret_cast<float*>(smem + Ly.red);            // [group][quarter][NQ]
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + Ly.bars);
-  uint64_t* raw_empty = raw_full + kIdxRawStages;
-  uint64_t* a_full = raw_empty + kIdxRawStages;                    // decoders -> MMA [2]
-  uint64_t* a_empty = a_full + 2;                                  // MMA -> decoders [2]
-  uint64_t* acc_full = a_empty + 2;                                // MMA -> epilogue [2]
-  uint64_t* acc_empty = acc_full + 2;                              // epilogue -> MMA [2]
-  uint64_t* red_full = acc_empty + 2;                              // group rendezvous [2]
-  int* meta = reinterpret_cast<int*>(smem + Ly.meta);              // [stage][b, i, kind, tile]
-  int* tinfo = reinterpret_cast<int*>(smem + Ly.tinfo);            // [A buffer][what, qsel]
-  int* pinfo = reinterpret_cast<int*>(smem + Ly.pinfo);            // [k % 4][b, i, kind, L, tile]
+  uint64_t* raw_empty = raw_full + S;
+  uint64_t* b_full = raw_empty + S;      // [2] decoders -> MMA: page k ready (k % 2)
+  uint64_t* b_empty = b_full + 2;        // [2] MMA -> decoders: page k consumed
+  uint64_t* d_full = b_empty + 2;        // [2] MMA -> epilogue
+  uint64_t* d_empty = d_full + 2;        // [2] epilogue -> MMA
+  int* meta = reinterpret_cast<int*>(smem + Ly.meta);
+  int* pinfo = reinterpret_cast<int*>(smem + Ly.pinfo);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
   int* prefix = reinterpret_cast<int*>(smem + Ly.prefix);
   int* scratch = reinterpret_cast<int*>(smem + Ly.scratch);
@@ -203,21 +193,20 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
 
   if (MODE == kIdxNvfp4) build_nvfp4_lut(lut, tid, blockDim.x);
   if (tid == 0) {
-    for (int s = 0; s < kIdxRawStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], kIdxDecoders);
+      mbar_init(&raw_empty[s], FP8 ? 1 : kIdxDecWarps);   // FP8: released by the MMA
     }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&a_full[x], kIdxDecoders);
-      mbar_init(&a_empty[x], 1);
-      mbar_init(&acc_full[x], 1);
-      mbar_init(&acc_empty[x], kIdxEpilogue);
-      mbar_init(&red_full[x], kIdxEpilogue);
+      mbar_init(&b_full[x], kIdxDecWarps);
+      mbar_init(&b_empty[x], 1);
+      mbar_init(&d_full[x], 1);
+      mbar_init(&d_empty[x], 4);
     }
     mbar_fence_init();
   }
   if (warp == kIdxMmaWarp) {
-    tmem_alloc(tslot, kCols);
+    tmem_alloc(tslot, kIdxTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -226,7 +215,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   const uint32_t tmem = *tslot;
 
   const int total = prefix[a.B];
-  const int gy = (kG * a.T + NQ - 1) / NQ;                  // query tiles
+  const int nq_all = kG * a.T;                                // index queries per sequence
+  const int gy = (nq_all + M - 1) / M;                        // query tiles
   const int nchunks = (total + kChunkPages - 1) / kChunkPages;
   const int items = nchunks * gy;
   const long long ctx = (long long)a.max_pages * kBlock;
@@ -234,11 +224,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   if (warp == kIdxProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int k = 0;                                  // page slot (stage k % kIdxRawStages)
+      int k = 0;                                  // page slot (stage k % S)
       bool ok = true;
       auto slot = [&](int kk) -> bool {           // wait until stage kk % S is free
-        return kk < kIdxRawStages ||
-               mbar_wait(&raw_empty[kk % kIdxRawStages], ((kk / kIdxRawStages) - 1) & 1);
+        return kk < S || mbar_wait(&raw_empty[kk % S], ((kk / S) - 1) & 1);
       };
       int first_b = -1, first = 0;                // part_blocks of sequence first_b
       int item = atomicAdd(&a.work[0], 1);
@@ -246,7 +235,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         const int nxt = atomicAdd(&a.work[0], 1);  // claimed early: its latency overlaps this item
         const int y = item / nchunks, p0 = (item % nchunks) * kChunkPages;
         const int p1 = min(total, p0 + kChunkPages);
-        const int t_last = min(a.T - 1, (y * NQ + NQ - 1) >> 2);
+        const int t_last = (min(nq_all, (y + 1) * M) - 1) >> 2;
         int b;
         {  // prefix[b] <= p0 < prefix[b+1]
           int l = 0, r = a.B;
@@ -256,7 +245,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         int li = p0 - prefix[b];                    // index among this part's blocks of b
         for (int pg = p0; pg < p1; ++pg, ++k, ++li) {
           if (!slot(k)) { report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1); ok = false; break; }
-          const int s = k % kIdxRawStages;
+          const int s = k % S;
           while (li >= prefix[b + 1] - prefix[b]) { li -= prefix[b + 1] - prefix[b]; ++b; }
           const int L = a.seq_lens[b];
           if (b != first_b) {                       // first block of b's part
@@ -268,36 +257,31 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + i]
                                            : (long long)b * a.max_pages + i;
           if (i * kBlock > L - a.T + t_last) {
-            kind = kPageMasked;
+            kind = kPageMasked;                     // no key of the block is visible to the tile
           } else if (p < 0 || p >= a.num_pages) {
             report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)p);
             kind = kPageBad;
           }
-          meta[4 * s + 0] = b;
-          meta[4 * s + 1] = i;
-          meta[4 * s + 2] = kind;
-          meta[4 * s + 3] = y;
-          uint8_t* dst = raw + s * Ly.raw_stride;
+          int* m = meta + 8 * s;
+          m[0] = b; m[1] = i; m[2] = kind; m[3] = y; m[4] = L;
+          uint8_t* dst = raw + s * C::kRawStride;
           if (kind == kPageLoad) {
-            if (FP8IDX) {
-              mbar_expect_tx(&raw_full[s], kBlock * kDim);
-              tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
-            } else {
-              mbar_expect_tx(&raw_full[s], kPageCodes + kPageScales);
-              tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
-              bulk_g2s(dst + kPageCodes, a.idx_scale + p * kPageScales, kPageScales, &raw_full[s]);
-            }
+            mbar_expect_tx(&raw_full[s], C::kRaw);
+            tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
+            if (!FP8) bulk_g2s(dst + kPageCodes, a.idx_scale + p * kPageScales, kPageScales, &raw_full[s]);
           } else {
             mbar_arrive(&raw_full[s]);
           }
         }
         item = nxt;
       }
-      // two end markers: one for each epilogue group
-      for (int e = 0; e < 2 && ok; ++e, ++k) {
-        if (!slot(k)) { report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1); break; }
-        meta[4 * (k % kIdxRawStages) + 2] = kPageEnd;
-        mbar_arrive(&raw_full[k % kIdxRawStages]);
+      if (ok) {   // end marker
+        if (!slot(k)) {
+          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1);
+        } else {
+          meta[8 * (k % S) + 2] = kPageEnd;
+          mbar_arrive(&raw_full[k % S]);
+        }
       }
       // every CTA has made its last claim once all have arrived here
       __threadfence();
@@ -309,199 +293,179 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   } else if (warp == kIdxMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = F16 ? idesc_f16_f32(128, NQ) : idesc_e4m3_f32(128, NQ);
-      constexpr uint32_t idesc_neg = idesc | (1u << 13);     // negate A
-      // B descriptors of the two query buffers; a K slice (32 E4M3 or 16
-      // FP16 values) starts 32 bytes further (2 in the descriptor's 16-byte
-      // address units); FP16 queries continue in a second 128-byte-wide tile
-      // NQ rows further for K >= 64.
-      const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(qbuf));
-      const uint64_t bdesc1 = desc_kmajor_sw128(smem_u32(qbuf + NQ * kQRow));
-      constexpr uint64_t kHalf = (uint64_t)(NQ * 128 / 16);    // second K-half, descriptor units
-      // Page k uses A buffer k % 2 and accumulator k % kND; with two
-      // accumulators one commit (to acc_full[k % 2]) releases both.
-      auto issue = [&](int k, int ab, int x, int& ends) -> bool {
-        if (!mbar_wait(&a_full[ab], (k >> 1) & 1)) { report(a.flags, 5, 2); return false; }
-        if (k >= kND && !mbar_wait(&acc_empty[x], ((k / kND) - 1) & 1)) { report(a.flags, 5, 3); return false; }
+      constexpr uint32_t idesc = idx_idesc<M>();
+      for (int k = 0;; ++k) {
+        const int x = k & 1;                       // accumulator and page-ready barrier
+        if (!mbar_wait(&b_full[x], (k >> 1) & 1)) { report(a.flags, 5, 2); break; }
+        if (k >= 2 && !mbar_wait(&d_empty[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 3); break; }
         tc_fence_after();
-        const int what = tinfo[2 * ab];            // 0 = MMA, 1 = nothing to score, 2 = end
-        ends += (what == 2);
-        if (what == 0) {
-          const uint32_t d = tmem + kACols + x * NQ;
-          const uint32_t ta = tmem + ab * kABufCols;
-          const uint64_t bd = tinfo[2 * ab + 1] ? bdesc1 : bdesc0;
+        const int* pf = pinfo + 8 * (k % kInfoRing);
+        const int kind = pf[2], qsel = pf[5];
+        if (kind == kPageLoad) {
+          const uint32_t d = tmem + (uint32_t)(x * kBlock);
+          const uint32_t qa = smem_u32(qbuf + qsel * M * C::kRow);
+          const uint32_t kb = FP8 ? smem_u32(raw + (k % S) * C::kRawStride)
+                                  : smem_u32(bbuf + x * C::kBBytes);
           if constexpr (F16) {
+            // K-half h of the queries starts M rows further, of the keys 128 rows further
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              tc_mma_f16_ts(d, ta + 8 * kk, bd + (kk >> 2) * kHalf + 2 * (kk & 3), idesc, kk > 0);
+              tc_mma_ss_f16(d, desc_kmajor_sw128(qa + (kk >> 2) * M * 128) + 2 * (kk & 3),
+                            desc_kmajor_sw128(kb + (kk >> 2) * kBlock * 128) + 2 * (kk & 3), idesc, kk > 0);
           } else {
+            const uint64_t ad = desc_kmajor_sw128(qa), bd = desc_kmajor_sw128(kb);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc, kk > 0);
-          }
-          if (MODE == kIdxNvfp4) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 32 + 8 * kk, bd + 2 * kk, idesc_neg, 1);
+            for (int kk = 0; kk < 4; ++kk) tc_mma_ss(d, ad + 2 * kk, bd + 2 * kk, idesc, kk > 0);
           }
         }
-        if constexpr (kND == 2) {
-          tc_commit(&acc_full[ab]);
-        } else {
-          tc_commit(&a_empty[ab]);
-          tc_commit(&acc_full[x]);
-        }
-        return true;
-      };
-      int ends = 0;
-      for (int k = 0; ends < 2; k += 2) {
-        if (!issue(k, 0, 0, ends)) break;
-        if (ends < 2 && !issue(k + 1, 1, kND == 2 ? 1 : 0, ends)) break;
+        tc_commit(&d_full[x]);
+        if (kind == kPageEnd) break;
+        if (FP8) tc_commit(&raw_empty[k % S]);   // the stage was the B operand
+        tc_commit(&b_empty[x]);                   // page k consumed (and its B buffer free)
       }
     }
   } else if (warp >= kIdxEpiWarp0) {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3, group = (warp - kIdxEpiWarp0) >> 2;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);   // this warp's TMEM lanes
-    const int g = lane >> 2, tq = lane & 3;
-    // With two accumulators the groups alternate pages; with one (NQ >= 128)
-    // group 0 takes every page, since a waiter two phases ahead of an
-    // mbarrier would read its parity wrong.
-    constexpr int kStep = kND == 2 ? 2 : 1;
-    const bool active = kND == 2 || group == 0;
-    for (int kk = group; active; kk += kStep) {
-      const int xd = kk % kND, xe = group, jr = kk / kStep;   // jr: this group's page count
-      if (!mbar_wait(&acc_full[xd], (kk / kND) & 1)) { report(a.flags, 5, 6); break; }
+    const int q = warp - kIdxEpiWarp0;             // TMEM lane quarter
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    // rows of the tile this warp reads: M = 64: 16q..16q+15; M = 128: 32q..32q+31
+    constexpr int kRows = M == 64 ? 16 : 32;
+    for (int k = 0;; ++k) {
+      const int x = k & 1;
+      if (!mbar_wait(&d_full[x], (k >> 1) & 1)) { report(a.flags, 5, 6); break; }
       tc_fence_after();
-      const int* pf = pinfo + 8 * (kk & 3);
-      const int pb = pf[0], pi = pf[1], pkind = pf[2], pL = pf[3];
-      if (pkind == kPageEnd) {
-        if (lane == 0) mbar_arrive(&acc_empty[xd]);
-        break;
-      }
-      const int qbase = pf[4] * NQ;                // first index query of this page's tile
-      const int t_first = qbase >> 2;
-      if (pkind == kPageLoad) {
-        const int pos0 = pL - a.T;
-        const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + t_first;
-        // 16x256b loads: thread (g, t) holds keys g, g+8 (first load) and
-        // g+16, g+24 (second) of this quarter's 32, columns 8c+2t and 8c+2t+1.
-        constexpr int kR = kChunk / 8;                       // column groups per load
+      const int* pf = pinfo + 8 * (k % kInfoRing);
+      const int pb = pf[0], pi = pf[1], pkind = pf[2], py = pf[3], pL = pf[4];
+      if (pkind == kPageEnd) break;
+      const int qbase = py * M + kRows * q;          // first index query of this warp's rows
+      const bool active = qbase < nq_all;            // warp-uniform
+      const int pos0 = pL - a.T;
+      if (active && pkind == kPageLoad) {
+        const uint32_t dcol = (uint32_t)(x * kBlock);
+        if constexpr (M == 64) {
+          // 16x256b: thread (g, t) holds rows g and g+8 of the quarter, columns 8c+2t, 8c+2t+1
+          const int g = lane >> 2, t = lane & 3;
+          float m0 = -INFINITY, m1 = -INFINITY;
+          const int qa0 = qbase + g, qa1 = qa0 + 8;
+          const int lim0 = pos0 + (qa0 >> 2), lim1 = pos0 + (qa1 >> 2);   // last visible key
+          const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + (qbase >> 2);
 #pragma unroll 1
-        for (int c0 = 0; c0 < NQ; c0 += kChunk) {
-          float va[4 * kR], vb[4 * kR];
-          tmem_ld_16x256b<kR>(lane_base + kACols + xd * NQ + c0, va);
-          tmem_ld_16x256b<kR>(lane_base + (16u << 16) + kACols + xd * NQ + c0, vb);
-          tmem_wait_ld();
-          const int kb = pi * kBlock + 32 * quarter + g;     // key of va[.][0..1]
-          if (need_mask) {   // keys after a query's position do not count
+          for (int h = 0; h < 2; ++h) {                // columns 64h .. 64h+63
+            float v[32];
+            tmem_ld_16x256b_x8(lane_base + dcol + 64 * h, v);
+            tmem_wait_ld();
+            if (need_mask) {
 #pragma unroll
-            for (int i = 0; i < 4 * kR; ++i) {
-              const int col = c0 + 8 * (i >> 2) + 2 * tq + (i & 1);
-              const int lim = pos0 + ((qbase + col) >> 2);
-              const int dk = (i & 2) ? 8 : 0;
-              if (kb + dk > lim) va[i] = -INFINITY;
-              if (kb + 16 + dk > lim) vb[i] = -INFINITY;
-            }
-          }
-          if (a.token_scores != nullptr) {
-#pragma unroll
-            for (int i = 0; i < 4 * kR; ++i) {
-              const int col = c0 + 8 * (i >> 2) + 2 * tq + (i & 1);
-              const int qg = qbase + col, t = qg >> 2;
-              const int dk = (i & 2) ? 8 : 0;
-              if (t < a.T) {
-                float* rowp = a.token_scores + (((long long)pb * a.T + t) * kG + (qg & 3)) * ctx;
-                rowp[kb + dk] = va[i] * a.score_scale;
-                rowp[kb + 16 + dk] = vb[i] * a.score_scale;
+              for (int i = 0; i < 32; ++i) {
+                const int key = pi * kBlock + 64 * h + 8 * (i >> 2) + 2 * t + (i & 1);
+                if (key > ((i & 2) ? lim1 : lim0)) v[i] = -INFINITY;
               }
             }
+            if (a.token_scores != nullptr) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                const int qa = (i & 2) ? qa1 : qa0, tt = qa >> 2;
+                if (tt < a.T) {
+                  float* rowp = a.token_scores + (((long long)pb * a.T + tt) * kG + (qa & 3)) * ctx;
+                  const int col = pi * kBlock + 64 * h + 8 * (i >> 2) + 2 * t;
+                  rowp[col] = v[i] * a.score_scale;
+                  rowp[col + 1] = v[i + 1] * a.score_scale;
+                }
+              }
+            }
+            float r0[16], r1[16];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              r0[2 * c] = v[4 * c]; r0[2 * c + 1] = v[4 * c + 1];
+              r1[2 * c] = v[4 * c + 2]; r1[2 * c + 1] = v[4 * c + 3];
+            }
+            m0 = fmaxf(m0, max_of<16>(r0));
+            m1 = fmaxf(m1, max_of<16>(r1));
           }
-          // max over this thread's 4 keys, then over the 8 lane groups g
-          float m[2 * kR];
-#pragma unroll
-          for (int c = 0; c < kR; ++c) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-              m[2 * c + e] = fmaxf(fmax3(va[4 * c + e], va[4 * c + 2 + e], vb[4 * c + e]),
-                                   vb[4 * c + 2 + e]);
+          m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+          m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+          if (t < 2) {
+            const int qa = t == 0 ? qa0 : qa1, tt = qa >> 2;
+            if (tt < a.T)
+              a.block_scores[(((long long)pb * a.T + tt) * kG + (qa & 3)) * a.max_pages + pi] =
+                  (t == 0 ? m0 : m1) * a.score_scale;
           }
+        } else {
+          // 32x32b: thread = row (index query qbase + lane), all 128 columns
+          const int qa = qbase + lane, tt = qa >> 2;
+          const int lim = pos0 + tt;
+          const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + (qbase >> 2);
+          float m = -INFINITY;
+#pragma unroll 1
+          for (int h = 0; h < 4; ++h) {
+            float v[32];
+            tmem_ld_32x32b_x32(lane_base + dcol + 32 * h, v);
+            tmem_wait_ld();
+            if (need_mask) {
 #pragma unroll
-          for (int off = 4; off < 32; off <<= 1) {
+              for (int i = 0; i < 32; ++i)
+                if (pi * kBlock + 32 * h + i > lim) v[i] = -INFINITY;
+            }
+            if (a.token_scores != nullptr && tt < a.T) {
+              float* rowp = a.token_scores + (((long long)pb * a.T + tt) * kG + (qa & 3)) * ctx +
+                            pi * kBlock + 32 * h;
 #pragma unroll
-            for (int i = 0; i < 2 * kR; ++i) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], off));
+              for (int i = 0; i < 32; ++i) rowp[i] = v[i] * a.score_scale;
+            }
+            m = fmaxf(m, max_of<32>(v));
           }
-          if (g == 0) {
-            float* dst = red + (xe * kIdxEpilogue + quarter) * NQ + c0 + 2 * tq;
-#pragma unroll
-            for (int c = 0; c < kR; ++c) { dst[8 * c] = m[2 * c]; dst[8 * c + 1] = m[2 * c + 1]; }
-          }
+          if (tt < a.T)
+            a.block_scores[(((long long)pb * a.T + tt) * kG + (qa & 3)) * a.max_pages + pi] =
+                m * a.score_scale;
+        }
+      } else if (active && pkind == kPageMasked) {
+        // no key of the block is visible to any query of the tile
+        for (int r = lane; r < kRows; r += 32) {
+          const int qa = qbase + r, tt = qa >> 2;
+          if (tt >= a.T) continue;
+          const long long row = ((long long)pb * a.T + tt) * kG + (qa & 3);
+          a.block_scores[row * a.max_pages + pi] = -INFINITY;
+          if (a.token_scores != nullptr)
+            for (int j = 0; j < kBlock; ++j) a.token_scores[row * ctx + pi * kBlock + j] = -INFINITY;
         }
       }
       tc_fence_before();
       __syncwarp();
-      // rendezvous of the four quarters (bounded mbarrier wait), then each
-      // warp combines a quarter of the columns
-      if (lane == 0) mbar_arrive(&red_full[xe]);
-      if (!mbar_wait(&red_full[xe], jr & 1)) { report(a.flags, 5, 7); break; }
-      if (pkind != kPageBad) {
-        constexpr int kPer = NQ / kIdxEpilogue;
-        for (int j = lane; j < kPer; j += 32) {
-          const int col = quarter * kPer + j;
-          const int qg = qbase + col, t = qg >> 2;
-          if (t >= a.T) continue;
-          float m = -INFINITY;
-          if (pkind == kPageLoad) {
-#pragma unroll
-            for (int w = 0; w < kIdxEpilogue; ++w) m = fmaxf(m, red[(xe * kIdxEpilogue + w) * NQ + col]);
-          }
-          a.block_scores[(((long long)pb * a.T + t) * kG + (qg & 3)) * a.max_pages + pi] =
-              m * a.score_scale;
-          if (pkind == kPageMasked && a.token_scores != nullptr) {
-            float* rowp = a.token_scores + (((long long)pb * a.T + t) * kG + (qg & 3)) * ctx;
-            for (int r = 0; r < kBlock; ++r) rowp[pi * kBlock + r] = -INFINITY;
-          }
-        }
-      }
-      __syncwarp();
-      // The accumulator (and, through the MMA order, this page's partial
-      // maxima and info slot) is released only after the combine: the MMA
-      // that refills it waits for all four arrivals, so red[xe] is not
-      // rewritten (page kk+2) before every warp has read it.
-      if (lane == 0) mbar_arrive(&acc_empty[xd]);
+      if (lane == 0) mbar_arrive(&d_empty[x]);
     }
   } else {
     // ------------------------------------------------------------ decoders
-    const int quarter = warp;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);   // this warp's TMEM lanes
-    const int row = 32 * quarter + lane;                                  // key row of this thread
-    int cur_b = -1, cur_y = -1, qsel = 1, L = 0, ends = 0;
-    for (int k = 0; ends < 2; ++k) {
-      const int s = k % kIdxRawStages, ab = k & 1;
-      if (!mbar_wait(&raw_full[s], (k / kIdxRawStages) & 1)) { report(a.flags, 5, 5); break; }
-      if (k >= 2 && !mbar_wait(kND == 2 ? &acc_full[ab] : &a_empty[ab], ((k >> 1) - 1) & 1)) {
+    const int row = 32 * warp + lane;                                     // key row of this thread
+    int cur_b = -1, cur_y = -1, qsel = 1;
+    for (int k = 0;; ++k) {
+      const int s = k % S;
+      if (!mbar_wait(&raw_full[s], (k / S) & 1)) { report(a.flags, 5, 5); break; }
+      // page k-2 consumed by the MMA: its B buffer (k % 2) and the page-ready
+      // barrier k % 2 are free, and every MMA of pages <= k-2 has completed
+      if (k >= 2 && !mbar_wait(&b_empty[k & 1], ((k >> 1) - 1) & 1)) {
         report(a.flags, 5, 4);
         break;
       }
-      tc_fence_after();
-      const int nb = meta[4 * s + 0], ni = meta[4 * s + 1], nkind = meta[4 * s + 2];
-      const int ny = meta[4 * s + 3];
-      ends += (nkind == kPageEnd);
+      const int* m = meta + 8 * s;
+      const int nb = m[0], ni = m[1], nkind = m[2], ny = m[3], nL = m[4];
       if (nkind != kPageEnd && (nb != cur_b || ny != cur_y)) {
         cur_b = nb;
         cur_y = ny;
-        L = a.seq_lens[nb];
         qsel ^= 1;
-        // B operand: the index queries of tile ny of sequence nb, swizzled
-        // (its previous user, an MMA of page k-2 or earlier, has completed:
-        // the wait above).
-        uint8_t* qb = qbuf + qsel * NQ * kQRow;
-        const int qbase = ny * NQ;
-        for (int idx = warp * 32 + lane; idx < NQ * 8; idx += kIdxDecoders * 32) {
-          const int nrow = idx / 8, c = idx % 8;
-          const int qg = qbase + nrow, t = qg >> 2;
+        // A operand: the index queries of tile ny of sequence nb, K-major
+        // with the 128-byte swizzle, zero rows past the sequence's queries.
+        // Its previous user (a tile that ended two or more pages ago) has
+        // completed: the MMA of page k-2 has (the wait above).
+        uint8_t* qb = qbuf + qsel * M * C::kRow;
+        const int qbase = ny * M;
+        for (int idx = row; idx < M * 8; idx += kIdxDecWarps * 32) {
+          const int nrow = idx >> 3, c = idx & 7;
+          const int qg = qbase + nrow;
           uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (t < a.T)
-            v = *reinterpret_cast<const uint4*>(
-                a.qi + (((long long)nb * a.T + t) * kG + (qg & 3)) * kDim + 16 * c);
+          if (qg < nq_all)
+            v = *reinterpret_cast<const uint4*>(a.qi + ((long long)nb * nq_all + qg) * kDim + 16 * c);
           if constexpr (F16) {
             // dims 16c..16c+15 -> FP16 chunks 2c, 2c+1 of 8 dims: K-half c / 4,
             // chunk positions (2c % 8, 2c % 8 + 1) ^ (row % 8) in its 128-byte row
@@ -509,7 +473,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
                                         e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
             const uint4 hi = make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
                                         e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
-            uint8_t* rowp = qb + (c >> 2) * NQ * 128 + nrow * 128;
+            uint8_t* rowp = qb + (c >> 2) * M * 128 + nrow * 128;
             const int j = (2 * c) & 7;
             sts128(rowp + ((j ^ (nrow & 7)) << 4), lo);
             sts128(rowp + (((j + 1) ^ (nrow & 7)) << 4), hi);
@@ -517,26 +481,18 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
             sts128(qb + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
           }
         }
-        fence_async_smem();
       }
-      if (nkind == kPageLoad) {
-        const uint8_t* rs = raw + s * Ly.raw_stride;
-        const uint32_t abase = lane_base + ab * kABufCols;
-        if constexpr (FP8IDX) {
-          // 128-byte rows loaded with the 128-byte swizzle: chunk c of row r
-          // sits at chunk position c ^ (r % 8).
-#pragma unroll
-          for (int c2 = 0; c2 < 4; ++c2) {
-            const uint4 x0 = lds128(rs + row * 128 + (((2 * c2) ^ (row & 7)) << 4));
-            const uint4 x1 = lds128(rs + row * 128 + (((2 * c2 + 1) ^ (row & 7)) << 4));
-            const uint32_t w8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            tmem_st8(abase + 8 * c2, w8);
-          }
-        } else if constexpr (F16) {
-          // 64-byte code rows (64-byte swizzle, as below); chunk c = elements
-          // 32c..32c+31 under scale bytes 2c and 2c+1 -> FP16 columns 16c..16c+15
-          const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
-          const int sw = (row >> 1) & 3;
+      if (!FP8 && nkind == kPageLoad) {
+        const uint8_t* rs = raw + s * C::kRawStride;
+        uint8_t* bb = bbuf + (k & 1) * C::kBBytes;
+        // 64-byte code rows loaded with the 64-byte swizzle: chunk c of row r
+        // sits at chunk position c ^ ((r / 2) % 4); chunk c = elements
+        // 32c..32c+31 under scale bytes 2c and 2c+1
+        const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
+        const int sw = (row >> 1) & 3;
+        if constexpr (F16) {
+          // FP16 key row: 256 bytes as two 128-byte K-halves (rows 128 apart),
+          // each with the 128-byte swizzle; chunk c -> 16-byte chunks 4c..4c+3
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
@@ -548,62 +504,45 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
             e2m1x8_to_f16x2(w4.z, o + 8);
             e2m1x8_to_f16x2(w4.w, o + 12);
 #pragma unroll
-            for (int m = 0; m < 16; ++m) o[m] = hmul2(o[m], m < 8 ? s_lo : s_hi);
-            tmem_st16(abase + 16 * c, o);
+            for (int mm = 0; mm < 16; ++mm) o[mm] = hmul2(o[mm], mm < 8 ? s_lo : s_hi);
+            uint8_t* rowp = bb + (c >> 1) * kBlock * 128 + row * 128;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int ch = 4 * (c & 1) + j;
+              sts128(rowp + ((ch ^ (row & 7)) << 4),
+                     make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]));
+            }
           }
         } else {
-          // 64-byte code rows loaded with the 64-byte swizzle: chunk c of
-          // row r sits at chunk position c ^ ((r / 2) % 4).
-          const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
-          const int sw = (row >> 1) & 3;
-          // warp-uniform branch: tcgen05.st is a .sync.aligned warp instruction
-          if (__all_sync(0xffffffffu, ((sc.x | sc.y) & 0x80808080u) == 0u)) {
+          // E4M3 key row: 128 bytes with the 128-byte swizzle; code chunk c ->
+          // row chunks 2c, 2c+1
+          uint8_t* rowp = bb + row * 128;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-              const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));   // scales 2c, 2c+1
-              const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
-              uint32_t pw[8], nw[8];
-              dq8_split_pos(w4.x, r0, pw[0], pw[1], nw[0], nw[1]);
-              dq8_split_pos(w4.y, r0, pw[2], pw[3], nw[2], nw[3]);
-              dq8_split_pos(w4.z, r1, pw[4], pw[5], nw[4], nw[5]);
-              dq8_split_pos(w4.w, r1, pw[6], pw[7], nw[6], nw[7]);
-              tmem_st8(abase + 8 * c, pw);
-              tmem_st8(abase + 32 + 8 * c, nw);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-              const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));
-              const uint32_t s0 = sb & 0xFFu, s1 = (sb >> 8) & 0xFFu;
-              const uint2 r0 = lut[s0 & 0x7Fu], r1 = lut[s1 & 0x7Fu];
-              const uint32_t f0 = (s0 & 0x80u) ? 0x88888888u : 0u;
-              const uint32_t f1 = (s1 & 0x80u) ? 0x88888888u : 0u;
-              uint32_t pw[8], nw[8];
-              dq8_split(w4.x, r0, f0, pw[0], pw[1], nw[0], nw[1]);
-              dq8_split(w4.y, r0, f0, pw[2], pw[3], nw[2], nw[3]);
-              dq8_split(w4.z, r1, f1, pw[4], pw[5], nw[4], nw[5]);
-              dq8_split(w4.w, r1, f1, pw[6], pw[7], nw[6], nw[7]);
-              tmem_st8(abase + 8 * c, pw);
-              tmem_st8(abase + 32 + 8 * c, nw);
-            }
+          for (int c = 0; c < 4; ++c) {
+            const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
+            const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));   // scales 2c, 2c+1
+            const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+            uint32_t o[8];
+            dq8(w4.x, r0, o[0], o[1]);
+            dq8(w4.y, r0, o[2], o[3]);
+            dq8(w4.z, r1, o[4], o[5]);
+            dq8(w4.w, r1, o[6], o[7]);
+            sts128(rowp + (((2 * c) ^ (row & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+            sts128(rowp + (((2 * c + 1) ^ (row & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
           }
         }
-        tmem_wait_st();
       }
-      tc_fence_before();
+      fence_async_smem();   // generic-proxy writes (queries, keys) -> the MMA
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&raw_empty[s]);
         if (warp == 0) {
-          tinfo[2 * ab] = nkind == kPageEnd ? 2 : (nkind != kPageLoad);
-          tinfo[2 * ab + 1] = qsel;
-          int* pf = pinfo + 8 * (k & 3);
-          pf[0] = nb; pf[1] = ni; pf[2] = nkind; pf[3] = L; pf[4] = ny;
+          int* pf = pinfo + 8 * (k % kInfoRing);
+          pf[0] = nb; pf[1] = ni; pf[2] = nkind; pf[3] = ny; pf[4] = nL; pf[5] = qsel;
         }
-        mbar_arrive(&a_full[ab]);
+        if (!FP8) mbar_arrive(&raw_empty[s]);
+        mbar_arrive(&b_full[k & 1]);
       }
+      if (nkind == kPageEnd) break;
     }
   }
 
@@ -611,41 +550,26 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kIdxMmaWarp) tmem_dealloc(tmem, kCols);
+  if (warp == kIdxMmaWarp) tmem_dealloc(tmem, kIdxTmemCols);
 }
 
-template <int NQ, int MODE>
-static cudaError_t launch_nq(const IdxArgs& a, int num_sms, cudaStream_t st) {
-  auto kern = indexer_kernel<NQ, MODE>;
-  const size_t smem = (size_t)idx_layout(NQ, MODE, a.B).total;
-  static size_t configured = 0;
-  if (configured < smem) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = smem;
-  }
-  const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), kIdxThreads, smem,
-                                 pow2_at_least(kACols + (NQ <= 64 ? 2 : 1) * NQ));
-  const int gx = num_sms * per_sm;              // persistent: items are claimed in the kernel
-  kern<<<gx, kIdxThreads, smem, st>>>(a);
+template <int MODE, int M>
+static cudaError_t launch_mode(const IdxArgs& a, cudaStream_t st) {
+  auto kern = indexer_kernel<MODE, M>;
+  const size_t smem = (size_t)idx_layout<MODE, M>(a.B).total;
+  int grid = 0;                                 // persistent: items are claimed in the kernel
+  cudaError_t e = persistent_grid(reinterpret_cast<const void*>(kern), kIdxThreads, smem,
+                                  kIdxTmemCols, &grid);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kIdxThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_indexer(const IdxArgs& a, int mode, int num_sms, cudaStream_t st) {
-  const int nq = idx_nq(a.T);
-#define MSA_IDX_CASE(NQV)                                                     \
-  if (nq == NQV) {                                                            \
-    if (mode == kIdxFp8) return launch_nq<NQV, kIdxFp8>(a, num_sms, st);      \
-    if (mode == kIdxF16) return launch_nq<NQV, kIdxF16>(a, num_sms, st);      \
-    return launch_nq<NQV, kIdxNvfp4>(a, num_sms, st);                         \
-  }
-  MSA_IDX_CASE(16)
-  MSA_IDX_CASE(32)
-  MSA_IDX_CASE(64)
-  MSA_IDX_CASE(128)
-  MSA_IDX_CASE(256)
-#undef MSA_IDX_CASE
-  return cudaErrorInvalidValue;
+cudaError_t launch_indexer(const IdxArgs& a, int mode, cudaStream_t st) {
+  const bool m64 = idx_tile_queries(a.T) == 64;
+  if (mode == kIdxFp8) return m64 ? launch_mode<kIdxFp8, 64>(a, st) : launch_mode<kIdxFp8, 128>(a, st);
+  if (mode == kIdxF16) return m64 ? launch_mode<kIdxF16, 64>(a, st) : launch_mode<kIdxF16, 128>(a, st);
+  return m64 ? launch_mode<kIdxNvfp4, 64>(a, st) : launch_mode<kIdxNvfp4, 128>(a, st);
 }
 
 }  // namespace msa

@@ -11,11 +11,10 @@
 
 namespace msa {
 
-constexpr int kIdxThreads = 14 * 32;    // 4 decoders, 8 epilogue warps, producer, MMA warp
+constexpr int kIdxThreads = 10 * 32;    // 4 decoders, 4 epilogue warps, producer, MMA warp
 // Indexer arithmetic: NVFP4 keys re-rounded to E4M3 (FP8 MMA), E4M3 keys, or
 // NVFP4 keys decoded exactly to FP16 (FP16 MMA).
 enum : int { kIdxNvfp4 = 0, kIdxFp8 = 1, kIdxF16 = 2 };
-constexpr int kIdxRawStages = 6;         // raw index-key pages in flight per CTA
 
 struct IdxArgs {
   CUtensorMap tmap_idx;        // rows of idx_data: 64-byte rows (64B swizzle) or 128 (128B swizzle)
@@ -34,13 +33,16 @@ struct IdxArgs {
 };
 
 size_t indexer_smem_bytes(int mode, int batch, int T);
-int idx_nq(int T);
-cudaError_t launch_indexer(const IdxArgs& a, int mode, int num_sms, cudaStream_t st);
+int idx_tile_queries(int T);   // index queries per tile (the MMA's M side): 64 or 128
+cudaError_t launch_indexer(const IdxArgs& a, int mode, cudaStream_t st);
 
-// CTAs of `kernel` resident per SM for `threads` threads and `smem` dynamic
-// shared memory (registers, shared memory, and `tmem_cols` of the 512 TMEM
-// columns each CTA allocates; 0 = none).
-int ctas_per_sm(const void* kernel, int threads, size_t smem, int tmem_cols);
+// Grid of a persistent kernel on the current device: the device's SMs times
+// the CTAs of `kernel` resident per SM for `threads` threads, `smem` bytes of
+// dynamic shared memory and `tmem_cols` of the 512 TMEM columns per CTA
+// (0 = none).  Raises the kernel's dynamic shared-memory limit to `smem` on
+// the current device first (once per device, kernel and size; thread-safe).
+// Any CUDA error is returned, never replaced by a default.
+cudaError_t persistent_grid(const void* kernel, int threads, size_t smem, int tmem_cols, int* grid);
 
 // Encode a tensor map over `rows` rows of `row_bytes` (64 or 128) bytes with
 // 128-row boxes and the matching shared-memory swizzle.  False on failure.
@@ -79,7 +81,7 @@ struct AttnArgs {
 
 size_t attn_smem_bytes();
 int attn_splits(long long rows, int num_sms);
-cudaError_t launch_attn(const AttnArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 
 // Quantise the new tokens into the cache (msa_kv_insert).
 struct InsArgs {

@@ -27,7 +27,14 @@
  *     library never allocates, frees or keeps a pointer after returning.
  *   - Every call is asynchronous on `stream` (NULL = legacy default stream).
  *   - Host-side argument checks run before any launch; a failed check returns
- *     an error code and launches nothing.
+ *     an error code and launches nothing.  Besides NULL pointers, alignment,
+ *     sizes and scales, they check that the first and the last byte of every
+ *     buffer (sized from the arguments) is device memory of the current
+ *     device, or managed memory: a pageable or pinned host buffer, another
+ *     device's memory or an address CUDA does not know returns
+ *     MSA_ERR_INVALID_ARG (MSA_ERR_WORKSPACE for the workspace) instead of
+ *     faulting the GPU.  A buffer that ends inside another allocation is not
+ *     detected.
  *   - Device-side checks (page ids, selected block ids, sequence lengths) never
  *     trap: a bad item is skipped and the first error code is recorded in the
  *     workspace; msa_get_last_error() reads it.
@@ -125,11 +132,12 @@ typedef struct {
     int32_t max_pages;          /* row length of page_table; upper bound on blocks */
 } msa_seqs;
 
-/* Bytes of device workspace the calls below need for `seqs` on the current
- * device (error flags, block scores, selection, attention partials).  The
+/* Bytes of device workspace the calls below need for `seqs` (error flags,
+ * block scores, selection, attention partials).  The size depends on `seqs`
+ * alone (not on the device), so it can be computed without a GPU.  The
  * workspace must be zeroed once (msa_workspace_init) before its first use and
  * may be reused by later calls on the same stream.  Returns 0 if seqs is
- * invalid. */
+ * invalid (its pointers are not dereferenced). */
 MSA_API size_t msa_workspace_size(const msa_seqs* seqs);
 
 /* Zero the workspace's error flags (asynchronous on stream). */
@@ -251,7 +259,10 @@ MSA_API msa_status msa_debug_nvfp4_table(uint8_t* out, msa_stream_t stream);
  *     msa_decode), MSA_ERR_INVALID_ARG / MSA_ERR_CUDA as msa_decode.
  *   - The first call on a device looks up the array's device address for
  *     that device (cudaGetSymbolAddress, with the device current); make that
- *     first call before any stream capture on the device.
+ *     first call before any stream capture on the device.  The address is
+ *     kept with the identity of the device's CUDA context; after a
+ *     cudaDeviceReset the next call finds a new context and looks the
+ *     address up again (that call, too, should come before any capture).
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents; each call clears what must start at zero.  Calls that
  *     overlap on the GPU (different streams, or different host threads

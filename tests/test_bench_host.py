@@ -45,10 +45,15 @@ def test_traffic_is_read_only_for_unchanged_sources(tmp_path, monkeypatch):
     assert bench.dram_traffic("probe_kernel", "wl") is None
 
 
-def test_measured_peaks_come_from_the_file():
+def test_measured_peaks_come_from_the_file(tmp_path, monkeypatch):
+    """The HBM peak is the driver-written measurement when the file exists,
+    else the stated fallback, labelled as such."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     peak, src = bench.measured_peaks()
-    d = json.load(open(bench.os.path.join(bench.ROOT, "MEASURED_PEAKS.json")))
-    assert src == "measured" and peak == float(d["hbm_gbs"])
+    assert src == "fallback" and peak == bench.FALLBACK_HBM_GBS
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6540.2}))
+    peak, src = bench.measured_peaks()
+    assert src == "measured" and peak == 6540.2
 
 
 def test_reference_arm_prints_the_contract_line():

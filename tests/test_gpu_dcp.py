@@ -4,8 +4,10 @@ The ranks of a context-parallel group are emulated as consecutive launches of
 msa_indexer_score_part on one GPU (they do not wait on one another).  Each
 part must write exactly its blocks, with the values the full launch writes
 for them (bit for bit), and the element-wise max of the parts must give the
-full launch's block scores and selection.  The exchange between ranks is
-covered on CPU (tests/test_dcp_cpu.py).
+full launch's block scores and selection.  The merged parts and the
+selection made from them are also compared with the float64 oracle, and the
+product orchestration (dcp.select) runs once with a single rank.  The exchange
+between ranks is covered on CPU (tests/test_dcp_cpu.py).
 """
 import numpy as np
 import pytest
@@ -14,6 +16,8 @@ import torch
 import block_sparse_attention_decode_b200 as msa
 from block_sparse_attention_decode_b200 import build as msa_build
 from block_sparse_attention_decode_b200 import dcp, synth
+import oracle
+from tests import parity
 
 pytestmark = pytest.mark.gpu
 
@@ -92,3 +96,63 @@ def test_part_arguments_checked():
         with pytest.raises(msa.MsaError) as e:
             msa.msa_indexer_score_part(cache, seqs, w.qi, w.s_qi, None, bs, part, nparts, ws)
         assert e.value.status == msa.MSA_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------ against the oracle --
+# The parts' merged block scores and the selection made from them, compared
+# with the float64 oracle (not with the GPU's own full launch), at the stated
+# tolerances: scores 1e-3 relative, selection exact up to near-ties
+# ([post, "NVFP4 indexer DCP"]: the selection stays exact).
+ORACLE_CASES = [
+    ("ragged_t1", dict(batch=4, seq_lens=[5000, 300, 2049, 7000], q_tokens=1, paged=True, seed=97), (2, 3, 4)),
+    ("t8", dict(batch=2, seq_lens=[9000, 3000], q_tokens=8, paged=True, seed=98), (2, 3, 4)),
+]
+
+
+def _oracle_block_scores(w):
+    c, _ = parity.host_cache(w)
+    rows = oracle.all_rows(c)
+    _, rbs = oracle.indexer(c, w.qi.cpu().numpy(), w.s_qi, rows, token_scores=False)
+    return c, rows, rbs
+
+
+@pytest.mark.parametrize("name,kw,nparts_list", ORACLE_CASES, ids=[c[0] for c in ORACLE_CASES])
+def test_merged_parts_match_the_oracle(name, kw, nparts_list):
+    w = synth.make_workload(name + "_orc", device="cuda", **kw)
+    c, rows, rbs = _oracle_block_scores(w)
+    ref_sel = oracle.select(c, rows, rbs)
+    nvis = np.array([(int(c.seq_lens[b]) - c.q_tokens + t) // 128 + 1 for b, t in rows])
+    for nparts in nparts_list:
+        merged = None
+        for part in range(nparts):
+            _, bs = _scores(w, part, nparts, fill=float("-inf"))
+            part_t = torch.from_numpy(bs)
+            # the element-wise max the all-reduce of dcp.merge_block_scores performs
+            merged = part_t if merged is None else torch.maximum(merged, part_t)
+        g = merged.numpy().reshape(len(rows), 4, -1)
+        for r, (b, t) in enumerate(rows):
+            nblk = (int(c.seq_lens[b]) + 127) // 128
+            parity.check_scores(g[r, :, :nblk], rbs[r, :, :nblk], "%s nparts %d row %d" % (name, nparts, r))
+        gsel = _select(w, merged.numpy()).reshape(len(rows), 4, 16)
+        parity.check_selection(gsel, ref_sel, rbs, nvis, "%s nparts %d" % (name, nparts))
+
+
+def test_dcp_select_world_one_matches_the_oracle():
+    """The product orchestration (dcp.select: part launch, merge, top-16) run
+    by a single process with no process group (one rank, one part)."""
+    w = synth.make_workload("dcp_select", 3, [6000, 2049, 400], 8, paged=True, seed=99, device="cuda")
+    cache, seqs = msa.cache_of(w), msa.seqs_of(w)
+    ws = msa.alloc_workspace(seqs)
+    bs = torch.empty(w.batch, w.q_tokens, 4, w.max_pages, device="cuda")
+    sel = torch.empty(w.batch, w.q_tokens, 4, 16, dtype=torch.int32, device="cuda")
+    dcp.select(cache, seqs, w.qi, w.s_qi, bs, sel, ws)
+    torch.cuda.synchronize()
+    assert msa.msa_get_last_error(ws)[0] == msa.MSA_OK
+    c, rows, rbs = _oracle_block_scores(w)
+    g = bs.cpu().numpy().reshape(len(rows), 4, -1)
+    for r, (b, t) in enumerate(rows):
+        nblk = (int(c.seq_lens[b]) + 127) // 128
+        parity.check_scores(g[r, :, :nblk], rbs[r, :, :nblk], "dcp.select row %d" % r)
+    nvis = np.array([(int(c.seq_lens[b]) - c.q_tokens + t) // 128 + 1 for b, t in rows])
+    parity.check_selection(sel.cpu().numpy().reshape(len(rows), 4, 16), oracle.select(c, rows, rbs),
+                           rbs, nvis, "dcp.select")
