@@ -75,6 +75,21 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def measured_bf16_tflops():
+    """Dense bf16 tensor throughput (burst) from the generated file, else
+    the pool's earlier measurement; the FP8 figure is twice it (the nominal
+    FP8 / bf16 ratio of the part)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
 def source_sha(files) -> str:
     h = hashlib.sha1()
     for f in files:
@@ -276,6 +291,115 @@ def cpu_baseline(name: str, budget_s: float = 20.0):
                       % (reps, nseq, int(w.seq_lens[0]), T, name, threads)}
 
 
+# --------------------------------------------------------- sub-records --
+def timed(fn, steps, flush, stream):
+    """Median CUDA-event time (ms) of fn over `steps` runs, L2 flushed before
+    each (outside the events), after 3 untimed runs."""
+    import torch
+    for _ in range(3):
+        fn()
+    ts = []
+    for _ in range(steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
+def prefill_record(steps, flush, stream):
+    """Chunked prefill (1 sequence, 65,536 cached + 2,048 new tokens, every
+    new token a query with its own top-16 over its causal prefix): step time,
+    tokens/s and the two contractions' FLOP/s against the FP8 dense peak
+    (2 x the measured bf16 burst)."""
+    import torch
+    import block_sparse_attention_decode_b200 as msa
+    from block_sparse_attention_decode_b200 import synth
+    name = "prefill_67584_t2048"
+    w = synth.make_workload(name, device="cuda", **dict(synth.WORKLOADS[name]))
+    cache, seqs = msa.cache_of(w), msa.seqs_of(w)
+    ws = msa.alloc_workspace(seqs)
+    B, T = w.batch, w.q_tokens
+    out = torch.empty(B, T, 64, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(B, T, 4, 16, dtype=torch.int32, device="cuda")
+    bs = torch.empty(B, T, 4, w.max_pages, device="cuda")
+    step = lambda: msa.msa_decode(cache, seqs, w.qi, w.s_qi, w.q, w.s_q, w.softmax_scale, out, sel, ws, stream)
+    ms = timed(step, steps, flush, stream)
+    per = {
+        "indexer": timed(lambda: msa.msa_indexer_score(cache, seqs, w.qi, w.s_qi, None, bs, ws, stream), steps, flush, stream),
+        "topk": timed(lambda: msa.msa_block_maxpool_topk(bs, False, seqs, sel, ws, stream), steps, flush, stream),
+        "attention": timed(lambda: msa.msa_sparse_attn_decode(cache, seqs, w.q, w.s_q, sel, w.softmax_scale, out, ws, stream),
+                           steps, flush, stream),
+    }
+    st, detail = msa.msa_get_last_error(ws, stream)
+    if st != msa.MSA_OK:
+        raise RuntimeError("device error %d (%d) in the prefill record" % (st, detail))
+    L = int(w.seq_lens[0])
+    pos = torch.arange(L - T, L, dtype=torch.float64)
+    # indexer: every index query (4 per token) against every visible key, 128-dim dot products
+    idx_flop = float(4 * 2 * 128 * (pos + 1).sum())
+    # attention: 16 heads per (token, group), QK and PV over the visible keys of the selection
+    s = sel[0].long().cpu()                                   # [T][4][16]
+    blk_keys = (torch.clamp((pos.view(T, 1, 1) + 1) - s.double() * 128, 0, 128) * (s >= 0))
+    att_flop = float(blk_keys.sum() * 16 * 128 * 2 * 2)
+    bf16, src = measured_bf16_tflops()
+    fp8 = 2 * bf16
+    rec = {"workload": name, "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3), "kernel_ms": per,
+           "fp8_peak_tflops": fp8, "peak_note": "2 x the %s dense bf16 burst (nominal FP8/bf16 ratio)" % src}
+    for k, f in (("indexer", idx_flop), ("attention", att_flop)):
+        tf = f / (per[k] * 1e-3) / 1e12
+        rec[k] = {"gflop": f / 1e9, "tflops": tf, "frac_of_fp8_peak": tf / fp8}
+    del w, cache, out, sel, bs, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
+def shared_prefix_record(steps, flush, stream):
+    """Shared-prefix decode ([post, "AMD GPU support", "NVFP4 MSA kernel"]):
+    64 sequences of 131,072 tokens whose first 65,536 tokens (512 blocks) are
+    the same cached pages, 8 query tokens each.  The grouped step reads and
+    decodes each shared page once per tile of 128 of the group's index
+    queries, the plain step once per sequence; both timed, bytes counting each
+    shared page once."""
+    import torch
+    import block_sparse_attention_decode_b200 as msa
+    from block_sparse_attention_decode_b200 import synth
+    B, L, T, pre = 64, 131072, 8, 512
+    w = synth.make_workload("prefix64k_b64_t8", B, [L] * B, T, paged=True, seed=1006, device="cuda",
+                            prefix_groups=[(B, pre)])
+    cache, seqs = msa.cache_of(w), msa.seqs_of(w)
+    groups = msa.PrefixGroups.of([(B, pre)])
+    ws = msa.alloc_workspace(seqs)
+    out = torch.empty(B, T, 64, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(B, T, 4, 16, dtype=torch.int32, device="cuda")
+    bs = torch.empty(B, T, 4, w.max_pages, device="cuda")
+    ms_g = timed(lambda: msa.msa_decode_grouped(cache, seqs, groups, w.qi, w.s_qi, w.q, w.s_q,
+                                                w.softmax_scale, out, sel, ws, stream), steps, flush, stream)
+    ms_u = timed(lambda: msa.msa_decode(cache, seqs, w.qi, w.s_qi, w.q, w.s_q, w.softmax_scale, out, sel,
+                                        ws, stream), steps, flush, stream)
+    idx_g = timed(lambda: msa.msa_indexer_score_grouped(cache, seqs, groups, w.qi, w.s_qi, None, bs, ws, stream),
+                  steps, flush, stream)
+    idx_u = timed(lambda: msa.msa_indexer_score(cache, seqs, w.qi, w.s_qi, None, bs, ws, stream), steps, flush, stream)
+    st, detail = msa.msa_get_last_error(ws, stream)
+    if st != msa.MSA_OK:
+        raise RuntimeError("device error %d (%d) in the shared-prefix record" % (st, detail))
+    by = algorithmic_bytes(w, sel)
+    idx_unique = w.num_pages * 128 * 72          # every distinct index page once
+    total = by["total"] - by["index_scan"] + idx_unique
+    peak, _ = measured_peaks()
+    rec = {"workload": "prefix64k_b64_t8: 64 x 131,072 tokens, the first 65,536 shared, 8 query tokens",
+           "grouped_ms": ms_g, "plain_ms": ms_u, "indexer_grouped_ms": idx_g, "indexer_plain_ms": idx_u,
+           "queries_per_s": B * T / (ms_g * 1e-3), "algorithmic_bytes": total,
+           "index_bytes_distinct_pages": idx_unique,
+           "achieved_gbs": total / (ms_g * 1e-3) / 1e9, "frac_of_measured": total / (ms_g * 1e-3) / 1e9 / peak}
+    del w, cache, out, sel, bs, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
 # ------------------------------------------------------------- GPU arm ----
 def run_gpu(args, rank, world, local_rank):
     import torch
@@ -475,6 +599,13 @@ def run_gpu(args, rank, world, local_rank):
     h2d = h_qi.numel() + h_q.numel() + h_lens.numel() * 4
     d2h = h_out[0].numel() * 2
 
+    # sub-records on other workloads (not part of the step): chunked prefill
+    # and a batch sharing a cached prefix
+    extra = {}
+    if rank == 0 and not args.no_extra:
+        extra["prefill"] = prefill_record(10, flush, stream)
+        extra["shared_prefix"] = shared_prefix_record(10, flush, stream)
+
     cache_bytes = (w.idx_data.numel() + 2 * (w.k_data.numel() + w.k_scale.numel())
                    + (w.idx_scale.numel() if w.idx_scale is not None else 0))
     l2_note, e2e_l2_note = l2_notes(cache_bytes)
@@ -516,6 +647,7 @@ def run_gpu(args, rank, world, local_rank):
                             "copy streams, overlapping other steps' decodes; " + e2e_l2_note},
             "wall_s_timed_region": t_wall,
         }
+        result.update(extra)
     return result
 
 
@@ -529,6 +661,8 @@ def main():
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the prefill and shared-prefix sub-records")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local_rank = rank_info()

@@ -24,6 +24,7 @@ EXPORTED = [
     "msa_workspace_size", "msa_workspace_init", "msa_indexer_score", "msa_block_maxpool_topk",
     "msa_sparse_attn_decode", "msa_decode", "msa_get_last_error", "msa_debug_nvfp4_table",
     "msa_status_string", "msa_decode_static", "msa_kv_insert", "msa_indexer_score_part",
+    "msa_indexer_score_grouped", "msa_decode_grouped",
 ]
 MAX_PARTS = 64
 STATIC_WORKSPACE_BYTES = 16 << 20
@@ -52,6 +53,13 @@ class msa_seqs(ctypes.Structure):
     ]
 
 
+class msa_prefix_groups(ctypes.Structure):
+    _fields_ = [
+        ("seq_start", ctypes.c_void_p), ("prefix_blocks", ctypes.c_void_p),
+        ("num_groups", ctypes.c_int32),
+    ]
+
+
 _lib = None
 
 
@@ -76,6 +84,12 @@ def load() -> ctypes.CDLL:
                                          sz, vp]
     L.msa_block_maxpool_topk.restype = ctypes.c_int
     L.msa_block_maxpool_topk.argtypes = [vp, i32, P(msa_seqs), vp, vp, sz, vp]
+    L.msa_indexer_score_grouped.restype = ctypes.c_int
+    L.msa_indexer_score_grouped.argtypes = [P(msa_cache), P(msa_seqs), P(msa_prefix_groups), vp, f32,
+                                            vp, vp, vp, sz, vp]
+    L.msa_decode_grouped.restype = ctypes.c_int
+    L.msa_decode_grouped.argtypes = [P(msa_cache), P(msa_seqs), P(msa_prefix_groups), vp, f32, vp,
+                                     f32, f32, vp, vp, vp, sz, vp]
     L.msa_sparse_attn_decode.restype = ctypes.c_int
     L.msa_sparse_attn_decode.argtypes = [P(msa_cache), P(msa_seqs), vp, f32, vp, f32, vp, vp, sz, vp]
     L.msa_decode.restype = ctypes.c_int
@@ -164,6 +178,27 @@ class Seqs:
         return self.c.batch * self.c.q_tokens * KV_HEADS
 
 
+class PrefixGroups:
+    """Groups of consecutive sequences sharing a cached prefix (device int32
+    tensors seq_start [G+1] and prefix_blocks [G]) and their C description."""
+
+    def __init__(self, seq_start, prefix_blocks):
+        self.tensors = (seq_start, prefix_blocks)
+        _device_tensors(self.tensors)
+        self.c = msa_prefix_groups(seq_start=seq_start.data_ptr(),
+                                   prefix_blocks=prefix_blocks.data_ptr(),
+                                   num_groups=int(prefix_blocks.shape[0]))
+
+    @classmethod
+    def of(cls, groups, device="cuda"):
+        """From [(users, prefix_blocks), ...] covering the batch in order."""
+        start = [0]
+        for users, _ in groups:
+            start.append(start[-1] + int(users))
+        return cls(torch.tensor(start, dtype=torch.int32, device=device),
+                   torch.tensor([int(p) for _, p in groups], dtype=torch.int32, device=device))
+
+
 def cache_of(w) -> Cache:
     return Cache(w.idx_data, w.idx_scale, w.k_data, w.k_scale, w.v_data, w.v_scale,
                  w.s_idx, w.s_k, w.s_v, idx_exact=w.idx_exact)
@@ -237,6 +272,25 @@ def msa_decode(cache: Cache, seqs: Seqs, qi, s_qi: float, q, s_q: float, softmax
     _check(load().msa_decode(ctypes.byref(cache.c), ctypes.byref(seqs.c), _ptr(qi), s_qi, _ptr(q),
                              s_q, softmax_scale, _ptr(out), _ptr(sel_out), _ptr(ws), _nbytes(ws),
                              _stream(stream)), "msa_decode")
+
+
+def msa_indexer_score_grouped(cache: Cache, seqs: Seqs, groups: PrefixGroups, qi, s_qi: float,
+                              token_scores, block_scores, ws, stream=None):
+    """msa_indexer_score with shared-prefix pages decoded once per tile of
+    the group's index queries (same scores)."""
+    _check(load().msa_indexer_score_grouped(ctypes.byref(cache.c), ctypes.byref(seqs.c),
+                                            ctypes.byref(groups.c), _ptr(qi), s_qi,
+                                            _ptr(token_scores), _ptr(block_scores), _ptr(ws),
+                                            _nbytes(ws), _stream(stream)), "msa_indexer_score_grouped")
+
+
+def msa_decode_grouped(cache: Cache, seqs: Seqs, groups: PrefixGroups, qi, s_qi: float, q,
+                       s_q: float, softmax_scale: float, out, sel_out, ws, stream=None):
+    """msa_decode over a batch with shared prefixes (the grouped indexer)."""
+    _check(load().msa_decode_grouped(ctypes.byref(cache.c), ctypes.byref(seqs.c),
+                                     ctypes.byref(groups.c), _ptr(qi), s_qi, _ptr(q), s_q,
+                                     softmax_scale, _ptr(out), _ptr(sel_out), _ptr(ws), _nbytes(ws),
+                                     _stream(stream)), "msa_decode_grouped")
 
 
 def msa_decode_static(cache: Cache, seqs: Seqs, qi, s_qi: float, q, s_q: float,

@@ -133,6 +133,21 @@ msa_status check_seqs_mem(const msa_seqs* s) {
   return check_buf(s->page_table, (size_t)s->batch * s->max_pages * 4);
 }
 
+// Prefix groups: present, 1 .. batch groups, and a page table to share pages.
+msa_status check_groups(const msa_prefix_groups* g, const msa_seqs* s) {
+  if (!g || !g->seq_start || !g->prefix_blocks) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(g->seq_start) || !aligned16(g->prefix_blocks)) return MSA_ERR_INVALID_ARG;
+  if (g->num_groups < 1 || g->num_groups > s->batch) return MSA_ERR_INVALID_ARG;
+  if (!s->page_table) return MSA_ERR_INVALID_ARG;
+  return MSA_OK;
+}
+
+msa_status check_groups_mem(const msa_prefix_groups* g) {
+  msa_status st = check_buf(g->seq_start, ((size_t)g->num_groups + 1) * 4);
+  if (st != MSA_OK) return st;
+  return check_buf(g->prefix_blocks, (size_t)g->num_groups * 4);
+}
+
 // Rows (sequence, token) of the step and the per-row byte counts of the
 // query, output and selection buffers.
 size_t n_tok(const msa_seqs* s) { return (size_t)s->batch * s->q_tokens; }
@@ -148,8 +163,15 @@ msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_E
 
 msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi, float s_qi,
                        float* token_scores, float* block_scores, void* ws, const Layout& L,
-                       cudaStream_t st, int part = 0, int nparts = 1) {
+                       cudaStream_t st, int part = 0, int nparts = 1,
+                       const msa_prefix_groups* groups = nullptr, int shared = 0) {
   IdxArgs a{};
+  if (groups != nullptr) {
+    a.grp_start = groups->seq_start;
+    a.grp_prefix = groups->prefix_blocks;
+    a.ngroups = groups->num_groups;
+    a.shared = shared;
+  }
   const bool fp8 = c->idx_dtype == MSA_IDX_FP8;
   if (!encode_row_tmap(&a.tmap_idx, c->idx_data, (uint64_t)c->num_pages * MSA_BLOCK_TOKENS,
                        fp8 ? MSA_HEAD_DIM : MSA_HEAD_DIM / 2))
@@ -445,6 +467,65 @@ msa_status msa_decode(const msa_cache* cache, const msa_seqs* seqs, const uint8_
   float* bs = at<float>(ws, L.bscores);
   int32_t* sel = sel_out ? sel_out : at<int32_t>(ws, L.sel);
   if ((st = run_indexer(cache, seqs, qi, s_qi, nullptr, bs, ws, L, s)) != MSA_OK) return st;
+  st = cuda_status(launch_topk(bs, seqs->seq_lens, seqs->batch, seqs->q_tokens, seqs->max_pages,
+                               sel, at<Flags>(ws, L.flags), s));
+  if (st != MSA_OK) return st;
+  return run_attn(cache, seqs, q, s_q, sel, softmax_scale, out, ws, L, s);
+}
+
+msa_status msa_indexer_score_grouped(const msa_cache* cache, const msa_seqs* seqs,
+                                     const msa_prefix_groups* groups, const uint8_t* qi, float s_qi,
+                                     float* token_scores, float* block_scores, void* ws,
+                                     size_t ws_bytes, msa_stream_t stream) {
+  if (!seqs_ok(seqs)) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_cache(cache, true, false);
+  if (st != MSA_OK) return st;
+  if ((st = check_groups(groups, seqs)) != MSA_OK) return st;
+  if (!qi || !aligned16(qi) || !block_scores || !aligned16(block_scores) || !good_scale(s_qi))
+    return MSA_ERR_INVALID_ARG;
+  if (token_scores && !aligned16(token_scores)) return MSA_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  const size_t nt = n_tok(seqs), bs_bytes = nt * MSA_KV_HEADS * seqs->max_pages * 4;
+  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+      (st = check_cache_mem(cache, true, false)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
+      (st = check_groups_mem(groups)) != MSA_OK ||
+      (st = check_buf(qi, nt * kQiBytes)) != MSA_OK || (st = check_buf(block_scores, bs_bytes)) != MSA_OK ||
+      (st = check_buf(token_scores, bs_bytes * MSA_BLOCK_TOKENS)) != MSA_OK)
+    return st;
+  const cudaStream_t s = (cudaStream_t)stream;
+  if ((st = run_indexer(cache, seqs, qi, s_qi, token_scores, block_scores, ws, L, s, 0, 1, groups, 1)) != MSA_OK)
+    return st;
+  return run_indexer(cache, seqs, qi, s_qi, token_scores, block_scores, ws, L, s, 0, 1, groups, 0);
+}
+
+msa_status msa_decode_grouped(const msa_cache* cache, const msa_seqs* seqs,
+                              const msa_prefix_groups* groups, const uint8_t* qi, float s_qi,
+                              const uint8_t* q, float s_q, float softmax_scale, uint16_t* out,
+                              int32_t* sel_out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  if (!seqs_ok(seqs)) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_cache(cache, true, true);
+  if (st != MSA_OK) return st;
+  if ((st = check_groups(groups, seqs)) != MSA_OK) return st;
+  if (!qi || !aligned16(qi) || !q || !aligned16(q) || !out || !aligned16(out))
+    return MSA_ERR_INVALID_ARG;
+  if (sel_out && !aligned16(sel_out)) return MSA_ERR_INVALID_ARG;
+  if (!good_scale(s_qi) || !good_scale(s_q) || !good_scale(softmax_scale))
+    return MSA_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
+  const size_t nt = n_tok(seqs);
+  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+      (st = check_cache_mem(cache, true, true)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
+      (st = check_groups_mem(groups)) != MSA_OK ||
+      (st = check_buf(qi, nt * kQiBytes)) != MSA_OK || (st = check_buf(q, nt * kQBytes)) != MSA_OK ||
+      (st = check_buf(out, nt * kOutBytes)) != MSA_OK || (st = check_buf(sel_out, nt * kSelBytes)) != MSA_OK)
+    return st;
+  const cudaStream_t s = (cudaStream_t)stream;
+  float* bs = at<float>(ws, L.bscores);
+  int32_t* sel = sel_out ? sel_out : at<int32_t>(ws, L.sel);
+  if ((st = run_indexer(cache, seqs, qi, s_qi, nullptr, bs, ws, L, s, 0, 1, groups, 1)) != MSA_OK) return st;
+  if ((st = run_indexer(cache, seqs, qi, s_qi, nullptr, bs, ws, L, s, 0, 1, groups, 0)) != MSA_OK) return st;
   st = cuda_status(launch_topk(bs, seqs->seq_lens, seqs->batch, seqs->q_tokens, seqs->max_pages,
                                sel, at<Flags>(ws, L.flags), s));
   if (st != MSA_OK) return st;

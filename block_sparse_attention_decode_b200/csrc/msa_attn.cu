@@ -59,7 +59,7 @@ constexpr int kAttTmemCols = 256;           // A[2] 0..63, S[2] 64..95, O[2] 96.
 constexpr int kColA = 0, kColS = 64, kColO = 96;
 constexpr float kPExp = 4.f;                // P carries a factor 2^4 (E4M3 normal range)
 constexpr float kLazy = 4.f;                // raise m only when a block max exceeds it by 2^4
-constexpr int kVB = 3;                      // V and P buffers (blocks between decode and O update)
+constexpr int kVB = 2;                      // V and P buffers (blocks between decode and O update)
 
 enum : int { kBlkLoad = 0, kBlkEmpty = 1, kBlkEnd = 2 };
 
@@ -83,7 +83,7 @@ __host__ __device__ inline AttLayout att_layout() {
   L.red = off;   off += 2 * 4 * kHpg * 4;                  // block maxima [parity][quarter][16]
   L.bc = off;    off += kAttSoft * 2 * kHh * 4;            // per softmax warp: offsets, alphas
   L.lsum = off;  off += 2 * 4 * kHpg * 4;                  // row sums [parity][quarter][16]
-  L.bars = off;  off += (2 * kAttStages + 17) * 8;
+  L.bars = off;  off += (2 * kAttStages + 19) * 8;
   L.meta = off;  off += kAttStages * kInfo * 4;
   L.binfo = off; off += 4 * kInfo * 4;
   L.tslot = off; off += 16;
@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   uint64_t* o_free = pv_done + kVB;              // [2] softmax -> MMA
   uint64_t* red_full = o_free + 2;               // [1] softmax rendezvous
   uint64_t* misc_bar = red_full + 1;             // [1] softmax rendezvous (item end)
+  uint64_t* s_free = misc_bar + 1;               // [2] softmax -> MMA: S buffer read
   int* meta = reinterpret_cast<int*>(smem + Ly.meta);
   int* binfo = reinterpret_cast<int*>(smem + Ly.binfo);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
@@ -188,6 +189,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     for (int x = 0; x < kVB; ++x) mbar_init(&pv_done[x], 1);
     mbar_init(red_full, kAttSoft);
     mbar_init(misc_bar, kAttSoft);
+    for (int x = 0; x < 2; ++x) mbar_init(&s_free[x], kAttSoft);
     mbar_fence_init();
   }
   if (warp == kAttMmaWarp) {
@@ -202,7 +204,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   if (warp == kAttProducerWarp) {
     // ------------------------------------------------------------ producer
     // The whole warp sets up an item (lane kk checks selected block kk: its
-    // id and page load in parallel); lane 0 issues the copies.
+    // id and page load in parallel); lane 0 issues the copies.  The next
+    // item's selection is read while the current item's blocks are issued.
     int k = 0, ki = 0;            // block slot, item sequence number
     bool ok = true;
     auto emit = [&](int kind, int blk, int first, int last, long long row, int sp, int pos,
@@ -235,18 +238,40 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       ++k;
       return good;
     };
-    long long item = 0;
-    if (lane == 0) item = atomicAdd(&a.work[0], 1);
+    // Item lookup, one lane per selected block of the item's slice: the
+    // block id (from sel) and its page (page table).  Done for the next item
+    // while the current item's blocks are issued, so its global loads do not
+    // stall the copies.
+    struct Look { long long row; int sp, b, t, g, L, pos, blk; long long page; bool valid; };
+    auto lookup = [&](long long it) -> Look {
+      Look r{};
+      r.valid = false;
+      if (it >= items) return r;
+      r.row = it / a.splits;
+      r.sp = (int)(it % a.splits);
+      r.b = (int)(r.row / (kG * a.T));
+      r.t = (int)((r.row / kG) % a.T);
+      r.g = (int)(r.row % kG);
+      r.L = a.seq_lens[r.b];
+      const int k0 = kTopk * r.sp / a.splits, k1 = kTopk * (r.sp + 1) / a.splits;
+      if (lane >= k0 && lane < k1) r.blk = a.sel[r.row * kTopk + lane];
+      return r;
+    };
+    // Items are claimed two ahead: the claim of item n+2 is issued before
+    // item n's blocks, and its value is only read one item later.
+    long long item = 0, nxt = 0, claim = 0;
+    if (lane == 0) {
+      item = atomicAdd(&a.work[0], 1);
+      nxt = atomicAdd(&a.work[0], 1);
+    }
     item = __shfl_sync(0xffffffffu, item, 0);
+    Look cur = lookup(item);
     while (item < items && ok) {
-      long long nxt = 0;
-      if (lane == 0) nxt = atomicAdd(&a.work[0], 1);     // claimed early: latency overlaps
-      const long long row = item / a.splits;
-      const int sp = (int)(item % a.splits);
-      const int b = (int)(row / (kG * a.T));
-      const int t = (int)((row / kG) % a.T);
-      const int g = (int)(row % kG);
-      const int L = a.seq_lens[b];
+      if (lane == 0) claim = atomicAdd(&a.work[0], 1);
+      nxt = __shfl_sync(0xffffffffu, nxt, 0);
+      const Look next = lookup(nxt);
+      const long long row = cur.row;
+      const int sp = cur.sp, b = cur.b, t = cur.t, g = cur.g, L = cur.L;
       const bool len_ok = L >= a.T && L <= a.max_pages * kBlock;
       const int pos = L - a.T + t;
       const int nvis = pos / kBlock + 1;
@@ -257,7 +282,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       long long page = -1;
       bool valid = false;
       if (len_ok && lane >= k0 && lane < k1) {
-        blk = a.sel[row * kTopk + lane];
+        blk = cur.blk;
         if (blk >= nvis) {
           report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, blk);
         } else if (blk >= 0) {
@@ -268,7 +293,6 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         }
       }
       const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-      nxt = __shfl_sync(0xffffffffu, nxt, 0);
       // the query rows of this item (previous user: item ki-2's last S MMA)
       const int qs = ki & 1;
       if (lane == 0) {
@@ -297,7 +321,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         }
       }
       ++ki;
+      cur = next;
       item = nxt;
+      nxt = claim;                                    // lane 0's value, broadcast next time
     }
     if (ok) emit(kBlkEnd, 0, 0, 0, 0, 0, 0, 0, 0);
     // every CTA has made its last claim once all have arrived here
@@ -315,56 +341,72 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       constexpr uint32_t idesc_o = idesc_e4m3_f32(128, 2 * kHpg) | (1u << 15) | (1u << 16);
       const uint64_t qd[2] = {desc_kmajor_sw128(smem_u32(qbuf)),
                               desc_kmajor_sw128(smem_u32(qbuf + kHpg * kDim))};
-      // S for block k; returns its kind (-1 on a timeout)
-      auto issue_s = [&](int k) -> int {
-        const int x = k & 1;
-        if (!mbar_wait(&kv_full[x], (k >> 1) & 1)) { report(a.flags, 5, 22); return -1; }
-        tc_fence_after();
-        const int* bi = binfo + (k & 3) * kInfo;
-        const int kind = bi[0], first = bi[2], last = bi[3], ki = bi[4];
-        if (kind == kBlkLoad) {
-          if (first && !mbar_wait(&q_full[ki & 1], (ki >> 1) & 1)) { report(a.flags, 5, 23); return -1; }
-          const uint32_t d = tmem + kColS + kHpg * x;
-          const uint32_t ta = tmem + kColA + 32 * x;
-          const uint64_t bd = qd[ki & 1];
+      // The S and O streams run independently: S of block ks as soon as its K
+      // is decoded and the softmax has read S of block ks-2 (same buffer);
+      // O of block ko as soon as its P is written.  Both are polled without
+      // blocking, so neither waits behind the other.
+      int ks = 0, ko = 0, s_end = -1;                 // next S, next O, index of the end block
+      uint32_t idle = 0;
+      for (;;) {
+        bool did = false;
+        if (s_end < 0) {
+          const int x = ks & 1;
+          if (mbar_test(&kv_full[x], (ks >> 1) & 1) &&
+              (ks < 2 || mbar_test(&s_free[x], ((ks >> 1) - 1) & 1))) {
+            tc_fence_after();
+            const int* bi = binfo + (ks & 3) * kInfo;
+            const int kind = bi[0], first = bi[2], last = bi[3], ki = bi[4];
+            if (kind != kBlkLoad || !first || mbar_test(&q_full[ki & 1], (ki >> 1) & 1)) {
+              if (kind == kBlkLoad) {
+                tc_fence_after();
+                const uint32_t d = tmem + kColS + kHpg * x;
+                const uint32_t ta = tmem + kColA + 32 * x;
+                const uint64_t bd = qd[ki & 1];
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc_s, kk > 0);
+                for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc_s, kk > 0);
+              }
+              tc_commit(&s_full[x]);
+              if (kind != kBlkEnd && last) tc_commit(&q_empty[ki & 1]);
+              if (kind == kBlkEnd) s_end = ks;
+              ++ks;
+              did = true;
+            }
+          }
         }
-        tc_commit(&s_full[x]);
-        if (kind != kBlkEnd && last) tc_commit(&q_empty[ki & 1]);
-        return kind;
-      };
-      // O update for block k
-      auto issue_o = [&](int k) -> bool {
-        const int x = k & 1;
-        if (!mbar_wait(&p_full[x], (k >> 1) & 1)) { report(a.flags, 5, 24); return false; }
-        tc_fence_after();
-        const int* bi = binfo + (k & 3) * kInfo;
-        const int kind = bi[0], first = bi[2], ki = bi[4];
-        const int ob = ki & 1;
-        if (first && ki >= 2 && !mbar_wait(&o_free[ob], ((ki >> 1) - 1) & 1)) {
-          report(a.flags, 5, 25);
-          return false;
-        }
-        tc_fence_after();
-        if (kind == kBlkLoad) {
-          const uint32_t d = tmem + kColO + 2 * kHpg * ob;
-          const uint32_t va = smem_u32(vbuf + (k % kVB) * kBlock * kDim);
-          const uint32_t pa = smem_u32(pbuf + (k % kVB) * 2 * kBlock * kHpg);
+        if (ko < ks && (s_end < 0 || ko < s_end)) {
+          const int x = ko & 1;
+          if (mbar_test(&p_full[x], (ko >> 1) & 1)) {
+            tc_fence_after();
+            const int* bi = binfo + (ko & 3) * kInfo;
+            const int kind = bi[0], first = bi[2], ki = bi[4];
+            const int ob = ki & 1;
+            if (!(first && ki >= 2) || mbar_test(&o_free[ob], ((ki >> 1) - 1) & 1)) {
+              tc_fence_after();
+              if (kind == kBlkLoad) {
+                const uint32_t d = tmem + kColO + 2 * kHpg * ob;
+                const uint32_t va = smem_u32(vbuf + (ko % kVB) * kBlock * kDim);
+                const uint32_t pa = smem_u32(pbuf + (ko % kVB) * 2 * kBlock * kHpg);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 32 keys per slice
-            tc_mma_ss(d, desc_mn_sw128(va + kk * 32 * kDim, 1024),
-                      desc_mn_plain(pa + kk * 32 * kHpg, 8 * kHpg, kBlock * kHpg), idesc_o,
-                      (first && kk == 0) ? 0u : 1u);
+                for (int kk = 0; kk < 4; ++kk)   // 32 keys per slice
+                  tc_mma_ss(d, desc_mn_sw128(va + kk * 32 * kDim, 1024),
+                            desc_mn_plain(pa + kk * 32 * kHpg, 8 * kHpg, kBlock * kHpg), idesc_o,
+                            (first && kk == 0) ? 0u : 1u);
+              }
+              tc_commit(&pv_done[ko % kVB]);
+              ++ko;
+              did = true;
+            }
+          }
         }
-        tc_commit(&pv_done[k % kVB]);
-        return true;
-      };
-      int kind = issue_s(0);
-      for (int k = 0; kind >= 0 && kind != kBlkEnd; ++k) {
-        const int next = issue_s(k + 1);
-        if (!issue_o(k)) break;
-        kind = next;
+        if (s_end >= 0 && ko >= s_end) break;
+        if (did) {
+          idle = 0;
+        } else if (++idle > kPollLimit) {
+          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 22);
+          break;
+        } else if (idle > 32) {
+          __nanosleep(64);
+        }
       }
     }
   } else if (warp >= kAttSoftWarp0) {
@@ -389,12 +431,17 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       const int sp = bi[6], pos = bi[7];
       if (kind == kBlkEnd) break;
       const int ob = ki & 1;
-      const int vb = k % kVB;                          // P buffer (its last reader: block k-3's O)
+      const int vb = k % kVB;                          // P buffer (its last reader: block k-kVB's O)
       if (k >= kVB && !mbar_wait(&pv_done[vb], ((k / kVB) - 1) & 1)) { report(a.flags, 5, 27); break; }
+      float s[kHh];
       if (kind == kBlkLoad) {
-        float s[kHh];
         tmem_ld8(lane_base + kColS + kHpg * x + h0, s);
         tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[x]);     // S buffer x may be overwritten (block k+2)
+      if (kind == kBlkLoad) {
         if (blk * kBlock + 32 * q + lane > pos) {      // key after the query position
 #pragma unroll
           for (int h = 0; h < kHh; ++h) s[h] = -INFINITY;
@@ -589,7 +636,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     for (int k = 0;; ++k) {
       const int s = k % kAttStages, x = k & 1;
       if (!mbar_wait(&raw_full[s], (k / kAttStages) & 1)) { report(a.flags, 5, 33); break; }
-      // A[x] was last read by block k-2's S; V buffer k % kVB by block k-3's O
+      // A[x] was last read by block k-2's S; V buffer k % kVB by block k-kVB's O
       if (k >= 2 && !mbar_wait(&s_full[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 34); break; }
       if (k >= kVB && !mbar_wait(&pv_done[k % kVB], ((k / kVB) - 1) & 1)) { report(a.flags, 5, 36); break; }
       tc_fence_after();

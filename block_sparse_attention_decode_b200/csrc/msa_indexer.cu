@@ -21,20 +21,24 @@
 // blocks.  Persistent CTAs take items from a counter in the workspace header
 // as they go (ragged batches and CTAs sharing an SM still finish together);
 // the last CTA to finish resets the counter.  Warp roles, a few pages apart:
-//   warp 8 (producer): per page one tiled TMA load of the codes (64-byte
+//   warp 12 (producer): the whole warp looks up the pages of the next work
+//     item (one lane per page: sequence, logical block, page table entry)
+//     while lane 0 issues the current item's pages: per page one tiled TMA
+//     load of the codes (64-byte
 //     swizzle, so that row-per-thread reads are bank-conflict free) and one
 //     bulk copy of the scales into a ring of shared-memory stages (FP8 index
 //     keys: one TMA load with the 128-byte swizzle, which is already the
 //     MMA's B operand);
-//   warps 0-3 (decoders): thread = key row.  NVFP4 rows are decoded to signed
-//     E4M3 (dq8: a table row per scale byte, byte permutes for magnitudes
-//     and signs) and stored as 128-byte rows with the 128-byte swizzle -- the
-//     K-major B operand -- into one of two buffers, so page k+1 is decoded
-//     while page k's MMAs run.  When the query tile changes they also stage
-//     the tile's index queries (the A operand) into one of two buffers;
-//   warp 9 (MMA): one thread issues per page 4 tcgen05.mma of K = 32 (E4M3;
+//   warps 0-7 (decoders): thread = half a key row (warps 0-3 elements 0-63,
+//     warps 4-7 elements 64-127).  NVFP4 is decoded to signed E4M3 (dq8: a
+//     table row per scale byte, byte permutes for magnitudes and signs) and
+//     stored as 128-byte rows with the 128-byte swizzle -- the K-major B
+//     operand -- into one of two buffers, so page k+1 is decoded while page
+//     k's MMAs run.  When the query tile changes they stage the tile's index
+//     queries (the A operand), after the MMAs of the previous tile are done;
+//   warp 13 (MMA): one thread issues per page 4 tcgen05.mma of K = 32 (E4M3;
 //     8 of K = 16 for FP16) into one of two TMEM accumulators;
-//   warps 4-7 (epilogue): warp 4+q reads the accumulator lanes of quarter q,
+//   warps 8-11 (epilogue): warp 8+q reads the accumulator lanes of quarter q,
 //     masks keys after each query's position, takes each query's maximum
 //     over the page's keys and writes the block score.
 // Every wait is a bounded mbarrier wait; on a timeout a thread records
@@ -52,11 +56,11 @@
 
 namespace msa {
 
-constexpr int kIdxDecWarps = 4;             // warps 0-3: one key row per thread
-constexpr int kIdxEpiWarp0 = 4;             // warps 4-7: one per TMEM lane quarter
-constexpr int kIdxProducerWarp = 8;
-constexpr int kIdxMmaWarp = 9;
-static_assert(kIdxThreads == 10 * 32, "warp roles");
+constexpr int kIdxDecWarps = 8;             // warps 0-7: half a key row per thread
+constexpr int kIdxEpiWarp0 = 8;             // warps 8-11: one per TMEM lane quarter
+constexpr int kIdxProducerWarp = 12;
+constexpr int kIdxMmaWarp = 13;
+static_assert(kIdxThreads == 14 * 32, "warp roles");
 
 enum : int { kPageLoad = 0, kPageMasked = 1, kPageBad = 2, kPageEnd = 3 };
 constexpr int kChunkPages = 8;              // pages per work item
@@ -70,7 +74,7 @@ struct IdxCfg {
   static constexpr int kRow = kF16 ? 256 : 128;            // bytes per query / key row
   static constexpr int kRaw = kFp8 ? kBlock * kDim : kPageCodes + kPageScales;
   static constexpr int kRawStride = (kRaw + 1023) / 1024 * 1024;
-  static constexpr int kStages = kFp8 ? 5 : (kF16 ? 3 : 4);   // raw pages in flight
+  static constexpr int kStages = kF16 ? 3 : 6;             // raw pages in flight
   static constexpr int kNB = kFp8 ? 0 : 2;                 // decoded key pages (B operand), page k in k % 2
   static constexpr int kBBytes = kBlock * kRow;
 };
@@ -84,15 +88,15 @@ __host__ __device__ inline IdxLayout idx_layout(int batch) {
   using C = IdxCfg<MODE>;
   IdxLayout L;
   int off = 0;
-  L.qbuf = off;    off += 2 * M * C::kRow;                 // two query tiles (multiples of 1024)
+  L.qbuf = off;    off += M * C::kRow;                     // the query tile (a multiple of 1024)
   L.raw = off;     off += C::kStages * C::kRawStride;
   L.bbuf = off;    off += C::kNB * C::kBBytes;
   L.lut = off;     off += MODE == kIdxNvfp4 ? 256 * 8 : 0;
   L.bars = off;    off += (2 * C::kStages + 8) * 8;
-  L.meta = off;    off += C::kStages * 8 * 4;              // per stage: b, i, kind, tile, L
-  L.pinfo = off;   off += kInfoRing * 8 * 4;               // per page: b, i, kind, tile, L, qsel
+  L.meta = off;    off += C::kStages * 8 * 4;              // per stage: ptrow, i, kind, row0, row1, minpos
+  L.pinfo = off;   off += kInfoRing * 8 * 4;               // per page: the same
   L.tslot = off;   off += 16;
-  L.prefix = off;  off += (batch + 1) * 4;
+  L.prefix = off;  off += (5 * batch + 2) * 4;           // item prefix [E+1], lengths [B], skip [B], groups
   L.scratch = off; off += kIdxThreads * 4;
   L.total = off + 1024;                                   // alignment slack
   return L;
@@ -124,37 +128,124 @@ __device__ __forceinline__ int part_blocks(const IdxArgs& a, int L, int* first) 
   return hi - lo;
 }
 
-// Exclusive prefix over the number of blocks this launch scores in each
-// sequence, in shared memory (prefix[B] = total pages).  Invalid lengths
-// count as 0 blocks and are reported once (by CTA 0).
-__device__ void page_prefix(const IdxArgs& a, int* prefix, int* scratch) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int per = (a.B + nt - 1) / nt;
-  const int lo = tid * per, hi = min(a.B, lo + per);
-  int sum = 0;
-  for (int b = lo; b < hi; ++b) {
-    const int L = a.seq_lens[b];
+// A work entity: logical blocks [lo, hi) of page-table row `ptrow`, scored
+// against the index-query rows [r0, r1) (row = (b*T + t)*4 + g, the row of
+// qi and of the block scores).  Without groups (or with shared = 0) entity b
+// is sequence b: its blocks of this launch's part from its group's prefix
+// on, against its own 4T rows.  With shared = 1 entity g is prefix group g:
+// its shared blocks (the group's first sequence's page-table row) against
+// the rows of all the group's sequences.
+struct Ent { int lo, hi, r0, r1, ptrow; };
+
+// Shared-memory tables (built by build_items): lengths, each sequence's own
+// first block, and the prefix groups clamped to the batch and the page table.
+struct Tabs { const int* lens; const int* skip; const int* gstart; const int* gpre; };
+
+__device__ __forceinline__ Ent entity(const IdxArgs& a, int e, const Tabs& tb) {
+  const int nq = kG * a.T;
+  Ent r;
+  if (a.shared) {
+    const int s0 = tb.gstart[e], s1 = max(tb.gstart[e + 1], s0);
+    r.lo = 0;
+    r.hi = tb.gpre[e];
+    r.r0 = s0 * nq;
+    r.r1 = s1 * nq;
+    r.ptrow = s0;
+  } else {
     int first;
-    const int nb = part_blocks(a, L, &first);
+    const int nb = part_blocks(a, tb.lens[e], &first);
+    r.lo = max(first, tb.skip[e]);
+    r.hi = max(r.lo, first + nb);
+    r.r0 = e * nq;
+    r.r1 = r.r0 + nq;
+    r.ptrow = e;
+  }
+  return r;
+}
+
+// Items (query tile x chunk of kChunkPages blocks) of an entity, M rows per tile.
+template <int M>
+__device__ __forceinline__ int entity_items(const Ent& E) {
+  return ((E.r1 - E.r0 + M - 1) / M) * ((E.hi - E.lo + kChunkPages - 1) / kChunkPages);
+}
+
+// Shared-memory tables built by every CTA at start: the lengths lens[B], the
+// first block of each sequence's own part skip[B] (its group's prefix), and
+// the exclusive prefix over the entities' item counts (prefix[E] = items).
+// Invalid lengths count as 0 blocks and are reported once (by CTA 0); so are
+// prefix groups whose shared blocks are not entirely visible to every query
+// of the group, or whose sequences do not map them to the same pages.
+template <int M>
+__device__ int build_items(const IdxArgs& a, int* prefix, int* lens, int* skip, int* gstart, int* gpre,
+                           int* scratch) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int E = a.shared ? a.ngroups : a.B;
+  for (int b = tid; b < a.B; b += nt) {
+    const int L = a.seq_lens[b];
+    lens[b] = L;
+    skip[b] = 0;
     if ((L < a.T || L > a.max_pages * kBlock) && blockIdx.x == 0)
       report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, L);
-    sum += nb;
   }
+  if (a.grp_start != nullptr) {
+    // clamped so that any group array stays inside the batch and the page
+    // table; inconsistent arrays are reported (by CTA 0)
+    for (int g = tid; g < a.ngroups; g += nt) {
+      const int g0 = a.grp_start[g], g1 = a.grp_start[g + 1], gp = a.grp_prefix[g];
+      const int s0 = min(max(g0, 0), a.B);
+      gstart[g] = s0;
+      gpre[g] = min(max(gp, 0), a.max_pages);
+      if (g == a.ngroups - 1) gstart[g + 1] = min(max(g1, s0), a.B);
+      if (blockIdx.x == 0 && (g0 != s0 || g1 < g0 || g1 > a.B || gp != gpre[g] ||
+                              (g == 0 && g0 != 0) || (g == a.ngroups - 1 && g1 != a.B)))
+        report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, g);
+    }
+  }
+  __syncthreads();
+  if (a.grp_start != nullptr) {
+    for (int g = tid; g < a.ngroups; g += nt) {
+      const int s0 = gstart[g], s1 = max(gstart[g + 1], s0), pre = gpre[g];
+      for (int b = s0; b < s1; ++b) {
+        skip[b] = pre;
+        if (blockIdx.x == 0 && (long long)pre * kBlock > (long long)lens[b] - a.T)
+          report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, b);
+      }
+    }
+    // the shared blocks' page-table entries, each checked by one CTA
+    if (a.shared && a.page_table != nullptr) {
+      for (int g = 0; g < a.ngroups; ++g) {
+        const int s0 = gstart[g], s1 = max(gstart[g + 1], s0), pre = gpre[g];
+        if (s1 - s0 < 2 || pre == 0) continue;
+        const long long n = (long long)(s1 - s0 - 1) * pre;
+        for (long long x = (long long)blockIdx.x * nt + tid; x < n; x += (long long)gridDim.x * nt) {
+          const int b = s0 + 1 + (int)(x / pre), i = (int)(x % pre);
+          if (a.page_table[(long long)b * a.max_pages + i] != a.page_table[(long long)s0 * a.max_pages + i])
+            report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, b);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const Tabs tb{lens, skip, gstart, gpre};
+  const int per = (E + nt - 1) / nt;
+  const int lo = tid * per, hi = min(E, lo + per);
+  int sum = 0;
+  for (int e = lo; e < hi; ++e) sum += entity_items<M>(entity(a, e, tb));
   scratch[tid] = sum;
   __syncthreads();
   if (tid == 0) {
     int run = 0;
     for (int k = 0; k < nt; ++k) { const int v = scratch[k]; scratch[k] = run; run += v; }
-    prefix[a.B] = run;
+    prefix[E] = run;
   }
   __syncthreads();
   int run = scratch[tid];
-  for (int b = lo; b < hi; ++b) {
-    prefix[b] = run;
-    int first;
-    run += part_blocks(a, a.seq_lens[b], &first);
+  for (int e = lo; e < hi; ++e) {
+    prefix[e] = run;
+    run += entity_items<M>(entity(a, e, tb));
   }
   __syncthreads();
+  return E;
 }
 
 __device__ __forceinline__ void sts128(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
@@ -187,7 +278,12 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   int* pinfo = reinterpret_cast<int*>(smem + Ly.pinfo);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
   int* prefix = reinterpret_cast<int*>(smem + Ly.prefix);
+  int* lens = prefix + a.B + 1;
+  int* skip = lens + a.B;
+  int* gstart = skip + a.B;          // [ngroups + 1] (ngroups <= B)
+  int* gpre = gstart + a.B + 1;      // [ngroups]
   int* scratch = reinterpret_cast<int*>(smem + Ly.scratch);
+  const Tabs tabs{lens, skip, gstart, gpre};
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -210,71 +306,111 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     tmem_relinquish();
   }
   tc_fence_before();
-  page_prefix(a, prefix, scratch);   // ends with __syncthreads
+  const int nent = build_items<M>(a, prefix, lens, skip, gstart, gpre, scratch);   // ends with __syncthreads
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  const int total = prefix[a.B];
+  const int items = prefix[nent];
   const int nq_all = kG * a.T;                                // index queries per sequence
-  const int gy = (nq_all + M - 1) / M;                        // query tiles
-  const int nchunks = (total + kChunkPages - 1) / kChunkPages;
-  const int items = nchunks * gy;
   const long long ctx = (long long)a.max_pages * kBlock;
 
   if (warp == kIdxProducerWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int k = 0;                                  // page slot (stage k % S)
-      bool ok = true;
-      auto slot = [&](int kk) -> bool {           // wait until stage kk % S is free
-        return kk < S || mbar_wait(&raw_empty[kk % S], ((kk / S) - 1) & 1);
-      };
-      int first_b = -1, first = 0;                // part_blocks of sequence first_b
-      int item = atomicAdd(&a.work[0], 1);
-      while (item < items && ok) {
-        const int nxt = atomicAdd(&a.work[0], 1);  // claimed early: its latency overlaps this item
-        const int y = item / nchunks, p0 = (item % nchunks) * kChunkPages;
-        const int p1 = min(total, p0 + kChunkPages);
-        const int t_last = (min(nq_all, (y + 1) * M) - 1) >> 2;
-        int b;
-        {  // prefix[b] <= p0 < prefix[b+1]
-          int l = 0, r = a.B;
-          while (r - l > 1) { const int m = (l + r) >> 1; if (prefix[m] <= p0) l = m; else r = m; }
-          b = l;
-        }
-        int li = p0 - prefix[b];                    // index among this part's blocks of b
-        for (int pg = p0; pg < p1; ++pg, ++k, ++li) {
-          if (!slot(k)) { report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1); ok = false; break; }
-          const int s = k % S;
-          while (li >= prefix[b + 1] - prefix[b]) { li -= prefix[b + 1] - prefix[b]; ++b; }
-          const int L = a.seq_lens[b];
-          if (b != first_b) {                       // first block of b's part
-            first_b = b;
-            part_blocks(a, L, &first);
-          }
-          const int i = first + li;                 // logical block
-          int kind = kPageLoad;
-          const long long p = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + i]
-                                           : (long long)b * a.max_pages + i;
-          if (i * kBlock > L - a.T + t_last) {
-            kind = kPageMasked;                     // no key of the block is visible to the tile
-          } else if (p < 0 || p >= a.num_pages) {
-            report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)p);
-            kind = kPageBad;
-          }
-          int* m = meta + 8 * s;
-          m[0] = b; m[1] = i; m[2] = kind; m[3] = y; m[4] = L;
-          uint8_t* dst = raw + s * C::kRawStride;
-          if (kind == kPageLoad) {
-            mbar_expect_tx(&raw_full[s], C::kRaw);
-            tma_load_2d(dst, &a.tmap_idx, 0, (int)(p * kBlock), &raw_full[s]);
-            if (!FP8) bulk_g2s(dst + kPageCodes, a.idx_scale + p * kPageScales, kPageScales, &raw_full[s]);
-          } else {
-            mbar_arrive(&raw_full[s]);
-          }
-        }
-        item = nxt;
+    int k = 0;                                    // page slot (stage k % S)
+    bool ok = true;
+    auto slot = [&](int kk) -> bool {             // wait until stage kk % S is free
+      return kk < S || mbar_wait(&raw_empty[kk % S], ((kk / S) - 1) & 1);
+    };
+    // Item `it` -> entity, query tile (rows [row0, row1)) and chunk; lane
+    // j < np looks up the chunk's block j: logical block, page-table entry,
+    // kind.  The page-table loads are issued here and consumed one item
+    // later, while the previous item's pages are issued.
+    struct Look { int np, ptrow, row0, row1, minpos, i, kind; long long p; };
+    auto lookup = [&](int it) -> Look {
+      Look r{};
+      r.np = 0;
+      if (it >= items) return r;
+      int e = 0;
+      {  // prefix[e] <= it < prefix[e+1]
+        int l = 0, rr = nent;
+        while (rr - l > 1) { const int m = (l + rr) >> 1; if (prefix[m] <= it) l = m; else rr = m; }
+        e = l;
       }
+      const Ent E = entity(a, e, tabs);
+      const int local = it - prefix[e];
+      const int tiles = (E.r1 - E.r0 + M - 1) / M;
+      const int chunks = (E.hi - E.lo + kChunkPages - 1) / kChunkPages;
+      // shared prefix: the tiles of one chunk are consecutive items, so the
+      // CTAs working on them at the same time read the same pages (from L2
+      // after the first); a sequence's own blocks: its chunks are consecutive
+      const int y = a.shared ? local % tiles : local / chunks;
+      const int c = a.shared ? local / tiles : local % chunks;
+      const int i0 = E.lo + c * kChunkPages;
+      r.np = min(E.hi - i0, kChunkPages);
+      r.ptrow = E.ptrow;
+      r.row0 = E.r0 + y * M;
+      r.row1 = min(r.row0 + M, E.r1);
+      // position of the tile's first and last query (a sequence's own rows;
+      // shared prefix blocks are visible to every query of the group)
+      const int L = lens[E.ptrow];
+      r.minpos = a.shared ? 0x7FFFFFFF : L - a.T + ((r.row0 - E.r0) >> 2);
+      const int maxpos = L - a.T + ((r.row1 - 1 - E.r0) >> 2);
+      if (lane < r.np) {
+        r.i = i0 + lane;                          // logical block
+        r.p = a.page_table ? (long long)a.page_table[(long long)E.ptrow * a.max_pages + r.i]
+                           : (long long)E.ptrow * a.max_pages + r.i;
+        r.kind = (!a.shared && r.i * kBlock > maxpos) ? kPageMasked : kPageLoad;
+      }
+      return r;
+    };
+    // Items are claimed two ahead: the claim of item n+2 (an atomic whose
+    // latency is a microsecond or more) is issued before item n's pages, and
+    // its value is only read one item later.
+    int item = 0, nxt = 0, claim = 0;
+    if (lane == 0) {
+      item = atomicAdd(&a.work[0], 1);
+      nxt = atomicAdd(&a.work[0], 1);
+    }
+    item = __shfl_sync(0xffffffffu, item, 0);
+    Look cur = lookup(item);
+    while (item < items && ok) {
+      if (lane == 0) claim = atomicAdd(&a.work[0], 1);
+      nxt = __shfl_sync(0xffffffffu, nxt, 0);
+      const Look next = lookup(nxt);
+      // page ids outside the pool: skipped and reported (kind Bad)
+      if (lane < cur.np && cur.kind == kPageLoad && (cur.p < 0 || cur.p >= a.num_pages)) {
+        report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)cur.p);
+        cur.kind = kPageBad;
+      }
+      for (int j = 0; j < cur.np && ok; ++j, ++k) {
+        const int ij = __shfl_sync(0xffffffffu, cur.i, j);
+        const int kj = __shfl_sync(0xffffffffu, cur.kind, j);
+        const long long pj = __shfl_sync(0xffffffffu, cur.p, j);
+        if (lane == 0) {
+          if (!slot(k)) {
+            report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1);
+            ok = false;
+          } else {
+            const int s = k % S;
+            int* m = meta + 8 * s;
+            m[0] = cur.ptrow; m[1] = ij; m[2] = kj; m[3] = cur.row0; m[4] = cur.row1; m[5] = cur.minpos;
+            uint8_t* dst = raw + s * C::kRawStride;
+            if (kj == kPageLoad) {
+              mbar_expect_tx(&raw_full[s], C::kRaw);
+              tma_load_2d(dst, &a.tmap_idx, 0, (int)(pj * kBlock), &raw_full[s]);
+              if (!FP8) bulk_g2s(dst + kPageCodes, a.idx_scale + pj * kPageScales, kPageScales, &raw_full[s]);
+            } else {
+              mbar_arrive(&raw_full[s]);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+      }
+      cur = next;
+      item = nxt;
+      nxt = claim;                                  // lane 0's value, broadcast next time
+    }
+    if (lane == 0) {
       if (ok) {   // end marker
         if (!slot(k)) {
           report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1);
@@ -300,10 +436,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         if (k >= 2 && !mbar_wait(&d_empty[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 3); break; }
         tc_fence_after();
         const int* pf = pinfo + 8 * (k % kInfoRing);
-        const int kind = pf[2], qsel = pf[5];
+        const int kind = pf[2];
         if (kind == kPageLoad) {
           const uint32_t d = tmem + (uint32_t)(x * kBlock);
-          const uint32_t qa = smem_u32(qbuf + qsel * M * C::kRow);
+          const uint32_t qa = smem_u32(qbuf);
           const uint32_t kb = FP8 ? smem_u32(raw + (k % S) * C::kRawStride)
                                   : smem_u32(bbuf + x * C::kBBytes);
           if constexpr (F16) {
@@ -335,20 +471,24 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       if (!mbar_wait(&d_full[x], (k >> 1) & 1)) { report(a.flags, 5, 6); break; }
       tc_fence_after();
       const int* pf = pinfo + 8 * (k % kInfoRing);
-      const int pb = pf[0], pi = pf[1], pkind = pf[2], py = pf[3], pL = pf[4];
+      const int pi = pf[1], pkind = pf[2], prow0 = pf[3], prow1 = pf[4], pminpos = pf[5];
       if (pkind == kPageEnd) break;
-      const int qbase = py * M + kRows * q;          // first index query of this warp's rows
-      const bool active = qbase < nq_all;            // warp-uniform
-      const int pos0 = pL - a.T;
+      const int rbase = prow0 + kRows * q;           // first query row of this warp's lanes
+      const bool active = rbase < prow1;             // warp-uniform
+      // a key j is visible to query row r when j <= pos(r) = L_b - T + t
+      const bool need_mask = pi * kBlock + kBlock - 1 > pminpos;
+      auto last_key = [&](int r) -> int {
+        const int b = r / nq_all;
+        return lens[b] - a.T + (r - b * nq_all) / kG;
+      };
       if (active && pkind == kPageLoad) {
         const uint32_t dcol = (uint32_t)(x * kBlock);
         if constexpr (M == 64) {
           // 16x256b: thread (g, t) holds rows g and g+8 of the quarter, columns 8c+2t, 8c+2t+1
           const int g = lane >> 2, t = lane & 3;
           float m0 = -INFINITY, m1 = -INFINITY;
-          const int qa0 = qbase + g, qa1 = qa0 + 8;
-          const int lim0 = pos0 + (qa0 >> 2), lim1 = pos0 + (qa1 >> 2);   // last visible key
-          const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + (qbase >> 2);
+          const int qa0 = rbase + g, qa1 = qa0 + 8;
+          const int lim0 = need_mask ? last_key(qa0) : 0, lim1 = need_mask ? last_key(qa1) : 0;
 #pragma unroll 1
           for (int h = 0; h < 2; ++h) {                // columns 64h .. 64h+63
             float v[32];
@@ -364,9 +504,9 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
             if (a.token_scores != nullptr) {
 #pragma unroll
               for (int i = 0; i < 32; i += 2) {
-                const int qa = (i & 2) ? qa1 : qa0, tt = qa >> 2;
-                if (tt < a.T) {
-                  float* rowp = a.token_scores + (((long long)pb * a.T + tt) * kG + (qa & 3)) * ctx;
+                const int qa = (i & 2) ? qa1 : qa0;
+                if (qa < prow1) {
+                  float* rowp = a.token_scores + (long long)qa * ctx;
                   const int col = pi * kBlock + 64 * h + 8 * (i >> 2) + 2 * t;
                   rowp[col] = v[i] * a.score_scale;
                   rowp[col + 1] = v[i + 1] * a.score_scale;
@@ -387,16 +527,13 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
           m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
           if (t < 2) {
-            const int qa = t == 0 ? qa0 : qa1, tt = qa >> 2;
-            if (tt < a.T)
-              a.block_scores[(((long long)pb * a.T + tt) * kG + (qa & 3)) * a.max_pages + pi] =
-                  (t == 0 ? m0 : m1) * a.score_scale;
+            const int qa = t == 0 ? qa0 : qa1;
+            if (qa < prow1) a.block_scores[(long long)qa * a.max_pages + pi] = (t == 0 ? m0 : m1) * a.score_scale;
           }
         } else {
-          // 32x32b: thread = row (index query qbase + lane), all 128 columns
-          const int qa = qbase + lane, tt = qa >> 2;
-          const int lim = pos0 + tt;
-          const bool need_mask = pi * kBlock + kBlock - 1 > pos0 + (qbase >> 2);
+          // 32x32b: thread = query row rbase + lane, all 128 columns
+          const int qa = rbase + lane;
+          const int lim = (need_mask && qa < prow1) ? last_key(qa) : 0;
           float m = -INFINITY;
 #pragma unroll 1
           for (int h = 0; h < 4; ++h) {
@@ -408,27 +545,23 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
               for (int i = 0; i < 32; ++i)
                 if (pi * kBlock + 32 * h + i > lim) v[i] = -INFINITY;
             }
-            if (a.token_scores != nullptr && tt < a.T) {
-              float* rowp = a.token_scores + (((long long)pb * a.T + tt) * kG + (qa & 3)) * ctx +
-                            pi * kBlock + 32 * h;
+            if (a.token_scores != nullptr && qa < prow1) {
+              float* rowp = a.token_scores + (long long)qa * ctx + pi * kBlock + 32 * h;
 #pragma unroll
               for (int i = 0; i < 32; ++i) rowp[i] = v[i] * a.score_scale;
             }
             m = fmaxf(m, max_of<32>(v));
           }
-          if (tt < a.T)
-            a.block_scores[(((long long)pb * a.T + tt) * kG + (qa & 3)) * a.max_pages + pi] =
-                m * a.score_scale;
+          if (qa < prow1) a.block_scores[(long long)qa * a.max_pages + pi] = m * a.score_scale;
         }
       } else if (active && pkind == kPageMasked) {
         // no key of the block is visible to any query of the tile
         for (int r = lane; r < kRows; r += 32) {
-          const int qa = qbase + r, tt = qa >> 2;
-          if (tt >= a.T) continue;
-          const long long row = ((long long)pb * a.T + tt) * kG + (qa & 3);
-          a.block_scores[row * a.max_pages + pi] = -INFINITY;
+          const int qa = rbase + r;
+          if (qa >= prow1) continue;
+          a.block_scores[(long long)qa * a.max_pages + pi] = -INFINITY;
           if (a.token_scores != nullptr)
-            for (int j = 0; j < kBlock; ++j) a.token_scores[row * ctx + pi * kBlock + j] = -INFINITY;
+            for (int j = 0; j < kBlock; ++j) a.token_scores[(long long)qa * ctx + pi * kBlock + j] = -INFINITY;
         }
       }
       tc_fence_before();
@@ -437,8 +570,11 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     }
   } else {
     // ------------------------------------------------------------ decoders
-    const int row = 32 * warp + lane;                                     // key row of this thread
-    int cur_b = -1, cur_y = -1, qsel = 1;
+    const int d = 32 * warp + lane;                 // 0 .. 255
+    const int row = d & (kBlock - 1);               // key row of this thread
+    const int half = d >> 7;                        // elements 64*half .. 64*half+63
+    const int sw = (row >> 1) & 3;                  // 64-byte swizzle of the code rows
+    int cur_row0 = -1;
     for (int k = 0;; ++k) {
       const int s = k % S;
       if (!mbar_wait(&raw_full[s], (k / S) & 1)) { report(a.flags, 5, 5); break; }
@@ -449,23 +585,21 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         break;
       }
       const int* m = meta + 8 * s;
-      const int nb = m[0], ni = m[1], nkind = m[2], ny = m[3], nL = m[4];
-      if (nkind != kPageEnd && (nb != cur_b || ny != cur_y)) {
-        cur_b = nb;
-        cur_y = ny;
-        qsel ^= 1;
-        // A operand: the index queries of tile ny of sequence nb, K-major
-        // with the 128-byte swizzle, zero rows past the sequence's queries.
-        // Its previous user (a tile that ended two or more pages ago) has
-        // completed: the MMA of page k-2 has (the wait above).
-        uint8_t* qb = qbuf + qsel * M * C::kRow;
-        const int qbase = ny * M;
-        for (int idx = row; idx < M * 8; idx += kIdxDecWarps * 32) {
+      const int nrowp = m[0], ni = m[1], nkind = m[2], nr0 = m[3], nr1 = m[4], nminpos = m[5];
+      if (nkind != kPageEnd && nr0 != cur_row0) {
+        // A operand: the index-query rows [nr0, nr1) of the tile (rows of qi),
+        // K-major with the 128-byte swizzle, zero rows past nr1.  The previous
+        // tile's last MMA (page k-1 at the latest) must be done.
+        if (k >= 1 && !mbar_wait(&b_empty[(k - 1) & 1], ((k - 1) >> 1) & 1)) {
+          report(a.flags, 5, 7);
+          break;
+        }
+        cur_row0 = nr0;
+        for (int idx = d; idx < M * 8; idx += kIdxDecWarps * 32) {
           const int nrow = idx >> 3, c = idx & 7;
-          const int qg = qbase + nrow;
+          const int qg = nr0 + nrow;
           uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (qg < nq_all)
-            v = *reinterpret_cast<const uint4*>(a.qi + ((long long)nb * nq_all + qg) * kDim + 16 * c);
+          if (qg < nr1) v = *reinterpret_cast<const uint4*>(a.qi + (long long)qg * kDim + 16 * c);
           if constexpr (F16) {
             // dims 16c..16c+15 -> FP16 chunks 2c, 2c+1 of 8 dims: K-half c / 4,
             // chunk positions (2c % 8, 2c % 8 + 1) ^ (row % 8) in its 128-byte row
@@ -473,12 +607,12 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
                                         e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
             const uint4 hi = make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
                                         e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
-            uint8_t* rowp = qb + (c >> 2) * M * 128 + nrow * 128;
-            const int j = (2 * c) & 7;
-            sts128(rowp + ((j ^ (nrow & 7)) << 4), lo);
-            sts128(rowp + (((j + 1) ^ (nrow & 7)) << 4), hi);
+            uint8_t* rowp = qbuf + (c >> 2) * M * 128 + nrow * 128;
+            const int jj = (2 * c) & 7;
+            sts128(rowp + ((jj ^ (nrow & 7)) << 4), lo);
+            sts128(rowp + (((jj + 1) ^ (nrow & 7)) << 4), hi);
           } else {
-            sts128(qb + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
+            sts128(qbuf + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
           }
         }
       }
@@ -487,16 +621,19 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         uint8_t* bb = bbuf + (k & 1) * C::kBBytes;
         // 64-byte code rows loaded with the 64-byte swizzle: chunk c of row r
         // sits at chunk position c ^ ((r / 2) % 4); chunk c = elements
-        // 32c..32c+31 under scale bytes 2c and 2c+1
-        const uint2 sc = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
-        const int sw = (row >> 1) & 3;
+        // 32c..32c+31 under scale bytes 2c and 2c+1.  This thread: chunks
+        // 2*half and 2*half+1, scale bytes 4*half .. 4*half+3.
+        const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(rs + kPageCodes + row * kRowScales + 4 * half);
         if constexpr (F16) {
           // FP16 key row: 256 bytes as two 128-byte K-halves (rows 128 apart),
-          // each with the 128-byte swizzle; chunk c -> 16-byte chunks 4c..4c+3
+          // each with the 128-byte swizzle; chunk c -> 16-byte chunks 4(c%2)..
+          // of K-half c / 2 (= half)
+          uint8_t* rowp = bb + half * kBlock * 128 + row * 128;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
             const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-            const uint32_t s2 = e4m3x2_to_f16x2((c < 2 ? sc.x : sc.y) >> (16 * (c & 1)));
+            const uint32_t s2 = e4m3x2_to_f16x2(sc4 >> (16 * cc));
             const uint32_t s_lo = prmt(s2, 0u, 0x1010u), s_hi = prmt(s2, 0u, 0x3232u);
             uint32_t o[16];
             e2m1x8_to_f16x2(w4.x, o + 0);
@@ -505,31 +642,35 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
             e2m1x8_to_f16x2(w4.w, o + 12);
 #pragma unroll
             for (int mm = 0; mm < 16; ++mm) o[mm] = hmul2(o[mm], mm < 8 ? s_lo : s_hi);
-            uint8_t* rowp = bb + (c >> 1) * kBlock * 128 + row * 128;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int ch = 4 * (c & 1) + j;
+            for (int jj = 0; jj < 4; ++jj) {
+              const int ch = 4 * cc + jj;
               sts128(rowp + ((ch ^ (row & 7)) << 4),
-                     make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]));
+                     make_uint4(o[4 * jj], o[4 * jj + 1], o[4 * jj + 2], o[4 * jj + 3]));
             }
           }
         } else {
           // E4M3 key row: 128 bytes with the 128-byte swizzle; code chunk c ->
           // row chunks 2c, 2c+1
           uint8_t* rowp = bb + row * 128;
+          const uint4 w0 = lds128(rs + row * kRowCodes + (((2 * half) ^ sw) << 4));
+          const uint4 w1 = lds128(rs + row * kRowCodes + (((2 * half + 1) ^ sw) << 4));
+          const uint2 r0 = lut[sc4 & 0xFFu], r1 = lut[(sc4 >> 8) & 0xFFu];
+          const uint2 r2 = lut[(sc4 >> 16) & 0xFFu], r3 = lut[sc4 >> 24];
+          uint32_t o[16];
+          dq8(w0.x, r0, o[0], o[1]);
+          dq8(w0.y, r0, o[2], o[3]);
+          dq8(w0.z, r1, o[4], o[5]);
+          dq8(w0.w, r1, o[6], o[7]);
+          dq8(w1.x, r2, o[8], o[9]);
+          dq8(w1.y, r2, o[10], o[11]);
+          dq8(w1.z, r3, o[12], o[13]);
+          dq8(w1.w, r3, o[14], o[15]);
+          const int c0 = 4 * half;                   // first of this thread's 4 row chunks
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-            const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));   // scales 2c, 2c+1
-            const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
-            uint32_t o[8];
-            dq8(w4.x, r0, o[0], o[1]);
-            dq8(w4.y, r0, o[2], o[3]);
-            dq8(w4.z, r1, o[4], o[5]);
-            dq8(w4.w, r1, o[6], o[7]);
-            sts128(rowp + (((2 * c) ^ (row & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
-            sts128(rowp + (((2 * c + 1) ^ (row & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
-          }
+          for (int jj = 0; jj < 4; ++jj)
+            sts128(rowp + (((c0 + jj) ^ (row & 7)) << 4),
+                   make_uint4(o[4 * jj], o[4 * jj + 1], o[4 * jj + 2], o[4 * jj + 3]));
         }
       }
       fence_async_smem();   // generic-proxy writes (queries, keys) -> the MMA
@@ -537,7 +678,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       if (lane == 0) {
         if (warp == 0) {
           int* pf = pinfo + 8 * (k % kInfoRing);
-          pf[0] = nb; pf[1] = ni; pf[2] = nkind; pf[3] = ny; pf[4] = nL; pf[5] = qsel;
+          pf[0] = nrowp; pf[1] = ni; pf[2] = nkind; pf[3] = nr0; pf[4] = nr1; pf[5] = nminpos;
         }
         if (!FP8) mbar_arrive(&raw_empty[s]);
         mbar_arrive(&b_full[k & 1]);
@@ -566,7 +707,8 @@ static cudaError_t launch_mode(const IdxArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_indexer(const IdxArgs& a, int mode, cudaStream_t st) {
-  const bool m64 = idx_tile_queries(a.T) == 64;
+  // shared-prefix tiles span the query rows of several sequences: 128 rows
+  const bool m64 = !a.shared && idx_tile_queries(a.T) == 64;
   if (mode == kIdxFp8) return m64 ? launch_mode<kIdxFp8, 64>(a, st) : launch_mode<kIdxFp8, 128>(a, st);
   if (mode == kIdxF16) return m64 ? launch_mode<kIdxF16, 64>(a, st) : launch_mode<kIdxF16, 128>(a, st);
   return m64 ? launch_mode<kIdxNvfp4, 64>(a, st) : launch_mode<kIdxNvfp4, 128>(a, st);

@@ -11,7 +11,7 @@
 
 namespace msa {
 
-constexpr int kIdxThreads = 10 * 32;    // 4 decoders, 4 epilogue warps, producer, MMA warp
+constexpr int kIdxThreads = 14 * 32;    // 8 decoders, 4 epilogue warps, producer, MMA warp
 // Indexer arithmetic: NVFP4 keys re-rounded to E4M3 (FP8 MMA), E4M3 keys, or
 // NVFP4 keys decoded exactly to FP16 (FP16 MMA).
 enum : int { kIdxNvfp4 = 0, kIdxFp8 = 1, kIdxF16 = 2 };
@@ -30,6 +30,16 @@ struct IdxArgs {
   float score_scale;           // s_qi * s_idx
   int B, T, max_pages, num_pages;
   int part, nparts;            // score blocks [nblk*part/nparts, nblk*(part+1)/nparts) of each sequence
+  // Sequences sharing a cached prefix (null grp_start: none): group g is the
+  // sequences [grp_start[g], grp_start[g+1]), whose first grp_prefix[g]
+  // logical blocks are the same physical pages.  shared = 1 scores only those
+  // prefix blocks, once per group, against the index queries of all the
+  // group's sequences; shared = 0 scores every sequence's blocks from its
+  // group's prefix on.
+  const int32_t* grp_start;
+  const int32_t* grp_prefix;
+  int ngroups;
+  int shared;
 };
 
 size_t indexer_smem_bytes(int mode, int batch, int T);
@@ -57,7 +67,7 @@ cudaError_t launch_maxpool(const float* token_scores, const int32_t* seq_lens, i
                            int max_pages, float* block_scores, Flags* flags, cudaStream_t st);
 
 constexpr int kAttThreads = 14 * 32;    // 8 decoders, 4 softmax warps, producer, MMA warp
-constexpr int kAttStages = 2;            // raw K/V blocks in flight per CTA
+constexpr int kAttStages = 3;            // raw K/V blocks in flight per CTA
 constexpr int kAttWorkOffset = 72;       // int[2] in the workspace header (see kWorkOffset)
 constexpr int kPartialFloats = kHpg * kDim + 2 * kHpg;   // O[16][128], m[16], l[16]
 

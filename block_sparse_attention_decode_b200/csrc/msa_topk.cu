@@ -3,16 +3,24 @@
 // post = vLLM 為 MiniMax-M3.1-Flash 提供 Day-0 支援 (hot.atechcom.net).
 //
 // One warp per (sequence, token, group) row, four rows per CTA, no block-wide
-// synchronisation.  The latest visible block is
-// kept; the other 15 are the best of blocks 0 .. latest-1 ranked by (score
-// descending, block id ascending).  Selection is an exact radix select over
-// order-preserving 32-bit keys of the fp32 scores (4 passes of 8 bits) that
-// finds the 15th key value and how many blocks equal to it are still needed;
-// a final pass in id order keeps every block above that value and the lowest
-// ids among the equal ones, which also emits the ids in ascending order.
-// No sort, no inter-CTA communication, and the result does not depend on how
-// the indexer split its work (the selection stays exact, as in the post's
-// "NVFP4 indexer DCP" section).
+// synchronisation.  The latest visible block is kept; the other 15 are the
+// best of blocks 0 .. latest-1 ranked by (score descending, block id
+// ascending), scores compared as order-preserving 32-bit keys of the fp32
+// values (-0 taken as +0).
+//
+// Fast path: the keys are staged in shared memory; tau = the 15th largest of
+// the 32 lanes' maxima is at most the 15th largest key (the 15 lanes with
+// the largest maxima hold 15 keys >= tau), so every block of the selection
+// has a key >= tau.  The blocks with key >= tau -- usually a few dozen -- are
+// compacted (ballots) into a candidate list, ranked exactly against each
+// other, and the 15 best are written in id order.  When more than
+// kTopkCand blocks reach tau (heavy ties), the row falls back to an exact
+// radix select over all keys (8-bit digits from the first byte where the
+// keys differ) that finds the 15th key and how many blocks equal to it are
+// needed, then keeps every block above it and the lowest ids among the equal
+// ones.  No sort, no inter-CTA communication, and the result does not depend
+// on how the indexer split its work (the selection stays exact, as in the
+// post's "NVFP4 indexer DCP" section).
 #include "msa_internal.h"
 
 namespace msa {
@@ -20,12 +28,19 @@ namespace msa {
 constexpr int kTopkRows = 4;                  // rows (warps) per CTA
 constexpr int kTopkThreads = 32 * kTopkRows;
 constexpr int kTopkCache = 2048;              // candidates per row cached in shared memory
+constexpr int kTopkCand = 64;                 // fast path: at most this many blocks reach tau
+
+// Order-preserving key of a block score with -0 taken as +0 (the ranking
+// compares values, and -0 == +0).
+__device__ __forceinline__ unsigned score_key(float f) { return float_key(f + 0.0f); }
 
 __global__ void __launch_bounds__(kTopkThreads)
 topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_lens, int B, int T,
             int max_pages, int32_t* __restrict__ sel, Flags* flags) {
   __shared__ unsigned keys_all[kTopkRows][kTopkCache];
   __shared__ unsigned hist_all[kTopkRows][256];
+  __shared__ unsigned cand_key_all[kTopkRows][kTopkCand];
+  __shared__ int cand_id_all[kTopkRows][kTopkCand];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const long long row = (long long)blockIdx.x * kTopkRows + w;   // (b * T + t) * 4 + g
   if (row >= (long long)B * T * kG) return;
@@ -51,15 +66,79 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_le
   const bool cached = n <= kTopkCache;
   unsigned kmin = 0xFFFFFFFFu, kmax = 0u;
   for (int i = lane; i < n; i += 32) {
-    const unsigned k = float_key(S[i]);
+    const unsigned k = score_key(S[i]);
     if (cached) keys[i] = k;
     kmin = min(kmin, k);
     kmax = max(kmax, k);
   }
   __syncwarp();
+  auto key_at = [&](int i) -> unsigned { return cached ? keys[i] : score_key(S[i]); };
+
+  // ---- fast path: candidates with key >= tau, ranked exactly
+  {
+    // tau = the 15th largest lane maximum (lanes without candidates hold 0,
+    // below every key; n >= 16 lanes hold one)
+    int above = 0;
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) {
+      const unsigned x = __shfl_sync(0xffffffffu, kmax, m);
+      above += (x > kmax) || (x == kmax && m < lane);
+    }
+    const unsigned tau = __shfl_sync(0xffffffffu, kmax, __ffs(__ballot_sync(0xffffffffu, above == kTopk - 2)) - 1);
+    unsigned* ck = cand_key_all[w];
+    int* cid = cand_id_all[w];
+    int count = 0;                       // candidates so far (warp-uniform)
+    for (int base = 0; base < n; base += 32) {
+      const int i = base + lane;
+      const bool c = i < n && key_at(i) >= tau;
+      const unsigned bal = __ballot_sync(0xffffffffu, c);
+      const int slot = count + __popc(bal & ((1u << lane) - 1u));
+      if (c && slot < kTopkCand) { ck[slot] = key_at(i); cid[slot] = i; }
+      count += __popc(bal);
+    }
+    __syncwarp();
+    if (count <= kTopkCand) {
+      // rank of candidate j = how many candidates precede it in (key desc, id asc)
+      int sel_mask_lo = 0, sel_mask_hi = 0;   // lane holds candidates lane and lane + 32
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = lane + 32 * h;
+        if (j < count) {
+          const unsigned kj = ck[j];
+          const int ij = cid[j];
+          int r = 0;
+          for (int m = 0; m < count; ++m) {
+            const unsigned km = ck[m];
+            r += (km > kj) || (km == kj && cid[m] < ij);
+          }
+          if (r < kTopk - 1) { if (h) sel_mask_hi = 1; else sel_mask_lo = 1; }
+        }
+      }
+      __syncwarp();
+      // the 15 selected ids in ascending order: position = selected ids below
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = lane + 32 * h;
+        const bool mine = h ? sel_mask_hi : sel_mask_lo;
+        const unsigned b0 = __ballot_sync(0xffffffffu, sel_mask_lo), b1 = __ballot_sync(0xffffffffu, sel_mask_hi);
+        if (mine) {
+          const int ij = cid[j];
+          int posn = 0;
+          for (int m = 0; m < 32; ++m) {
+            if ((b0 >> m) & 1u) posn += cid[m] < ij;
+            if ((b1 >> m) & 1u) posn += cid[m + 32] < ij;
+          }
+          out[posn] = ij;
+        }
+      }
+      if (lane == 0) out[kTopk - 1] = nb - 1;
+      return;
+    }
+  }
+
+  // ---- fallback: exact radix select over all keys (heavy ties)
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
-  auto key_at = [&](int i) -> unsigned { return cached ? keys[i] : float_key(S[i]); };
 
   // Radix select, 8 bits per pass from the top: after the passes `prefix`
   // is the key of the 15th best candidate and `need` how many candidates

@@ -111,17 +111,36 @@ class Workload:
         return self.k_data.device
 
 
-def _page_map(batch, nblk, max_pages, paged, seed, device):
-    """Logical (b, i) -> physical page.  Contiguous: page = b*max_pages + i."""
+def _page_map(batch, nblk, max_pages, paged, seed, device, prefix_groups=None):
+    """Logical (b, i) -> physical page.  Contiguous: page = b*max_pages + i.
+
+    prefix_groups: [(users, prefix_blocks), ...] covering the batch in order:
+    the sequences of a group map their first prefix_blocks logical blocks to
+    the same physical pages (those of the group's first sequence)."""
     if not paged:
+        assert not prefix_groups, "shared prefixes need a page table"
         return None, batch * max_pages
-    total = int(sum(nblk))
+    groups = prefix_groups or [(1, 0)] * batch
+    assert sum(u for u, _ in groups) == batch
+    total = 0
+    b = 0
+    for users, pre in groups:
+        assert all(pre <= nblk[b + j] for j in range(users))
+        total += pre + sum(nblk[b + j] - pre for j in range(users))
+        b += users
     perm = torch.randperm(total, generator=_gen(seed, 1, "cpu"))
     pt = torch.full((batch, max_pages), -1, dtype=torch.int32)
     off = 0
-    for b in range(batch):
-        pt[b, : nblk[b]] = perm[off: off + nblk[b]].to(torch.int32)
-        off += nblk[b]
+    b = 0
+    for users, pre in groups:
+        shared = perm[off: off + pre].to(torch.int32)
+        off += pre
+        for j in range(users):
+            pt[b, :pre] = shared
+            n = nblk[b] - pre
+            pt[b, pre: nblk[b]] = perm[off: off + n].to(torch.int32)
+            off += n
+            b += 1
     return pt.to(device), total
 
 
@@ -129,19 +148,23 @@ def make_workload(name: str, batch: int, seq_lens, q_tokens: int, *, paged: bool
                   seed: int, device="cpu", idx_fp8: bool = False, max_pages: int | None = None,
                   plant_every: int = 0, scale_floor_byte: int = 0,
                   neg_scale_frac: float = 0.0, chunk_pages: int = 2048,
-                  idx_exact: bool = False) -> Workload:
+                  idx_exact: bool = False, prefix_groups=None) -> Workload:
     """Build a workload.  seq_lens counts the q_tokens new tokens (which are the
     last q_tokens positions of each sequence).
 
     ``neg_scale_frac`` > 0 sets the sign bit of that fraction of the block-scale
-    bytes (index, K and V), to exercise signed E4M3 block scales."""
+    bytes (index, K and V), to exercise signed E4M3 block scales.
+
+    ``prefix_groups`` = [(users, prefix_blocks), ...] (paged only): consecutive
+    groups of sequences whose first prefix_blocks logical blocks are the same
+    physical pages, as a serving engine's prefix cache shares them."""
     seq_lens = [int(L) for L in seq_lens]
     assert len(seq_lens) == batch and all(L >= q_tokens >= 1 for L in seq_lens)
     nblk = [(L + BLOCK - 1) // BLOCK for L in seq_lens]
     if max_pages is None:
         max_pages = max(nblk)
     assert max_pages >= max(nblk)
-    page_table, num_pages = _page_map(batch, nblk, max_pages, paged, seed, device)
+    page_table, num_pages = _page_map(batch, nblk, max_pages, paged, seed, device, prefix_groups)
 
     # queries (pre-quantisation N(0,1), one stream per tensor)
     qi_f = torch.randn(batch, q_tokens, G, D, generator=_gen(seed, 2, device), device=device)

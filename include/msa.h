@@ -132,6 +132,24 @@ typedef struct {
     int32_t max_pages;          /* row length of page_table; upper bound on blocks */
 } msa_seqs;
 
+/* Sequences of the batch that share a cached prefix: [post, "AMD GPU
+ * support", "NVFP4 MSA kernel"] dequantises a shared-prefix page once for
+ * the requests that share it.  Group g is the sequences [seq_start[g],
+ * seq_start[g+1]) (consecutive in the batch); the first prefix_blocks[g]
+ * logical blocks of each of them are the same physical pages (equal page
+ * table entries), and every key of those blocks is visible to every query of
+ * the group (prefix_blocks[g]*128 <= seq_lens[b] - q_tokens).  Groups cover
+ * the batch: seq_start[0] = 0, non-decreasing, seq_start[num_groups] = batch;
+ * a sequence without a shared prefix is a group of one with prefix 0.
+ * Arrays that break these rules are reported on the device
+ * (MSA_ERR_DEVICE_BOUNDS) and give unspecified scores; they are clamped to
+ * the batch and the page table, so no access leaves the buffers. */
+typedef struct {
+    const int32_t* seq_start;      /* device [num_groups + 1] */
+    const int32_t* prefix_blocks;  /* device [num_groups] */
+    int32_t num_groups;            /* 1 .. batch */
+} msa_prefix_groups;
+
 /* Bytes of device workspace the calls below need for `seqs` (error flags,
  * block scores, selection, attention partials).  The size depends on `seqs`
  * alone (not on the device), so it can be computed without a GPU.  The
@@ -201,10 +219,32 @@ MSA_API msa_status msa_sparse_attn_decode(const msa_cache* cache, const msa_seqs
                                   float softmax_scale, uint16_t* out,
                                   void* ws, size_t ws_bytes, msa_stream_t stream);
 
+/* msa_indexer_score for a batch whose sequences share prefixes (`groups`,
+ * which requires a page table): the same scores, but each shared-prefix
+ * page is read and decoded for a tile of up to 128 index queries drawn from
+ * all the sequences of its group (the tiles of one page run side by side,
+ * so the page comes from HBM once and from L2 after that), instead of once
+ * per sequence; the remaining blocks of each sequence are scored as by
+ * msa_indexer_score.  [post, "AMD GPU support", "NVFP4 MSA kernel"]. */
+MSA_API msa_status msa_indexer_score_grouped(const msa_cache* cache, const msa_seqs* seqs,
+                             const msa_prefix_groups* groups,
+                             const uint8_t* qi, float s_qi,
+                             float* token_scores, float* block_scores,
+                             void* ws, size_t ws_bytes, msa_stream_t stream);
+
 /* The whole decode step: indexer -> max-pool -> top-16 -> sparse attention,
  * back to back on `stream` with intermediates in the workspace.
  * sel_out: optional [B][T][4][16] copy of the selection (NULL = skip). */
 MSA_API msa_status msa_decode(const msa_cache* cache, const msa_seqs* seqs,
+                      const uint8_t* qi, float s_qi, const uint8_t* q, float s_q,
+                      float softmax_scale, uint16_t* out, int32_t* sel_out,
+                      void* ws, size_t ws_bytes, msa_stream_t stream);
+
+/* msa_decode with the indexer of msa_indexer_score_grouped (shared-prefix
+ * pages decoded once per tile of the group's index queries); the selection
+ * and the output are those of msa_decode. */
+MSA_API msa_status msa_decode_grouped(const msa_cache* cache, const msa_seqs* seqs,
+                      const msa_prefix_groups* groups,
                       const uint8_t* qi, float s_qi, const uint8_t* q, float s_q,
                       float softmax_scale, uint16_t* out, int32_t* sel_out,
                       void* ws, size_t ws_bytes, msa_stream_t stream);

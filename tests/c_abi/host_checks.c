@@ -37,6 +37,9 @@ int main(void)
            offsetof(msa_seqs, page_table), offsetof(msa_seqs, seq_lens),
            offsetof(msa_seqs, batch), offsetof(msa_seqs, q_tokens),
            offsetof(msa_seqs, max_pages));
+    printf("msa_prefix_groups %zu %zu %zu %zu\n", sizeof(msa_prefix_groups),
+           offsetof(msa_prefix_groups, seq_start), offsetof(msa_prefix_groups, prefix_blocks),
+           offsetof(msa_prefix_groups, num_groups));
 
     CHECK(msa_workspace_size(&s) > 0);
     s.batch = 0;
@@ -64,6 +67,21 @@ int main(void)
                                  big, NULL) == MSA_ERR_INVALID_ARG);
     CHECK(msa_kv_insert(&c, &s, NULL, (const uint16_t*)FAKE, (const uint16_t*)FAKE, FAKE, big,
                         NULL) == MSA_ERR_INVALID_ARG);
+    {   /* prefix groups: present, 1..batch groups, and a page table */
+        msa_prefix_groups g = {(const int32_t*)FAKE, (const int32_t*)FAKE, 1};
+        CHECK(msa_indexer_score_grouped(&c, &s, NULL, q, 1.0f, NULL, (float*)FAKE, FAKE, big, NULL) ==
+              MSA_ERR_INVALID_ARG);
+        CHECK(msa_indexer_score_grouped(&c, &s, &g, q, 1.0f, NULL, (float*)FAKE, FAKE, big, NULL) ==
+              MSA_ERR_INVALID_ARG);   /* s.page_table is NULL */
+        s.page_table = (const int32_t*)FAKE;
+        g.num_groups = 3;             /* more groups than sequences */
+        CHECK(msa_decode_grouped(&c, &s, &g, q, 1.0f, q, 1.0f, 0.1f, out, NULL, FAKE, big, NULL) ==
+              MSA_ERR_INVALID_ARG);
+        g.num_groups = 0;
+        CHECK(msa_decode_grouped(&c, &s, &g, q, 1.0f, q, 1.0f, 0.1f, out, NULL, FAKE, big, NULL) ==
+              MSA_ERR_INVALID_ARG);
+        s.page_table = NULL;
+    }
     CHECK(msa_status_string(MSA_OK) != NULL && msa_status_string(MSA_ERR_TIMEOUT) != NULL);
     puts("ok");
     return 0;

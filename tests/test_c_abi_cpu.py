@@ -35,7 +35,8 @@ def test_c_program_host_checks_and_layout(program):
     lines = {l.split()[0]: [int(x) for x in l.split()[1:]] for l in r.stdout.splitlines()
              if l.startswith("msa_")}
     assert r.stdout.strip().endswith("ok")
-    for struct, name in ((msa.msa_cache, "msa_cache"), (msa.msa_seqs, "msa_seqs")):
+    for struct, name in ((msa.msa_cache, "msa_cache"), (msa.msa_seqs, "msa_seqs"),
+                         (msa.msa_prefix_groups, "msa_prefix_groups")):
         size, *offsets = lines[name]
         assert size == ctypes.sizeof(struct), name
         assert offsets == [getattr(struct, f).offset for f, _ in struct._fields_], name
