@@ -176,6 +176,15 @@ msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi,
   if (!encode_row_tmap(&a.tmap_idx, c->idx_data, (uint64_t)c->num_pages * MSA_BLOCK_TOKENS,
                        fp8 ? MSA_HEAD_DIM : MSA_HEAD_DIM / 2))
     return MSA_ERR_CUDA;
+  const int mode = fp8 ? kIdxFp8 : (c->idx_dtype == MSA_IDX_NVFP4_EXACT ? kIdxF16 : kIdxNvfp4);
+  // the query tiles: 64 rows when a sequence has at most 64 index queries,
+  // else (and for shared prefixes, whose tiles span sequences) 128; loaded
+  // in boxes of 8 rows when they are spread over the four lane quarters
+  a.spread = idx_spread_rows(s->q_tokens, mode, shared) ? 1 : 0;
+  const int tile = a.spread ? 8 : (shared || idx_tile_queries(s->q_tokens) == 128) ? 128 : 64;
+  if (!encode_row_tmap(&a.tmap_qi, qi, (uint64_t)s->batch * s->q_tokens * MSA_KV_HEADS, MSA_HEAD_DIM,
+                       tile))
+    return MSA_ERR_CUDA;
   a.idx_data = c->idx_data;
   a.idx_scale = c->idx_scale;
   a.page_table = s->page_table;
@@ -192,7 +201,6 @@ msa_status run_indexer(const msa_cache* c, const msa_seqs* s, const uint8_t* qi,
   a.num_pages = c->num_pages;
   a.part = part;
   a.nparts = nparts;
-  const int mode = fp8 ? kIdxFp8 : (c->idx_dtype == MSA_IDX_NVFP4_EXACT ? kIdxF16 : kIdxNvfp4);
   return cuda_status(launch_indexer(a, mode, st));
 }
 

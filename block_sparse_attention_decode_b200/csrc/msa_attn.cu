@@ -25,8 +25,8 @@
 //       S^T[128 keys x 16 heads]  = K Q^T   (4 MMAs, A from TMEM)
 //       O^T[128 dims x 32]       += V^T [P_hi | P_lo]^T  (4 MMAs, A and B in
 //                                   shared memory, both MN-major),
-//     issuing block k+1's S before block k's O so that the softmax of the
-//     next block overlaps the O update;
+//     the two streams polled independently, so that the S of the next block
+//     is issued while the softmax of this one runs;
 //   warps 4-11 (softmax): warp 4+4j+q reads heads 8j..8j+7 of the S^T lanes
 //     of quarter q (thread = key), masks keys after the query position,
 //     takes the per-head block maximum (warp reduction, then across the four
@@ -52,6 +52,7 @@ constexpr int kAttDecoders = 4;             // warps 0-3, one per TMEM lane quar
 constexpr int kAttSoftWarp0 = 4;            // softmax warps 4-11: two per lane quarter
 constexpr int kAttSoft = 8;
 constexpr int kHh = kHpg / 2;               // heads per softmax warp
+static_assert(kHh == 8, "softmax warps hold eight heads (two float4 of block maxima)");
 constexpr int kAttProducerWarp = 12;
 constexpr int kAttMmaWarp = 13;
 constexpr int kAttRawStride = 2 * (kPageCodes + kPageScales);   // 18432 = 18 x 1024
@@ -59,7 +60,7 @@ constexpr int kAttTmemCols = 256;           // A[2] 0..63, S[2] 64..95, O[2] 96.
 constexpr int kColA = 0, kColS = 64, kColO = 96;
 constexpr float kPExp = 4.f;                // P carries a factor 2^4 (E4M3 normal range)
 constexpr float kLazy = 4.f;                // raise m only when a block max exceeds it by 2^4
-constexpr int kVB = 2;                      // V and P buffers (blocks between decode and O update)
+constexpr int kVB = 3;                      // V and P buffers (blocks between decode and O update)
 
 enum : int { kBlkLoad = 0, kBlkEmpty = 1, kBlkEnd = 2 };
 
@@ -200,6 +201,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // launched with programmatic serialisation: the prologue above overlapped
+  // the previous kernel; its outputs (the selection) are read from here on
+  grid_dependency_wait();
 
   if (warp == kAttProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -238,14 +242,16 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       ++k;
       return good;
     };
-    // Item lookup, one lane per selected block of the item's slice: the
-    // block id (from sel) and its page (page table).  Done for the next item
-    // while the current item's blocks are issued, so its global loads do not
-    // stall the copies.
-    struct Look { long long row; int sp, b, t, g, L, pos, blk; long long page; bool valid; };
-    auto lookup = [&](long long it) -> Look {
+    // Item lookup, one lane per selected block of the item's slice, in two
+    // steps one item apart, so that no global load is waited for right after
+    // it is issued: lookup_sel reads the item's length and selected block id
+    // (two items ahead), lookup_page its page-table entry (one item ahead).
+    struct Look { long long it, row; int sp, b, t, g, L, blk; long long page; };
+    auto lookup_sel = [&](long long it) -> Look {
       Look r{};
-      r.valid = false;
+      r.it = it;
+      r.page = -1;
+      r.blk = -1;
       if (it >= items) return r;
       r.row = it / a.splits;
       r.sp = (int)(it % a.splits);
@@ -257,19 +263,29 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       if (lane >= k0 && lane < k1) r.blk = a.sel[r.row * kTopk + lane];
       return r;
     };
-    // Items are claimed two ahead: the claim of item n+2 is issued before
+    auto lookup_page = [&](Look& r) {
+      if (r.it >= items) return;
+      const bool len_ok = r.L >= a.T && r.L <= a.max_pages * kBlock;
+      if (!len_ok || r.blk < 0 || r.blk >= (r.L - a.T + r.t) / kBlock + 1) return;
+      r.page = a.page_table ? (long long)a.page_table[(long long)r.b * a.max_pages + r.blk]
+                            : (long long)r.b * a.max_pages + r.blk;
+    };
+    // Items are claimed three ahead: the claim of item n+3 is issued before
     // item n's blocks, and its value is only read one item later.
-    long long item = 0, nxt = 0, claim = 0;
+    long long c0 = 0, c1 = 0, nxt2 = 0, claim = 0;
     if (lane == 0) {
-      item = atomicAdd(&a.work[0], 1);
-      nxt = atomicAdd(&a.work[0], 1);
+      c0 = atomicAdd(&a.work[0], 1);
+      c1 = atomicAdd(&a.work[0], 1);
+      nxt2 = atomicAdd(&a.work[0], 1);
     }
-    item = __shfl_sync(0xffffffffu, item, 0);
-    Look cur = lookup(item);
+    Look cur = lookup_sel(__shfl_sync(0xffffffffu, c0, 0));
+    lookup_page(cur);
+    Look next = lookup_sel(__shfl_sync(0xffffffffu, c1, 0));
+    long long item = cur.it;
     while (item < items && ok) {
       if (lane == 0) claim = atomicAdd(&a.work[0], 1);
-      nxt = __shfl_sync(0xffffffffu, nxt, 0);
-      const Look next = lookup(nxt);
+      lookup_page(next);
+      const Look next2 = lookup_sel(__shfl_sync(0xffffffffu, nxt2, 0));
       const long long row = cur.row;
       const int sp = cur.sp, b = cur.b, t = cur.t, g = cur.g, L = cur.L;
       const bool len_ok = L >= a.T && L <= a.max_pages * kBlock;
@@ -286,8 +302,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         if (blk >= nvis) {
           report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, blk);
         } else if (blk >= 0) {
-          page = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + blk]
-                              : (long long)b * a.max_pages + blk;
+          page = cur.page;                         // looked up one item ago
           if (page < 0 || page >= a.num_pages) report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)page);
           else valid = true;
         }
@@ -322,8 +337,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       }
       ++ki;
       cur = next;
-      item = nxt;
-      nxt = claim;                                    // lane 0's value, broadcast next time
+      next = next2;
+      item = cur.it;
+      nxt2 = claim;                                   // lane 0's value, broadcast next time
     }
     if (ok) emit(kBlkEnd, 0, 0, 0, 0, 0, 0, 0, 0);
     // every CTA has made its last claim once all have arrived here
@@ -339,8 +355,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_e4m3_f32(128, kHpg);
       constexpr uint32_t idesc_o = idesc_e4m3_f32(128, 2 * kHpg) | (1u << 15) | (1u << 16);
-      const uint64_t qd[2] = {desc_kmajor_sw128(smem_u32(qbuf)),
-                              desc_kmajor_sw128(smem_u32(qbuf + kHpg * kDim))};
+      const uint64_t qd0 = desc_kmajor_sw128(smem_u32(qbuf));
+      const uint64_t qd1 = desc_kmajor_sw128(smem_u32(qbuf + kHpg * kDim));
       // The S and O streams run independently: S of block ks as soon as its K
       // is decoded and the softmax has read S of block ks-2 (same buffer);
       // O of block ko as soon as its P is written.  Both are polled without
@@ -361,7 +377,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
                 tc_fence_after();
                 const uint32_t d = tmem + kColS + kHpg * x;
                 const uint32_t ta = tmem + kColA + 32 * x;
-                const uint64_t bd = qd[ki & 1];
+                const uint64_t bd = (ki & 1) ? qd1 : qd0;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc_s, kk > 0);
               }
@@ -448,10 +464,12 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         }
         // block maximum per head: this warp's 32 keys, then the four quarters
         float* rq = red + ((nred & 1) * 4 + q) * kHpg + h0;
+        float mh[kHh];
 #pragma unroll
-        for (int h = 0; h < kHh; ++h) {
-          const float mh = warp_max(s[h]);
-          if (lane == h) rq[h] = mh;
+        for (int h = 0; h < kHh; ++h) mh[h] = warp_max(s[h]);
+        if (lane == 0) {
+          reinterpret_cast<float4*>(rq)[0] = make_float4(mh[0], mh[1], mh[2], mh[3]);
+          reinterpret_cast<float4*>(rq)[1] = make_float4(mh[4], mh[5], mh[6], mh[7]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(red_full);
@@ -715,8 +733,7 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   cudaError_t e = persistent_grid(reinterpret_cast<const void*>(attn_kernel), kAttThreads, smem,
                                   kAttTmemCols, &grid);
   if (e != cudaSuccess) return e;
-  attn_kernel<<<grid, kAttThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(attn_kernel, dim3(grid), dim3(kAttThreads), smem, st, a);
 }
 
 // ----------------------------------------------------- parity debug hook --

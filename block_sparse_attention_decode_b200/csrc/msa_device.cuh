@@ -38,6 +38,18 @@ struct Flags {
 };
 constexpr int kWorkOffset = 64;   // int[2]: next work item, CTAs finished (0 between calls)
 
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed and their writes are visible (returns at once when the
+// kernel was launched without programmatic serialisation), and let the next
+// kernel on the stream start launching once every CTA of this one has called
+// it or exited.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 __device__ __forceinline__ void report(Flags* f, int code, int detail) {
   if (atomicCAS(&f->code, 0, code) == 0) atomicExch(&f->detail, detail);
 }

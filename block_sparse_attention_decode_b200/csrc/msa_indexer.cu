@@ -88,11 +88,11 @@ __host__ __device__ inline IdxLayout idx_layout(int batch) {
   using C = IdxCfg<MODE>;
   IdxLayout L;
   int off = 0;
-  L.qbuf = off;    off += M * C::kRow;                     // the query tile (a multiple of 1024)
+  L.qbuf = off;    off += (C::kF16 ? 1 : 2) * M * C::kRow;  // query tiles (multiples of 1024)
   L.raw = off;     off += C::kStages * C::kRawStride;
   L.bbuf = off;    off += C::kNB * C::kBBytes;
   L.lut = off;     off += MODE == kIdxNvfp4 ? 256 * 8 : 0;
-  L.bars = off;    off += (2 * C::kStages + 8) * 8;
+  L.bars = off;    off += (2 * C::kStages + 12) * 8;
   L.meta = off;    off += C::kStages * 8 * 4;              // per stage: ptrow, i, kind, row0, row1, minpos
   L.pinfo = off;   off += kInfoRing * 8 * 4;               // per page: the same
   L.tslot = off;   off += 16;
@@ -104,6 +104,8 @@ __host__ __device__ inline IdxLayout idx_layout(int batch) {
 
 // Index queries per tile: a tile is the M side of the MMA.
 int idx_tile_queries(int T) { return kG * T <= 64 ? 64 : 128; }
+
+bool idx_spread_rows(int T, int mode, int shared) { return !shared && mode != kIdxF16 && kG * T <= 32; }
 
 size_t indexer_smem_bytes(int mode, int batch, int T) {
   const bool m64 = idx_tile_queries(T) == 64;
@@ -274,6 +276,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   uint64_t* b_empty = b_full + 2;        // [2] MMA -> decoders: page k consumed
   uint64_t* d_full = b_empty + 2;        // [2] MMA -> epilogue
   uint64_t* d_empty = d_full + 2;        // [2] epilogue -> MMA
+  uint64_t* q_full = d_empty + 2;        // [2] producer (TMA) -> MMA: an item's query tile
+  uint64_t* q_empty = q_full + 2;        // [2] MMA -> producer: the item's last MMA done
   int* meta = reinterpret_cast<int*>(smem + Ly.meta);
   int* pinfo = reinterpret_cast<int*>(smem + Ly.pinfo);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
@@ -298,6 +302,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       mbar_init(&b_empty[x], 1);
       mbar_init(&d_full[x], 1);
       mbar_init(&d_empty[x], 4);
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
     }
     mbar_fence_init();
   }
@@ -308,6 +314,9 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   tc_fence_before();
   const int nent = build_items<M>(a, prefix, lens, skip, gstart, gpre, scratch);   // ends with __syncthreads
   tc_fence_after();
+  // the next kernel on the stream (the top-16) may start launching: its CTAs
+  // take SMs as this kernel's persistent CTAs leave, and wait for its end
+  grid_launch_dependents();
   const uint32_t tmem = *tslot;
 
   const int items = prefix[nent];
@@ -366,7 +375,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     // Items are claimed two ahead: the claim of item n+2 (an atomic whose
     // latency is a microsecond or more) is issued before item n's pages, and
     // its value is only read one item later.
-    int item = 0, nxt = 0, claim = 0;
+    int item = 0, nxt = 0, claim = 0, ki = 0;      // ki: items of this CTA so far
     if (lane == 0) {
       item = atomicAdd(&a.work[0], 1);
       nxt = atomicAdd(&a.work[0], 1);
@@ -382,6 +391,26 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         report(a.flags, 4 /*MSA_ERR_DEVICE_BOUNDS*/, (int)cur.p);
         cur.kind = kPageBad;
       }
+      // the item's query tile (E4M3 modes): one TMA load of its rows into
+      // buffer ki % 2 once the MMAs of item ki-2 are done; rows past the
+      // tile's end are read too (zero past the end of qi) and never used
+      const int qx = ki & 1;
+      if (!F16 && lane == 0) {
+        if (ki >= 2 && !mbar_wait(&q_empty[qx], ((ki >> 1) - 1) & 1)) {
+          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 8);
+          ok = false;
+        } else if (M == 64 && a.spread) {
+          // boxes of 8 rows at MMA rows 16j.. (one 1 KB swizzle atom each)
+          const int nbox = (cur.row1 - cur.row0 + 7) >> 3;
+          mbar_expect_tx(&q_full[qx], nbox * 8 * 128);
+          for (int j = 0; j < nbox; ++j)
+            tma_load_2d(qbuf + qx * M * 128 + j * 16 * 128, &a.tmap_qi, 0, cur.row0 + 8 * j, &q_full[qx]);
+        } else {
+          mbar_expect_tx(&q_full[qx], M * 128);
+          tma_load_2d(qbuf + qx * M * 128, &a.tmap_qi, 0, cur.row0, &q_full[qx]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
       for (int j = 0; j < cur.np && ok; ++j, ++k) {
         const int ij = __shfl_sync(0xffffffffu, cur.i, j);
         const int kj = __shfl_sync(0xffffffffu, cur.kind, j);
@@ -394,6 +423,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
             const int s = k % S;
             int* m = meta + 8 * s;
             m[0] = cur.ptrow; m[1] = ij; m[2] = kj; m[3] = cur.row0; m[4] = cur.row1; m[5] = cur.minpos;
+            m[6] = ki; m[7] = (j == 0) | ((j == cur.np - 1) << 1);   // first / last page of the item
             uint8_t* dst = raw + s * C::kRawStride;
             if (kj == kPageLoad) {
               mbar_expect_tx(&raw_full[s], C::kRaw);
@@ -409,6 +439,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       cur = next;
       item = nxt;
       nxt = claim;                                  // lane 0's value, broadcast next time
+      ++ki;
     }
     if (lane == 0) {
       if (ok) {   // end marker
@@ -436,10 +467,16 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         if (k >= 2 && !mbar_wait(&d_empty[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 3); break; }
         tc_fence_after();
         const int* pf = pinfo + 8 * (k % kInfoRing);
-        const int kind = pf[2];
+        const int kind = pf[2], ki = pf[6], flg = pf[7];
+        const int qx = F16 ? 0 : (ki & 1);
+        if (!F16 && kind != kPageEnd && (flg & 1) && !mbar_wait(&q_full[qx], (ki >> 1) & 1)) {
+          report(a.flags, 5, 9);
+          break;
+        }
+        tc_fence_after();
         if (kind == kPageLoad) {
           const uint32_t d = tmem + (uint32_t)(x * kBlock);
-          const uint32_t qa = smem_u32(qbuf);
+          const uint32_t qa = smem_u32(qbuf + qx * M * 128);
           const uint32_t kb = FP8 ? smem_u32(raw + (k % S) * C::kRawStride)
                                   : smem_u32(bbuf + x * C::kBBytes);
           if constexpr (F16) {
@@ -458,14 +495,17 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         if (kind == kPageEnd) break;
         if (FP8) tc_commit(&raw_empty[k % S]);   // the stage was the B operand
         tc_commit(&b_empty[x]);                   // page k consumed (and its B buffer free)
+        if (!F16 && (flg & 2)) tc_commit(&q_empty[qx]);   // the item's query tile is free
       }
     }
   } else if (warp >= kIdxEpiWarp0) {
     // ------------------------------------------------------------ epilogue
     const int q = warp - kIdxEpiWarp0;             // TMEM lane quarter
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-    // rows of the tile this warp reads: M = 64: 16q..16q+15; M = 128: 32q..32q+31
-    constexpr int kRows = M == 64 ? 16 : 32;
+    // rows of the tile this warp reads: M = 64: 16q..16q+15 (spread: 8q..8q+7);
+    // M = 128: 32q..32q+31
+    const bool spread = M == 64 && a.spread;
+    const int kRows = M == 64 ? (spread ? 8 : 16) : 32;
     for (int k = 0;; ++k) {
       const int x = k & 1;
       if (!mbar_wait(&d_full[x], (k >> 1) & 1)) { report(a.flags, 5, 6); break; }
@@ -477,18 +517,20 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       const bool active = rbase < prow1;             // warp-uniform
       // a key j is visible to query row r when j <= pos(r) = L_b - T + t
       const bool need_mask = pi * kBlock + kBlock - 1 > pminpos;
-      auto last_key = [&](int r) -> int {
+      auto last_key = [&](int r) -> int {    // rows past the last sequence hold no query
+        if (r >= a.B * nq_all) return -1;
         const int b = r / nq_all;
         return lens[b] - a.T + (r - b * nq_all) / kG;
       };
       if (active && pkind == kPageLoad) {
         const uint32_t dcol = (uint32_t)(x * kBlock);
         if constexpr (M == 64) {
-          // 16x256b: thread (g, t) holds rows g and g+8 of the quarter, columns 8c+2t, 8c+2t+1
+          // 16x256b: thread (g, t) holds rows g and g+8 of the quarter, columns
+          // 8c+2t, 8c+2t+1 (spread: the rows g+8 hold no query)
           const int g = lane >> 2, t = lane & 3;
           float m0 = -INFINITY, m1 = -INFINITY;
-          const int qa0 = rbase + g, qa1 = qa0 + 8;
-          const int lim0 = need_mask ? last_key(qa0) : 0, lim1 = need_mask ? last_key(qa1) : 0;
+          const int qa0 = rbase + g, qa1 = spread ? 0x7FFFFFFF : qa0 + 8;
+          const int lim0 = need_mask ? last_key(qa0) : 0, lim1 = (need_mask && !spread) ? last_key(qa1) : 0;
 #pragma unroll 1
           for (int h = 0; h < 2; ++h) {                // columns 64h .. 64h+63
             float v[32];
@@ -520,12 +562,14 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
               r1[2 * c] = v[4 * c + 2]; r1[2 * c + 1] = v[4 * c + 3];
             }
             m0 = fmaxf(m0, max_of<16>(r0));
-            m1 = fmaxf(m1, max_of<16>(r1));
+            if (!spread) m1 = fmaxf(m1, max_of<16>(r1));
           }
           m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
           m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+          if (!spread) {
+            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+          }
           if (t < 2) {
             const int qa = t == 0 ? qa0 : qa1;
             if (qa < prow1) a.block_scores[(long long)qa * a.max_pages + pi] = (t == 0 ? m0 : m1) * a.score_scale;
@@ -575,9 +619,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     const int half = d >> 7;                        // elements 64*half .. 64*half+63
     const int sw = (row >> 1) & 3;                  // 64-byte swizzle of the code rows
     int cur_row0 = -1;
+    int s = 0;                                      // stage of page k
+    uint32_t sph = 0;                               // its phase parity
     for (int k = 0;; ++k) {
-      const int s = k % S;
-      if (!mbar_wait(&raw_full[s], (k / S) & 1)) { report(a.flags, 5, 5); break; }
+      if (!mbar_wait(&raw_full[s], sph)) { report(a.flags, 5, 5); break; }
       // page k-2 consumed by the MMA: its B buffer (k % 2) and the page-ready
       // barrier k % 2 are free, and every MMA of pages <= k-2 has completed
       if (k >= 2 && !mbar_wait(&b_empty[k & 1], ((k >> 1) - 1) & 1)) {
@@ -585,11 +630,13 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         break;
       }
       const int* m = meta + 8 * s;
-      const int nrowp = m[0], ni = m[1], nkind = m[2], nr0 = m[3], nr1 = m[4], nminpos = m[5];
-      if (nkind != kPageEnd && nr0 != cur_row0) {
-        // A operand: the index-query rows [nr0, nr1) of the tile (rows of qi),
-        // K-major with the 128-byte swizzle, zero rows past nr1.  The previous
-        // tile's last MMA (page k-1 at the latest) must be done.
+      const int nkind = m[2];
+      if (F16 && nkind != kPageEnd && m[3] != cur_row0) {
+        const int nr0 = m[3], nr1 = m[4];
+        // FP16 A operand: the index-query rows [nr0, nr1) of the tile widened
+        // to FP16, K-major, two 128-byte-swizzled K-halves, zero rows past
+        // nr1.  The previous tile's last MMA (page k-1 at the latest) must be
+        // done.  (E4M3 tiles are loaded by the producer's TMA.)
         if (k >= 1 && !mbar_wait(&b_empty[(k - 1) & 1], ((k - 1) >> 1) & 1)) {
           report(a.flags, 5, 7);
           break;
@@ -600,20 +647,16 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           const int qg = nr0 + nrow;
           uint4 v = make_uint4(0u, 0u, 0u, 0u);
           if (qg < nr1) v = *reinterpret_cast<const uint4*>(a.qi + (long long)qg * kDim + 16 * c);
-          if constexpr (F16) {
-            // dims 16c..16c+15 -> FP16 chunks 2c, 2c+1 of 8 dims: K-half c / 4,
-            // chunk positions (2c % 8, 2c % 8 + 1) ^ (row % 8) in its 128-byte row
-            const uint4 lo = make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
-                                        e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
-            const uint4 hi = make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
-                                        e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
-            uint8_t* rowp = qbuf + (c >> 2) * M * 128 + nrow * 128;
-            const int jj = (2 * c) & 7;
-            sts128(rowp + ((jj ^ (nrow & 7)) << 4), lo);
-            sts128(rowp + (((jj + 1) ^ (nrow & 7)) << 4), hi);
-          } else {
-            sts128(qbuf + nrow * 128 + ((c ^ (nrow & 7)) << 4), v);
-          }
+          // dims 16c..16c+15 -> FP16 chunks 2c, 2c+1 of 8 dims: K-half c / 4,
+          // chunk positions (2c % 8, 2c % 8 + 1) ^ (row % 8) in its 128-byte row
+          const uint4 lo = make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
+                                      e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
+          const uint4 hi = make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
+                                      e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
+          uint8_t* rowp = qbuf + (c >> 2) * M * 128 + nrow * 128;
+          const int jj = (2 * c) & 7;
+          sts128(rowp + ((jj ^ (nrow & 7)) << 4), lo);
+          sts128(rowp + (((jj + 1) ^ (nrow & 7)) << 4), hi);
         }
       }
       if (!FP8 && nkind == kPageLoad) {
@@ -676,14 +719,17 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       fence_async_smem();   // generic-proxy writes (queries, keys) -> the MMA
       __syncwarp();
       if (lane == 0) {
-        if (warp == 0) {
-          int* pf = pinfo + 8 * (k % kInfoRing);
-          pf[0] = nrowp; pf[1] = ni; pf[2] = nkind; pf[3] = nr0; pf[4] = nr1; pf[5] = nminpos;
+        if (warp == 0) {   // the page's info, for the MMA and the epilogue
+          const int4* src = reinterpret_cast<const int4*>(m);
+          int4* dst = reinterpret_cast<int4*>(pinfo + 8 * (k % kInfoRing));
+          dst[0] = src[0];
+          dst[1] = src[1];
         }
         if (!FP8) mbar_arrive(&raw_empty[s]);
         mbar_arrive(&b_full[k & 1]);
       }
       if (nkind == kPageEnd) break;
+      if (++s == S) { s = 0; sph ^= 1u; }
     }
   }
 

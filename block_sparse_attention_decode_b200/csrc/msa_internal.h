@@ -4,12 +4,33 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "msa_device.cuh"
 
 namespace msa {
+
+// Launch `kernel` with programmatic stream serialisation: it may start while
+// the previous kernel on the stream is finishing (its launch and prologue
+// overlap that kernel's last CTAs).  The kernel calls grid_dependency_wait()
+// before it touches global memory the previous work writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr int kIdxThreads = 14 * 32;    // 8 decoders, 4 epilogue warps, producer, MMA warp
 // Indexer arithmetic: NVFP4 keys re-rounded to E4M3 (FP8 MMA), E4M3 keys, or
@@ -18,6 +39,7 @@ enum : int { kIdxNvfp4 = 0, kIdxFp8 = 1, kIdxF16 = 2 };
 
 struct IdxArgs {
   CUtensorMap tmap_idx;        // rows of idx_data: 64-byte rows (64B swizzle) or 128 (128B swizzle)
+  CUtensorMap tmap_qi;         // rows of qi (128 bytes, 128B swizzle), boxes of one query tile
   const uint8_t* idx_data;     // NVFP4 codes [P][128][64] or FP8 keys [P][128][128]
   const uint8_t* idx_scale;    // [P][128][8] (NVFP4 keys only)
   const int32_t* page_table;   // [B][max_pages] or null
@@ -40,10 +62,15 @@ struct IdxArgs {
   const int32_t* grp_prefix;
   int ngroups;
   int shared;
+  // 64-row tiles of at most 32 query rows (E4M3 query modes): tile row r sits
+  // at MMA row 16 (r / 8) + r % 8, so that each TMEM lane quarter holds eight
+  // rows and all four epilogue warps share the work; tmap_qi has 8-row boxes
+  int spread;
 };
 
 size_t indexer_smem_bytes(int mode, int batch, int T);
 int idx_tile_queries(int T);   // index queries per tile (the MMA's M side): 64 or 128
+bool idx_spread_rows(int T, int mode, int shared);   // the `spread` placement above
 cudaError_t launch_indexer(const IdxArgs& a, int mode, cudaStream_t st);
 
 // Grid of a persistent kernel on the current device: the device's SMs times
@@ -66,8 +93,8 @@ cudaError_t launch_topk(const float* block_scores, const int32_t* seq_lens, int 
 cudaError_t launch_maxpool(const float* token_scores, const int32_t* seq_lens, int B, int T,
                            int max_pages, float* block_scores, Flags* flags, cudaStream_t st);
 
-constexpr int kAttThreads = 14 * 32;    // 8 decoders, 4 softmax warps, producer, MMA warp
-constexpr int kAttStages = 3;            // raw K/V blocks in flight per CTA
+constexpr int kAttThreads = 14 * 32;    // 4 decoders, 8 softmax warps, producer, MMA warp
+constexpr int kAttStages = 2;            // raw K/V blocks in flight per CTA
 constexpr int kAttWorkOffset = 72;       // int[2] in the workspace header (see kWorkOffset)
 constexpr int kPartialFloats = kHpg * kDim + 2 * kHpg;   // O[16][128], m[16], l[16]
 

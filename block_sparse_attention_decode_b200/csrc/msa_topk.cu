@@ -42,6 +42,8 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_le
   __shared__ unsigned cand_key_all[kTopkRows][kTopkCand];
   __shared__ int cand_id_all[kTopkRows][kTopkCand];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  grid_dependency_wait();   // launched with programmatic serialisation: scores ready
+  grid_launch_dependents(); // the attention may start its prologue
   const long long row = (long long)blockIdx.x * kTopkRows + w;   // (b * T + t) * 4 + g
   if (row >= (long long)B * T * kG) return;
   unsigned* keys = keys_all[w];
@@ -65,11 +67,24 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_le
   const int n = nb - 1;                      // candidates 0 .. nb-2
   const bool cached = n <= kTopkCache;
   unsigned kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int i = lane; i < n; i += 32) {
-    const unsigned k = score_key(S[i]);
-    if (cached) keys[i] = k;
-    kmin = min(kmin, k);
-    kmax = max(kmax, k);
+  // 16 loads in flight per lane (the scores come from L2 or HBM)
+  for (int base = 0; base < n; base += 16 * 32) {
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int i = base + 32 * j + lane;
+      v[j] = i < n ? __ldcg(S + i) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int i = base + 32 * j + lane;
+      if (i < n) {
+        const unsigned k = score_key(v[j]);
+        if (cached) keys[i] = k;
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+    }
   }
   __syncwarp();
   auto key_at = [&](int i) -> unsigned { return cached ? keys[i] : score_key(S[i]); };
@@ -234,9 +249,8 @@ cudaError_t launch_topk(const float* block_scores, const int32_t* seq_lens, int 
   const long long rows = (long long)B * T * kG;
   if (rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   const long long ctas = (rows + kTopkRows - 1) / kTopkRows;
-  topk_kernel<<<(unsigned)ctas, kTopkThreads, 0, st>>>(block_scores, seq_lens, B, T, max_pages,
-                                                       sel, flags);
-  return cudaGetLastError();
+  return launch_dependent(topk_kernel, dim3((unsigned)ctas), dim3(kTopkThreads), 0, st, block_scores,
+                          seq_lens, B, T, max_pages, sel, flags);
 }
 
 cudaError_t launch_maxpool(const float* token_scores, const int32_t* seq_lens, int B, int T,
