@@ -292,9 +292,9 @@ def cpu_baseline(name: str, budget_s: float = 20.0):
 
 
 # --------------------------------------------------------- sub-records --
-def timed(fn, steps, flush, stream):
-    """Median CUDA-event time (ms) of fn over `steps` runs, L2 flushed before
-    each (outside the events), after 3 untimed runs."""
+def timed(fn, steps, flush, stream, mean=False):
+    """Median (or mean) CUDA-event time (ms) of fn over `steps` runs, L2
+    flushed before each (outside the events), after 3 untimed runs."""
     import torch
     for _ in range(3):
         fn()
@@ -307,7 +307,7 @@ def timed(fn, steps, flush, stream):
         e1.record(stream)
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1))
-    return statistics.median(ts)
+    return statistics.mean(ts) if mean else statistics.median(ts)
 
 
 def prefill_record(steps, flush, stream):
@@ -459,22 +459,18 @@ def run_gpu(args, rank, world, local_rank):
     ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
     ms_max = max_over_ranks(ms, world)
 
-    # ---- per-kernel times (the same kernels through the stage entry points)
+    # ---- per-kernel times: each stage entry point timed on its own (L2
+    # flushed before each launch, outside the events), so that no kernel's
+    # time includes a neighbour's tail overlapped by programmatic launch
     names = ("indexer", "topk", "attention")
-    per = {k: 0.0 for k in names}
-    for _ in range(args.steps):
-        flush.fill_(1)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        e[0].record(stream)
-        msa.msa_indexer_score(cache, seqs, w.qi, w.s_qi, None, bscores, ws, stream)
-        e[1].record(stream)
-        msa.msa_block_maxpool_topk(bscores, False, seqs, sel, ws, stream)
-        e[2].record(stream)
-        msa.msa_sparse_attn_decode(cache, seqs, w.q, w.s_q, sel, w.softmax_scale, out, ws, stream)
-        e[3].record(stream)
-        torch.cuda.synchronize()
-        for i, k in enumerate(names):
-            per[k] += e[i].elapsed_time(e[i + 1]) / args.steps
+    per = {
+        "indexer": timed(lambda: msa.msa_indexer_score(cache, seqs, w.qi, w.s_qi, None, bscores, ws, stream),
+                         args.steps, flush, stream, mean=True),
+        "topk": timed(lambda: msa.msa_block_maxpool_topk(bscores, False, seqs, sel, ws, stream),
+                      args.steps, flush, stream, mean=True),
+        "attention": timed(lambda: msa.msa_sparse_attn_decode(cache, seqs, w.q, w.s_q, sel, w.softmax_scale,
+                                                              out, ws, stream), args.steps, flush, stream, mean=True),
+    }
     st, detail = msa.msa_get_last_error(ws)
     if st != msa.MSA_OK:
         raise RuntimeError("device error %d (%d) during timing" % (st, detail))

@@ -23,24 +23,25 @@
 // the last CTA to finish resets the counter.  Warp roles, a few pages apart:
 //   warp 12 (producer): the whole warp looks up the pages of the next work
 //     item (one lane per page: sequence, logical block, page table entry)
-//     while lane 0 issues the current item's pages: per page one tiled TMA
-//     load of the codes (64-byte
-//     swizzle, so that row-per-thread reads are bank-conflict free) and one
-//     bulk copy of the scales into a ring of shared-memory stages (FP8 index
-//     keys: one TMA load with the 128-byte swizzle, which is already the
-//     MMA's B operand);
-//   warps 0-7 (decoders): thread = half a key row (warps 0-3 elements 0-63,
-//     warps 4-7 elements 64-127).  NVFP4 is decoded to signed E4M3 (dq8: a
-//     table row per scale byte, byte permutes for magnitudes and signs) and
-//     stored as 128-byte rows with the 128-byte swizzle -- the K-major B
-//     operand -- into one of two buffers, so page k+1 is decoded while page
-//     k's MMAs run.  When the query tile changes they stage the tile's index
-//     queries (the A operand), after the MMAs of the previous tile are done;
+//     and issues the current item's pages, lane j page j, as their stages
+//     free: per page one tiled TMA load of the codes (64-byte swizzle, so
+//     that row-per-thread reads are bank-conflict free) and one bulk copy of
+//     the scales into a ring of shared-memory stages (FP8 index keys: one TMA
+//     load with the 128-byte swizzle, which is already the MMA's B operand);
+//     and, per item, the TMA load of the item's index-query tile;
+//   warps 0-3 (decoders): thread = key row.  NVFP4 is decoded to signed E4M3
+//     (dq8: a table row per scale byte, byte permutes for magnitudes and
+//     signs) and stored as 128-byte rows with the 128-byte swizzle -- the
+//     K-major B operand -- into one of two buffers, so page k+1 is decoded
+//     while page k's MMAs run (FP16 mode: they also stage the tile's index
+//     queries, the A operand, when the tile changes);
 //   warp 13 (MMA): one thread issues per page 4 tcgen05.mma of K = 32 (E4M3;
-//     8 of K = 16 for FP16) into one of two TMEM accumulators;
-//   warps 8-11 (epilogue): warp 8+q reads the accumulator lanes of quarter q,
-//     masks keys after each query's position, takes each query's maximum
-//     over the page's keys and writes the block score.
+//     8 of K = 16 for FP16) into TMEM accumulator k % 2;
+//   warps 4-11 (epilogue): warp w reads the accumulator lanes of quarter
+//     w % 4 for the pages of parity (w - 4) / 4, so that two pages are read
+//     out at once; it masks keys after each query's position, takes each
+//     query's maximum over the page's keys and writes the block score.  The
+//     producer ends the page stream with two end markers, one per parity.
 // Every wait is a bounded mbarrier wait; on a timeout a thread records
 // MSA_ERR_TIMEOUT and leaves its loop, and TMEM is freed before exit.
 //
@@ -56,8 +57,8 @@
 
 namespace msa {
 
-constexpr int kIdxDecWarps = 8;             // warps 0-7: half a key row per thread
-constexpr int kIdxEpiWarp0 = 8;             // warps 8-11: one per TMEM lane quarter
+constexpr int kIdxDecWarps = 4;             // warps 0-3: one key row per thread
+constexpr int kIdxEpiWarp0 = 4;             // warps 4-11: lane quarter warp % 4, pages of parity (warp - 4) / 4
 constexpr int kIdxProducerWarp = 12;
 constexpr int kIdxMmaWarp = 13;
 static_assert(kIdxThreads == 14 * 32, "warp roles");
@@ -411,40 +412,56 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         }
       }
       ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
-      for (int j = 0; j < cur.np && ok; ++j, ++k) {
-        const int ij = __shfl_sync(0xffffffffu, cur.i, j);
-        const int kj = __shfl_sync(0xffffffffu, cur.kind, j);
-        const long long pj = __shfl_sync(0xffffffffu, cur.p, j);
-        if (lane == 0) {
-          if (!slot(k)) {
-            report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1);
-            ok = false;
+      // The item's pages, lane j: page j, stage (k + j) % S, issued in passes.
+      // Stages are freed in page order (the decoders release them in order),
+      // so the free stages of the pending pages are a prefix: each pass
+      // issues that prefix at once, or waits for the first pending page's
+      // stage when it is empty.  A lane only tests its stage once the page S
+      // before it has been issued, so no barrier it reads is two phases behind.
+      for (int jn = 0; jn < cur.np && ok;) {
+        const int jend = min(cur.np, jn + S);
+        const int kk = k + lane;                    // this lane's page slot
+        const bool mine = lane >= jn && lane < jend;
+        const bool fr = mine && (kk < S || mbar_test(&raw_empty[kk % S], ((kk / S) - 1) & 1));
+        const unsigned pend = (jend >= 32 ? 0xffffffffu : (1u << jend) - 1u) & ~((1u << jn) - 1u);
+        const unsigned busy = pend & ~__ballot_sync(0xffffffffu, fr);
+        const int jx = busy ? __ffs(busy) - 1 : jend;   // pages [jn, jx) have free stages
+        if (lane >= jn && lane < jx) {
+          const int s = kk % S;
+          int4* m4 = reinterpret_cast<int4*>(meta + 8 * s);
+          m4[0] = make_int4(cur.ptrow, cur.i, cur.kind, cur.row0);
+          m4[1] = make_int4(cur.row1, cur.minpos, ki, (lane == 0) | ((lane == cur.np - 1) << 1));
+          uint8_t* dst = raw + s * C::kRawStride;
+          if (cur.kind == kPageLoad) {
+            mbar_expect_tx(&raw_full[s], C::kRaw);
+            tma_load_2d(dst, &a.tmap_idx, 0, (int)(cur.p * kBlock), &raw_full[s]);
+            if (!FP8) bulk_g2s(dst + kPageCodes, a.idx_scale + cur.p * kPageScales, kPageScales, &raw_full[s]);
           } else {
-            const int s = k % S;
-            int* m = meta + 8 * s;
-            m[0] = cur.ptrow; m[1] = ij; m[2] = kj; m[3] = cur.row0; m[4] = cur.row1; m[5] = cur.minpos;
-            m[6] = ki; m[7] = (j == 0) | ((j == cur.np - 1) << 1);   // first / last page of the item
-            uint8_t* dst = raw + s * C::kRawStride;
-            if (kj == kPageLoad) {
-              mbar_expect_tx(&raw_full[s], C::kRaw);
-              tma_load_2d(dst, &a.tmap_idx, 0, (int)(pj * kBlock), &raw_full[s]);
-              if (!FP8) bulk_g2s(dst + kPageCodes, a.idx_scale + pj * kPageScales, kPageScales, &raw_full[s]);
-            } else {
-              mbar_arrive(&raw_full[s]);
-            }
+            mbar_arrive(&raw_full[s]);
           }
         }
-        ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+        if (jx == jn) {   // no free stage: wait for page jn's (its slot is >= S)
+          bool good = true;
+          if (lane == jn) good = mbar_wait(&raw_empty[kk % S], ((kk / S) - 1) & 1);
+          if (!__shfl_sync(0xffffffffu, (int)good, jn)) {
+            if (lane == 0) report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1);
+            ok = false;
+          }
+        }
+        jn = jx;
       }
+      k += cur.np;
       cur = next;
       item = nxt;
       nxt = claim;                                  // lane 0's value, broadcast next time
       ++ki;
     }
     if (lane == 0) {
-      if (ok) {   // end marker
+      // two end markers, one for each of the epilogue's two page parities
+      for (int e = 0; e < 2 && ok; ++e, ++k) {
         if (!slot(k)) {
           report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 1);
+          ok = false;
         } else {
           meta[8 * (k % S) + 2] = kPageEnd;
           mbar_arrive(&raw_full[k % S]);
@@ -461,6 +478,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idx_idesc<M>();
+      int nend = 0;
       for (int k = 0;; ++k) {
         const int x = k & 1;                       // accumulator and page-ready barrier
         if (!mbar_wait(&b_full[x], (k >> 1) & 1)) { report(a.flags, 5, 2); break; }
@@ -492,7 +510,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           }
         }
         tc_commit(&d_full[x]);
-        if (kind == kPageEnd) break;
+        if (kind == kPageEnd) {
+          if (++nend == 2) break;
+          continue;
+        }
         if (FP8) tc_commit(&raw_empty[k % S]);   // the stage was the B operand
         tc_commit(&b_empty[x]);                   // page k consumed (and its B buffer free)
         if (!F16 && (flg & 2)) tc_commit(&q_empty[qx]);   // the item's query tile is free
@@ -500,14 +521,15 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     }
   } else if (warp >= kIdxEpiWarp0) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp - kIdxEpiWarp0;             // TMEM lane quarter
+    const int q = warp & 3;                         // TMEM lane quarter
+    const int par = (warp - kIdxEpiWarp0) >> 2;     // pages k with k % 2 == par (accumulator par)
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     // rows of the tile this warp reads: M = 64: 16q..16q+15 (spread: 8q..8q+7);
     // M = 128: 32q..32q+31
     const bool spread = M == 64 && a.spread;
     const int kRows = M == 64 ? (spread ? 8 : 16) : 32;
-    for (int k = 0;; ++k) {
-      const int x = k & 1;
+    for (int k = par;; k += 2) {
+      const int x = par;
       if (!mbar_wait(&d_full[x], (k >> 1) & 1)) { report(a.flags, 5, 6); break; }
       tc_fence_after();
       const int* pf = pinfo + 8 * (k % kInfoRing);
@@ -614,10 +636,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     }
   } else {
     // ------------------------------------------------------------ decoders
-    const int d = 32 * warp + lane;                 // 0 .. 255
-    const int row = d & (kBlock - 1);               // key row of this thread
-    const int half = d >> 7;                        // elements 64*half .. 64*half+63
+    const int d = 32 * warp + lane;                 // 0 .. 127
+    const int row = d;                              // key row of this thread
     const int sw = (row >> 1) & 3;                  // 64-byte swizzle of the code rows
+    int nend = 0;
     int cur_row0 = -1;
     int s = 0;                                      // stage of page k
     uint32_t sph = 0;                               // its phase parity
@@ -664,56 +686,60 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         uint8_t* bb = bbuf + (k & 1) * C::kBBytes;
         // 64-byte code rows loaded with the 64-byte swizzle: chunk c of row r
         // sits at chunk position c ^ ((r / 2) % 4); chunk c = elements
-        // 32c..32c+31 under scale bytes 2c and 2c+1.  This thread: chunks
-        // 2*half and 2*half+1, scale bytes 4*half .. 4*half+3.
-        const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(rs + kPageCodes + row * kRowScales + 4 * half);
-        if constexpr (F16) {
-          // FP16 key row: 256 bytes as two 128-byte K-halves (rows 128 apart),
-          // each with the 128-byte swizzle; chunk c -> 16-byte chunks 4(c%2)..
-          // of K-half c / 2 (= half)
-          uint8_t* rowp = bb + half * kBlock * 128 + row * 128;
+        // 32c..32c+31 under scale bytes 2c and 2c+1.  This thread: the whole
+        // row, as two halves (chunks 2h, 2h+1 under scale bytes 4h..4h+3).
+        const uint2 sc8 = *reinterpret_cast<const uint2*>(rs + kPageCodes + row * kRowScales);
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
-            const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
-            const uint32_t s2 = e4m3x2_to_f16x2(sc4 >> (16 * cc));
-            const uint32_t s_lo = prmt(s2, 0u, 0x1010u), s_hi = prmt(s2, 0u, 0x3232u);
-            uint32_t o[16];
-            e2m1x8_to_f16x2(w4.x, o + 0);
-            e2m1x8_to_f16x2(w4.y, o + 4);
-            e2m1x8_to_f16x2(w4.z, o + 8);
-            e2m1x8_to_f16x2(w4.w, o + 12);
-#pragma unroll
-            for (int mm = 0; mm < 16; ++mm) o[mm] = hmul2(o[mm], mm < 8 ? s_lo : s_hi);
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              const int ch = 4 * cc + jj;
-              sts128(rowp + ((ch ^ (row & 7)) << 4),
-                     make_uint4(o[4 * jj], o[4 * jj + 1], o[4 * jj + 2], o[4 * jj + 3]));
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t sc4 = half ? sc8.y : sc8.x;
+          if constexpr (F16) {
+            // FP16 key row: 256 bytes as two 128-byte K-halves (rows 128 apart),
+            // each with the 128-byte swizzle; chunk c -> 16-byte chunks 4(c%2)..
+            // of K-half c / 2 (= half)
+            uint8_t* rowp = bb + half * kBlock * 128 + row * 128;
+  #pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const int c = 2 * half + cc;
+              const uint4 w4 = lds128(rs + row * kRowCodes + ((c ^ sw) << 4));
+              const uint32_t s2 = e4m3x2_to_f16x2(sc4 >> (16 * cc));
+              const uint32_t s_lo = prmt(s2, 0u, 0x1010u), s_hi = prmt(s2, 0u, 0x3232u);
+              uint32_t o[16];
+              e2m1x8_to_f16x2(w4.x, o + 0);
+              e2m1x8_to_f16x2(w4.y, o + 4);
+              e2m1x8_to_f16x2(w4.z, o + 8);
+              e2m1x8_to_f16x2(w4.w, o + 12);
+  #pragma unroll
+              for (int mm = 0; mm < 16; ++mm) o[mm] = hmul2(o[mm], mm < 8 ? s_lo : s_hi);
+  #pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                const int ch = 4 * cc + jj;
+                sts128(rowp + ((ch ^ (row & 7)) << 4),
+                       make_uint4(o[4 * jj], o[4 * jj + 1], o[4 * jj + 2], o[4 * jj + 3]));
+              }
             }
+          } else {
+            // E4M3 key row: 128 bytes with the 128-byte swizzle; code chunk c ->
+            // row chunks 2c, 2c+1
+            uint8_t* rowp = bb + row * 128;
+            const uint4 w0 = lds128(rs + row * kRowCodes + (((2 * half) ^ sw) << 4));
+            const uint4 w1 = lds128(rs + row * kRowCodes + (((2 * half + 1) ^ sw) << 4));
+            const uint2 r0 = lut[sc4 & 0xFFu], r1 = lut[(sc4 >> 8) & 0xFFu];
+            const uint2 r2 = lut[(sc4 >> 16) & 0xFFu], r3 = lut[sc4 >> 24];
+            uint32_t o[16];
+            dq8(w0.x, r0, o[0], o[1]);
+            dq8(w0.y, r0, o[2], o[3]);
+            dq8(w0.z, r1, o[4], o[5]);
+            dq8(w0.w, r1, o[6], o[7]);
+            dq8(w1.x, r2, o[8], o[9]);
+            dq8(w1.y, r2, o[10], o[11]);
+            dq8(w1.z, r3, o[12], o[13]);
+            dq8(w1.w, r3, o[14], o[15]);
+            const int c0 = 4 * half;                   // first of this thread's 4 row chunks
+  #pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+              sts128(rowp + (((c0 + jj) ^ (row & 7)) << 4),
+                     make_uint4(o[4 * jj], o[4 * jj + 1], o[4 * jj + 2], o[4 * jj + 3]));
           }
-        } else {
-          // E4M3 key row: 128 bytes with the 128-byte swizzle; code chunk c ->
-          // row chunks 2c, 2c+1
-          uint8_t* rowp = bb + row * 128;
-          const uint4 w0 = lds128(rs + row * kRowCodes + (((2 * half) ^ sw) << 4));
-          const uint4 w1 = lds128(rs + row * kRowCodes + (((2 * half + 1) ^ sw) << 4));
-          const uint2 r0 = lut[sc4 & 0xFFu], r1 = lut[(sc4 >> 8) & 0xFFu];
-          const uint2 r2 = lut[(sc4 >> 16) & 0xFFu], r3 = lut[sc4 >> 24];
-          uint32_t o[16];
-          dq8(w0.x, r0, o[0], o[1]);
-          dq8(w0.y, r0, o[2], o[3]);
-          dq8(w0.z, r1, o[4], o[5]);
-          dq8(w0.w, r1, o[6], o[7]);
-          dq8(w1.x, r2, o[8], o[9]);
-          dq8(w1.y, r2, o[10], o[11]);
-          dq8(w1.z, r3, o[12], o[13]);
-          dq8(w1.w, r3, o[14], o[15]);
-          const int c0 = 4 * half;                   // first of this thread's 4 row chunks
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-            sts128(rowp + (((c0 + jj) ^ (row & 7)) << 4),
-                   make_uint4(o[4 * jj], o[4 * jj + 1], o[4 * jj + 2], o[4 * jj + 3]));
         }
       }
       fence_async_smem();   // generic-proxy writes (queries, keys) -> the MMA
@@ -728,7 +754,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         if (!FP8) mbar_arrive(&raw_empty[s]);
         mbar_arrive(&b_full[k & 1]);
       }
-      if (nkind == kPageEnd) break;
+      if (nkind == kPageEnd && ++nend == 2) break;
       if (++s == S) { s = 0; sph ^= 1u; }
     }
   }
