@@ -32,9 +32,9 @@
 //   warps 0-3 (decoders): thread = key row.  NVFP4 is decoded to signed E4M3
 //     (dq8: a table row per scale byte, byte permutes for magnitudes and
 //     signs) and stored as 128-byte rows with the 128-byte swizzle -- the
-//     K-major B operand -- into one of two buffers, so page k+1 is decoded
-//     while page k's MMAs run (FP16 mode: they also stage the tile's index
-//     queries, the A operand, when the tile changes);
+//     K-major B operand -- into one of two buffers, so that page k+1 is
+//     decoded while page k's MMAs run (FP16 mode: they also stage the
+//     tile's index queries, the A operand, when the tile changes);
 //   warp 13 (MMA): one thread issues per page 4 tcgen05.mma of K = 32 (E4M3;
 //     8 of K = 16 for FP16) into TMEM accumulator k % 2;
 //   warps 4-11 (epilogue): warp w reads the accumulator lanes of quarter
@@ -76,7 +76,8 @@ struct IdxCfg {
   static constexpr int kRaw = kFp8 ? kBlock * kDim : kPageCodes + kPageScales;
   static constexpr int kRawStride = (kRaw + 1023) / 1024 * 1024;
   static constexpr int kStages = kF16 ? 3 : 6;             // raw pages in flight
-  static constexpr int kNB = kFp8 ? 0 : 2;                 // decoded key pages (B operand), page k in k % 2
+  static constexpr int kNB = kFp8 ? 0 : 2;                 // decoded key pages (B operand), page k in k % kNB
+  static constexpr int kBR = kFp8 ? 2 : kNB;               // page-ready barriers (FP8: the raw stage is B)
   static constexpr int kBBytes = kBlock * kRow;
 };
 
@@ -93,7 +94,7 @@ __host__ __device__ inline IdxLayout idx_layout(int batch) {
   L.raw = off;     off += C::kStages * C::kRawStride;
   L.bbuf = off;    off += C::kNB * C::kBBytes;
   L.lut = off;     off += MODE == kIdxNvfp4 ? 256 * 8 : 0;
-  L.bars = off;    off += (2 * C::kStages + 12) * 8;
+  L.bars = off;    off += (2 * C::kStages + 2 * C::kBR + 8) * 8;
   L.meta = off;    off += C::kStages * 8 * 4;              // per stage: ptrow, i, kind, row0, row1, minpos
   L.pinfo = off;   off += kInfoRing * 8 * 4;               // per page: the same
   L.tslot = off;   off += 16;
@@ -236,10 +237,20 @@ __device__ int build_items(const IdxArgs& a, int* prefix, int* lens, int* skip, 
   for (int e = lo; e < hi; ++e) sum += entity_items<M>(entity(a, e, tb));
   scratch[tid] = sum;
   __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int k = 0; k < nt; ++k) { const int v = scratch[k]; scratch[k] = run; run += v; }
-    prefix[E] = run;
+  if (tid < 32) {   // exclusive scan of the per-thread counts: lane l owns a run of them
+    const int per_lane = (nt + 31) / 32;
+    const int k0 = tid * per_lane, k1 = min(nt, k0 + per_lane);
+    int own = 0;
+    for (int k = k0; k < k1; ++k) own += scratch[k];
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += v;
+    }
+    int run = incl - own;
+    for (int k = k0; k < k1; ++k) { const int v = scratch[k]; scratch[k] = run; run += v; }
+    if (tid == 31) prefix[E] = incl;
   }
   __syncthreads();
   int run = scratch[tid];
@@ -273,9 +284,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
   uint2* lut = reinterpret_cast<uint2*>(smem + Ly.lut);
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + Ly.bars);
   uint64_t* raw_empty = raw_full + S;
-  uint64_t* b_full = raw_empty + S;      // [2] decoders -> MMA: page k ready (k % 2)
-  uint64_t* b_empty = b_full + 2;        // [2] MMA -> decoders: page k consumed
-  uint64_t* d_full = b_empty + 2;        // [2] MMA -> epilogue
+  constexpr int BR = C::kBR;
+  uint64_t* b_full = raw_empty + S;      // [BR] decoders -> MMA: page k ready (k % BR)
+  uint64_t* b_empty = b_full + BR;       // [BR] MMA -> decoders: page k consumed
+  uint64_t* d_full = b_empty + BR;       // [2] MMA -> epilogue
   uint64_t* d_empty = d_full + 2;        // [2] epilogue -> MMA
   uint64_t* q_full = d_empty + 2;        // [2] producer (TMA) -> MMA: an item's query tile
   uint64_t* q_empty = q_full + 2;        // [2] MMA -> producer: the item's last MMA done
@@ -298,9 +310,11 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       mbar_init(&raw_full[s], 1);
       mbar_init(&raw_empty[s], FP8 ? 1 : kIdxDecWarps);   // FP8: released by the MMA
     }
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < BR; ++x) {
       mbar_init(&b_full[x], kIdxDecWarps);
       mbar_init(&b_empty[x], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
       mbar_init(&d_full[x], 1);
       mbar_init(&d_empty[x], 4);
       mbar_init(&q_full[x], 1);
@@ -481,7 +495,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       int nend = 0;
       for (int k = 0;; ++k) {
         const int x = k & 1;                       // accumulator and page-ready barrier
-        if (!mbar_wait(&b_full[x], (k >> 1) & 1)) { report(a.flags, 5, 2); break; }
+        if (!mbar_wait(&b_full[k % BR], (k / BR) & 1)) { report(a.flags, 5, 2); break; }
         if (k >= 2 && !mbar_wait(&d_empty[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 3); break; }
         tc_fence_after();
         const int* pf = pinfo + 8 * (k % kInfoRing);
@@ -496,7 +510,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           const uint32_t d = tmem + (uint32_t)(x * kBlock);
           const uint32_t qa = smem_u32(qbuf + qx * M * 128);
           const uint32_t kb = FP8 ? smem_u32(raw + (k % S) * C::kRawStride)
-                                  : smem_u32(bbuf + x * C::kBBytes);
+                                  : smem_u32(bbuf + (k % BR) * C::kBBytes);
           if constexpr (F16) {
             // K-half h of the queries starts M rows further, of the keys 128 rows further
 #pragma unroll
@@ -515,7 +529,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           continue;
         }
         if (FP8) tc_commit(&raw_empty[k % S]);   // the stage was the B operand
-        tc_commit(&b_empty[x]);                   // page k consumed (and its B buffer free)
+        tc_commit(&b_empty[k % BR]);              // page k consumed (and its B buffer free)
         if (!F16 && (flg & 2)) tc_commit(&q_empty[qx]);   // the item's query tile is free
       }
     }
@@ -645,9 +659,9 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
     uint32_t sph = 0;                               // its phase parity
     for (int k = 0;; ++k) {
       if (!mbar_wait(&raw_full[s], sph)) { report(a.flags, 5, 5); break; }
-      // page k-2 consumed by the MMA: its B buffer (k % 2) and the page-ready
-      // barrier k % 2 are free, and every MMA of pages <= k-2 has completed
-      if (k >= 2 && !mbar_wait(&b_empty[k & 1], ((k >> 1) - 1) & 1)) {
+      // page k-BR consumed by the MMA: its B buffer and page-ready barrier
+      // (k % BR) are free, and every MMA of pages <= k-BR has completed
+      if (k >= BR && !mbar_wait(&b_empty[k % BR], ((k / BR) - 1) & 1)) {
         report(a.flags, 5, 4);
         break;
       }
@@ -659,7 +673,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
         // to FP16, K-major, two 128-byte-swizzled K-halves, zero rows past
         // nr1.  The previous tile's last MMA (page k-1 at the latest) must be
         // done.  (E4M3 tiles are loaded by the producer's TMA.)
-        if (k >= 1 && !mbar_wait(&b_empty[(k - 1) & 1], ((k - 1) >> 1) & 1)) {
+        if (k >= 1 && !mbar_wait(&b_empty[(k - 1) % BR], ((k - 1) / BR) & 1)) {
           report(a.flags, 5, 7);
           break;
         }
@@ -683,7 +697,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
       }
       if (!FP8 && nkind == kPageLoad) {
         const uint8_t* rs = raw + s * C::kRawStride;
-        uint8_t* bb = bbuf + (k & 1) * C::kBBytes;
+        uint8_t* bb = bbuf + (k % BR) * C::kBBytes;
         // 64-byte code rows loaded with the 64-byte swizzle: chunk c of row r
         // sits at chunk position c ^ ((r / 2) % 4); chunk c = elements
         // 32c..32c+31 under scale bytes 2c and 2c+1.  This thread: the whole
@@ -752,7 +766,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_co
           dst[1] = src[1];
         }
         if (!FP8) mbar_arrive(&raw_empty[s]);
-        mbar_arrive(&b_full[k & 1]);
+        mbar_arrive(&b_full[k % BR]);
       }
       if (nkind == kPageEnd && ++nend == 2) break;
       if (++s == S) { s = 0; sph ^= 1u; }

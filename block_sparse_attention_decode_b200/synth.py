@@ -277,6 +277,9 @@ WORKLOADS = {
     "ragged_b16_t1": dict(batch=16, seq_lens=None, q_tokens=1, paged=True, seed=1004),
     "prefill_67584_t2048": dict(batch=1, seq_lens=[65536 + 2048], q_tokens=2048, paged=True,
                                 seed=1005),
+    # a reduced prefill chunk (256 new tokens), small enough for counter captures
+    "prefill_65792_t256": dict(batch=1, seq_lens=[65536 + 256], q_tokens=256, paged=True,
+                               seed=1007),
 }
 
 
