@@ -68,14 +68,16 @@ constexpr int kChunkPages = 8;              // pages per work item
 constexpr int kInfoRing = 8;                // per-page info slots (decoders -> MMA, epilogue)
 constexpr int kIdxTmemCols = 256;           // two accumulators of 128 columns
 
-template <int MODE>
+template <int MODE, int M>
 struct IdxCfg {
   static constexpr bool kFp8 = MODE == kIdxFp8;
   static constexpr bool kF16 = MODE == kIdxF16;
   static constexpr int kRow = kF16 ? 256 : 128;            // bytes per query / key row
   static constexpr int kRaw = kFp8 ? kBlock * kDim : kPageCodes + kPageScales;
   static constexpr int kRawStride = (kRaw + 1023) / 1024 * 1024;
-  static constexpr int kStages = kF16 ? 3 : 6;             // raw pages in flight
+  // raw pages in flight, as many as leave room for two CTAs per SM: 6 (FP8
+  // pages, twice as large: 5), 4 with 128-row query tiles
+  static constexpr int kStages = kF16 ? 3 : M == 128 ? 4 : kFp8 ? 5 : 6;
   static constexpr int kNB = kFp8 ? 0 : 2;                 // decoded key pages (B operand), page k in k % kNB
   static constexpr int kBR = kFp8 ? 2 : kNB;               // page-ready barriers (FP8: the raw stage is B)
   static constexpr int kBBytes = kBlock * kRow;
@@ -87,7 +89,7 @@ struct IdxLayout {
 
 template <int MODE, int M>
 __host__ __device__ inline IdxLayout idx_layout(int batch) {
-  using C = IdxCfg<MODE>;
+  using C = IdxCfg<MODE, M>;
   IdxLayout L;
   int off = 0;
   L.qbuf = off;    off += (C::kF16 ? 1 : 2) * M * C::kRow;  // query tiles (multiples of 1024)
@@ -272,7 +274,7 @@ __host__ __device__ constexpr uint32_t idx_idesc() { return idesc_e4m3_f32(M, kB
 
 template <int MODE, int M>
 __global__ void __launch_bounds__(kIdxThreads, 2) indexer_kernel(const __grid_constant__ IdxArgs a) {
-  using C = IdxCfg<MODE>;
+  using C = IdxCfg<MODE, M>;
   constexpr bool FP8 = C::kFp8, F16 = C::kF16;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_dyn[];
