@@ -27,9 +27,19 @@ bool good_scale(float s) { return std::isfinite(s) && s > 0.f; }
 
 // Workspace layout (byte offsets).
 struct Layout {
-  size_t flags, bscores, sel, counters, partials, total;
+  size_t flags, bscores, sel, counters, partials, dkv, total_base, total;
   int splits;
+  bool dkv_ok;     // the batch qualifies for the decode-once attention
+  bool use_dkv;    // ... and the caller's workspace holds its rows
+  size_t used() const { return use_dkv ? total : total_base; }   // bytes the call touches
 };
+
+// Decode-once attention: when every (sequence, group) selects each of its
+// blocks several times over (T x 16 >= 4 x max_pages, as in prefill), all
+// visible blocks are decoded to E4M3 once into the workspace (32 KB per
+// (sequence, block, KV head)) and the attention reads them instead of
+// decoding per (token, group); the scratch is capped at 1 GiB.
+constexpr unsigned long long kDkvMaxBytes = 1ull << 30;
 
 bool seqs_ok(const msa_seqs* s) {
   if (!s || !s->seq_lens) return false;
@@ -52,7 +62,13 @@ Layout layout_for(const msa_seqs* s) {
   L.counters = off; off += align_up((size_t)rows * sizeof(int));
   L.partials = off;
   if (L.splits > 1) off += align_up((size_t)rows * L.splits * kPartialFloats * sizeof(float));
+  L.total_base = off;
+  const unsigned long long dkv_bytes = 2ull * s->batch * s->max_pages * kG * kBlock * kDim;
+  L.dkv_ok = (long long)s->q_tokens * kTopk >= 4LL * s->max_pages && dkv_bytes <= kDkvMaxBytes;
+  L.dkv = off;
+  if (L.dkv_ok) off += align_up((size_t)dkv_bytes);
   L.total = off;
+  L.use_dkv = false;
   return L;
 }
 
@@ -77,9 +93,13 @@ msa_status check_cache(const msa_cache* c, bool need_index, bool need_kv) {
   return MSA_OK;
 }
 
+// The decode-once rows are used when the workspace holds them (the size
+// msa_workspace_size reports); a workspace of the base size runs the same
+// step with the attention decoding per item.
 msa_status check_ws(const msa_seqs* s, void* ws, size_t ws_bytes, Layout* L) {
   *L = layout_for(s);
-  if (!ws || !aligned16(ws) || ws_bytes < L->total) return MSA_ERR_WORKSPACE;
+  if (!ws || !aligned16(ws) || ws_bytes < L->total_base) return MSA_ERR_WORKSPACE;
+  L->use_dkv = L->dkv_ok && ws_bytes >= L->total;
   return MSA_OK;
 }
 
@@ -221,6 +241,15 @@ msa_status run_attn(const msa_cache* c, const msa_seqs* s, const uint8_t* q, flo
       !encode_row_tmap(&a.tmap_q, q, (uint64_t)rows * (MSA_Q_HEADS / MSA_KV_HEADS), MSA_HEAD_DIM,
                        MSA_Q_HEADS / MSA_KV_HEADS))
     return MSA_ERR_CUDA;
+  if (L.use_dkv) {
+    const uint64_t drows = (uint64_t)s->batch * s->max_pages * MSA_KV_HEADS * MSA_BLOCK_TOKENS;
+    a.kd = at<uint8_t>(ws, L.dkv);
+    a.vd = a.kd + drows * MSA_HEAD_DIM;
+    if (!encode_row_tmap(&a.tmap_kd, a.kd, drows, MSA_HEAD_DIM) ||
+        !encode_row_tmap(&a.tmap_vd, a.vd, drows, MSA_HEAD_DIM))
+      return MSA_ERR_CUDA;
+    a.dkv = 1;
+  }
   a.k_data = c->k_data;
   a.k_scale = c->k_scale;
   a.v_data = c->v_data;
@@ -318,6 +347,8 @@ int g_grid_n = 0;
 
 }  // namespace
 
+size_t workspace_base_size(const msa_seqs* s) { return seqs_ok(s) ? layout_for(s).total_base : 0; }
+
 cudaError_t persistent_grid(const void* kernel, int threads, size_t smem, int tmem_cols, int* grid) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -397,7 +428,7 @@ msa_status msa_indexer_score_part(const msa_cache* cache, const msa_seqs* seqs, 
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
   const size_t nt = n_tok(seqs), bs_bytes = nt * MSA_KV_HEADS * seqs->max_pages * 4;
-  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+  if ((st = check_buf(ws, L.used(), MSA_ERR_WORKSPACE)) != MSA_OK ||
       (st = check_cache_mem(cache, true, false)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
       (st = check_buf(qi, nt * kQiBytes)) != MSA_OK || (st = check_buf(block_scores, bs_bytes)) != MSA_OK ||
       (st = check_buf(token_scores, bs_bytes * MSA_BLOCK_TOKENS)) != MSA_OK)
@@ -415,7 +446,7 @@ msa_status msa_block_maxpool_topk(const float* scores, int32_t is_token_level, c
   msa_status st = check_ws(seqs, ws, ws_bytes, &L);
   if (st != MSA_OK) return st;
   const size_t nt = n_tok(seqs), bs_bytes = nt * MSA_KV_HEADS * seqs->max_pages * 4;
-  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
+  if ((st = check_buf(ws, L.used(), MSA_ERR_WORKSPACE)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
       (st = check_buf(scores, is_token_level ? bs_bytes * MSA_BLOCK_TOKENS : bs_bytes)) != MSA_OK ||
       (st = check_buf(sel, nt * kSelBytes)) != MSA_OK)
     return st;
@@ -444,7 +475,7 @@ msa_status msa_sparse_attn_decode(const msa_cache* cache, const msa_seqs* seqs, 
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
   const size_t nt = n_tok(seqs);
-  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+  if ((st = check_buf(ws, L.used(), MSA_ERR_WORKSPACE)) != MSA_OK ||
       (st = check_cache_mem(cache, false, true)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
       (st = check_buf(q, nt * kQBytes)) != MSA_OK || (st = check_buf(sel, nt * kSelBytes)) != MSA_OK ||
       (st = check_buf(out, nt * kOutBytes)) != MSA_OK)
@@ -466,7 +497,7 @@ msa_status msa_decode(const msa_cache* cache, const msa_seqs* seqs, const uint8_
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
   const size_t nt = n_tok(seqs);
-  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+  if ((st = check_buf(ws, L.used(), MSA_ERR_WORKSPACE)) != MSA_OK ||
       (st = check_cache_mem(cache, true, true)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
       (st = check_buf(qi, nt * kQiBytes)) != MSA_OK || (st = check_buf(q, nt * kQBytes)) != MSA_OK ||
       (st = check_buf(out, nt * kOutBytes)) != MSA_OK || (st = check_buf(sel_out, nt * kSelBytes)) != MSA_OK)
@@ -495,7 +526,7 @@ msa_status msa_indexer_score_grouped(const msa_cache* cache, const msa_seqs* seq
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
   const size_t nt = n_tok(seqs), bs_bytes = nt * MSA_KV_HEADS * seqs->max_pages * 4;
-  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+  if ((st = check_buf(ws, L.used(), MSA_ERR_WORKSPACE)) != MSA_OK ||
       (st = check_cache_mem(cache, true, false)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
       (st = check_groups_mem(groups)) != MSA_OK ||
       (st = check_buf(qi, nt * kQiBytes)) != MSA_OK || (st = check_buf(block_scores, bs_bytes)) != MSA_OK ||
@@ -523,7 +554,7 @@ msa_status msa_decode_grouped(const msa_cache* cache, const msa_seqs* seqs,
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
   const size_t nt = n_tok(seqs);
-  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+  if ((st = check_buf(ws, L.used(), MSA_ERR_WORKSPACE)) != MSA_OK ||
       (st = check_cache_mem(cache, true, true)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
       (st = check_groups_mem(groups)) != MSA_OK ||
       (st = check_buf(qi, nt * kQiBytes)) != MSA_OK || (st = check_buf(q, nt * kQBytes)) != MSA_OK ||
@@ -551,7 +582,7 @@ msa_status msa_kv_insert(const msa_cache* cache, const msa_seqs* seqs, const uin
   Layout L;
   if ((st = check_ws(seqs, ws, ws_bytes, &L)) != MSA_OK) return st;
   const size_t nt = n_tok(seqs);
-  if ((st = check_buf(ws, L.total, MSA_ERR_WORKSPACE)) != MSA_OK ||
+  if ((st = check_buf(ws, L.used(), MSA_ERR_WORKSPACE)) != MSA_OK ||
       (st = check_cache_mem(cache, true, true)) != MSA_OK || (st = check_seqs_mem(seqs)) != MSA_OK ||
       (st = check_buf(k_new, nt * MSA_KV_HEADS * MSA_HEAD_DIM * 2)) != MSA_OK ||
       (st = check_buf(v_new, nt * MSA_KV_HEADS * MSA_HEAD_DIM * 2)) != MSA_OK ||

@@ -73,10 +73,15 @@ struct AttLayout {
   int raw, vbuf, pbuf, qbuf, lut, red, bc, lsum, bars, meta, binfo, tslot, misc, total;
 };
 
+// Decode-once mode: a stage holds the block's E4M3 K rows (the A operand of S),
+// its V rows go straight to a V buffer
+constexpr int kDkvTile = kBlock * kDim;         // 16 KB of E4M3 rows
+
+template <bool PRE>
 __host__ __device__ inline AttLayout att_layout() {
   AttLayout L;
   int off = 0;
-  L.raw = off;   off += kAttStages * kAttRawStride;
+  L.raw = off;   off += kAttStages * (PRE ? kDkvTile : kAttRawStride);
   L.vbuf = off;  off += kVB * kBlock * kDim;               // V rows, E4M3, 128-byte swizzle
   L.qbuf = off;  off += 2 * kHpg * kDim;                   // Q rows, E4M3, 128-byte swizzle
   L.pbuf = off;  off += kVB * 2 * kBlock * kHpg;           // [kVB][hi, lo][key][16 heads]
@@ -93,7 +98,7 @@ __host__ __device__ inline AttLayout att_layout() {
   return L;
 }
 
-size_t attn_smem_bytes() { return (size_t)att_layout().total; }
+size_t attn_smem_bytes() { return (size_t)att_layout<false>().total; }
 
 int attn_splits(long long rows, int num_sms) {
   int s = 1;
@@ -140,10 +145,11 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 
+template <bool PRE>
 __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
-  const AttLayout Ly = att_layout();
+  const AttLayout Ly = att_layout<PRE>();
   uint8_t* raw = smem + Ly.raw;
   uint8_t* vbuf = smem + Ly.vbuf;
   uint8_t* qbuf = smem + Ly.qbuf;
@@ -177,7 +183,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   if (tid == 0) {
     for (int s = 0; s < kAttStages; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], kAttDecoders);
+      mbar_init(&raw_empty[s], PRE ? 1 : kAttDecoders);   // decode-once: released by the S MMA
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&q_full[x], 1);
@@ -219,6 +225,25 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         if (k >= kAttStages && !mbar_wait(&raw_empty[k % kAttStages], ((k / kAttStages) - 1) & 1)) {
           report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 20);
           good = false;
+        } else if (PRE && k >= kVB && !mbar_wait(&pv_done[k % kVB], ((k / kVB) - 1) & 1)) {
+          // decode-once: V buffer k % kVB and block info slot k % 4 are free
+          // once block k-kVB's O update is done
+          report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 23);
+          good = false;
+        } else if (PRE) {
+          const int s = k % kAttStages;
+          int* bi = binfo + (k & 3) * kInfo;
+          bi[0] = kind; bi[1] = blk; bi[2] = first; bi[3] = last;
+          bi[4] = ki; bi[5] = (int)row; bi[6] = sp; bi[7] = pos;
+          if (kind == kBlkLoad) {
+            const long long b = row / ((long long)kG * a.T);
+            const long long r0 = ((b * a.max_pages + blk) * kG + g) * kBlock;   // first decoded row
+            mbar_expect_tx(&raw_full[s], 2 * kDkvTile);
+            tma_load_2d(raw + s * kDkvTile, &a.tmap_kd, 0, (int)r0, &raw_full[s]);
+            tma_load_2d(vbuf + (k % kVB) * kDkvTile, &a.tmap_vd, 0, (int)r0, &raw_full[s]);
+          } else {
+            mbar_arrive(&raw_full[s]);
+          }
         } else {
           const int s = k % kAttStages;
           int* m = meta + s * kInfo;
@@ -367,8 +392,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         bool did = false;
         if (s_end < 0) {
           const int x = ks & 1;
-          if (mbar_test(&kv_full[x], (ks >> 1) & 1) &&
-              (ks < 2 || mbar_test(&s_free[x], ((ks >> 1) - 1) & 1))) {
+          const bool in = PRE ? mbar_test(&raw_full[ks % kAttStages], (ks / kAttStages) & 1)
+                              : mbar_test(&kv_full[x], (ks >> 1) & 1);
+          if (in && (ks < 2 || mbar_test(&s_free[x], ((ks >> 1) - 1) & 1))) {
             tc_fence_after();
             const int* bi = binfo + (ks & 3) * kInfo;
             const int kind = bi[0], first = bi[2], last = bi[3], ki = bi[4];
@@ -376,12 +402,19 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
               if (kind == kBlkLoad) {
                 tc_fence_after();
                 const uint32_t d = tmem + kColS + kHpg * x;
-                const uint32_t ta = tmem + kColA + 32 * x;
                 const uint64_t bd = (ki & 1) ? qd1 : qd0;
+                if constexpr (PRE) {   // A = the block's E4M3 K rows in the stage
+                  const uint64_t ad = desc_kmajor_sw128(smem_u32(raw + (ks % kAttStages) * kDkvTile));
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc_s, kk > 0);
+                  for (int kk = 0; kk < 4; ++kk) tc_mma_ss(d, ad + 2 * kk, bd + 2 * kk, idesc_s, kk > 0);
+                } else {
+                  const uint32_t ta = tmem + kColA + 32 * x;
+#pragma unroll
+                  for (int kk = 0; kk < 4; ++kk) tc_mma_e4m3_ts(d, ta + 8 * kk, bd + 2 * kk, idesc_s, kk > 0);
+                }
               }
               tc_commit(&s_full[x]);
+              if (PRE) tc_commit(&raw_empty[ks % kAttStages]);   // the stage was the A operand
               if (kind != kBlkEnd && last) tc_commit(&q_empty[ki & 1]);
               if (kind == kBlkEnd) s_end = ks;
               ++ks;
@@ -646,7 +679,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       ++nitem;
       m_used = -INFINITY;
     }
-  } else {
+  } else if (!PRE) {
     // ------------------------------------------------------------ decoders
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     const int row = 32 * warp + lane;                // key row of this thread
@@ -727,13 +760,69 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   if (warp == kAttMmaWarp) tmem_dealloc(tmem, kAttTmemCols);
 }
 
-cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
-  const size_t smem = attn_smem_bytes();
+// Decode-once pass: every visible block of every sequence, K and V of each
+// KV head, decoded to E4M3 (the same dq8 rounding as the attention's own
+// decoders) into the workspace rows the decode-once attention loads.  One
+// thread per key row; tiles (sequence, block, head, K or V) grid-strided.
+__global__ void __launch_bounds__(kBlock) dkv_kernel(const __grid_constant__ AttnArgs a) {
+  __shared__ uint2 lut[256];
+  build_nvfp4_lut(lut, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const int row = threadIdx.x;
+  const long long tiles = (long long)a.B * a.max_pages * kG * 2;
+  for (long long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const int kv = (int)(tile & 1);
+    const long long r = tile >> 1;
+    const int g = (int)(r % kG);
+    const int blk = (int)((r / kG) % a.max_pages);
+    const int b = (int)(r / ((long long)kG * a.max_pages));
+    const int L = a.seq_lens[b];
+    // invalid lengths and page ids are reported by the attention itself
+    if (L < a.T || L > a.max_pages * kBlock || blk * kBlock >= L) continue;
+    const long long page = a.page_table ? (long long)a.page_table[(long long)b * a.max_pages + blk]
+                                        : (long long)b * a.max_pages + blk;
+    if (page < 0 || page >= a.num_pages) continue;
+    const long long src = (page * kG + g) * kBlock + row;              // (page, head, token) row
+    const uint8_t* codes = (kv ? a.v_data : a.k_data) + src * kRowCodes;
+    const uint2 sc = *reinterpret_cast<const uint2*>((kv ? a.v_scale : a.k_scale) + src * kRowScales);
+    uint8_t* dst = (kv ? a.vd : a.kd) + ((((long long)b * a.max_pages + blk) * kG + g) * kBlock + row) * kDim;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {   // 32 codes under scale bytes 2c, 2c+1
+      const uint4 w4 = *reinterpret_cast<const uint4*>(codes + 16 * c);
+      const uint32_t sb = (c < 2 ? sc.x : sc.y) >> (16 * (c & 1));
+      const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+      uint32_t o[8];
+      dq8(w4.x, r0, o[0], o[1]);
+      dq8(w4.y, r0, o[2], o[3]);
+      dq8(w4.z, r1, o[4], o[5]);
+      dq8(w4.w, r1, o[6], o[7]);
+      *reinterpret_cast<uint4*>(dst + 32 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(dst + 32 * c + 16) = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+template <bool PRE>
+static cudaError_t launch_attn_mode(const AttnArgs& a, cudaStream_t st) {
+  const size_t smem = (size_t)att_layout<PRE>().total;
   int grid = 0;
-  cudaError_t e = persistent_grid(reinterpret_cast<const void*>(attn_kernel), kAttThreads, smem,
+  cudaError_t e = persistent_grid(reinterpret_cast<const void*>(attn_kernel<PRE>), kAttThreads, smem,
                                   kAttTmemCols, &grid);
   if (e != cudaSuccess) return e;
-  return launch_dependent(attn_kernel, dim3(grid), dim3(kAttThreads), smem, st, a);
+  return launch_dependent(attn_kernel<PRE>, dim3(grid), dim3(kAttThreads), smem, st, a);
+}
+
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+  if (!a.dkv) return launch_attn_mode<false>(a, st);
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const long long tiles = (long long)a.B * a.max_pages * kG * 2;
+  const int grid = (int)std::min<long long>(tiles, 8LL * sms);
+  dkv_kernel<<<grid, kBlock, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_attn_mode<true>(a, st);
 }
 
 // ----------------------------------------------------- parity debug hook --

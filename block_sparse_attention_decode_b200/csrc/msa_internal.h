@@ -2,6 +2,7 @@
 // C-ABI layer (msa_api.cu) and the kernel files.  Not part of the ABI.
 #pragma once
 
+#include "msa.h"
 #include <cstddef>
 #include <cstdint>
 #include <utility>
@@ -81,6 +82,10 @@ cudaError_t launch_indexer(const IdxArgs& a, int mode, cudaStream_t st);
 // Any CUDA error is returned, never replaced by a default.
 cudaError_t persistent_grid(const void* kernel, int threads, size_t smem, int tmem_cols, int* grid);
 
+// Workspace bytes of a step without the decode-once rows (0 for invalid
+// sequences): what a fixed-size workspace must hold at least.
+size_t workspace_base_size(const msa_seqs* s);
+
 // Encode a tensor map over `rows` rows of `row_bytes` (64 or 128) bytes with
 // 128-row boxes and the matching shared-memory swizzle.  False on failure.
 bool encode_row_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes,
@@ -100,6 +105,13 @@ constexpr int kPartialFloats = kHpg * kDim + 2 * kHpg;   // O[16][128], m[16], l
 
 struct AttnArgs {
   CUtensorMap tmap_k, tmap_v;  // K / V code rows [P*4*128][64 B], 64-byte swizzle, 128-row boxes
+  // Decode-once mode (dkv = 1): every visible block of every sequence is
+  // decoded to E4M3 once, into kd / vd = [B][max_pages][4][128 keys][128 B]
+  // in the workspace, and the attention loads those rows (128-byte swizzle)
+  // instead of decoding per item
+  CUtensorMap tmap_kd, tmap_vd;
+  uint8_t *kd, *vd;
+  int dkv;
   CUtensorMap tmap_q;          // query rows [B*T*64][128 B], 128-byte swizzle, 16-row boxes
   const uint8_t *k_data, *k_scale, *v_data, *v_scale;
   const int32_t* page_table;

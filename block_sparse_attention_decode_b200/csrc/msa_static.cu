@@ -84,7 +84,7 @@ extern "C" MSA_API msa_status msa_decode_static(const msa_cache* cache, const ms
                                                 const uint8_t* qi, float s_qi, const uint8_t* q,
                                                 float s_q, float softmax_scale, uint16_t* out,
                                                 int32_t* sel_out, msa_stream_t stream) {
-  const size_t need = msa_workspace_size(seqs);
+  const size_t need = msa::workspace_base_size(seqs);   // decode-once rows only if they fit too
   if (need == 0) return MSA_ERR_INVALID_ARG;
   if (need > (size_t)MSA_STATIC_WORKSPACE_BYTES) return MSA_ERR_WORKSPACE;
   void* ws = nullptr;

@@ -155,7 +155,16 @@ typedef struct {
  * alone (not on the device), so it can be computed without a GPU.  The
  * workspace must be zeroed once (msa_workspace_init) before its first use and
  * may be reused by later calls on the same stream.  Returns 0 if seqs is
- * invalid (its pointers are not dereferenced). */
+ * invalid (its pointers are not dereferenced).
+ * When every (sequence, group) selects its blocks several times over
+ * (q_tokens * 16 >= 4 * max_pages, as in prefill) and the rows fit in 1 GiB,
+ * the size also holds the decode-once rows: every visible block's K and V
+ * decoded to E4M3 once per step (32 KB per sequence, block and KV head), which
+ * the attention then reads instead of decoding per (token, group) ([post,
+ * "AMD GPU support", "NVFP4 MSA kernel"]: a page dequantised once for the
+ * requests that read it).  A workspace smaller than this size but large
+ * enough for the rest runs the same step without those rows; the results are
+ * bit-identical. */
 MSA_API size_t msa_workspace_size(const msa_seqs* seqs);
 
 /* Zero the workspace's error flags (asynchronous on stream). */
@@ -294,9 +303,11 @@ MSA_API msa_status msa_debug_nvfp4_table(uint8_t* out, msa_stream_t stream);
  * are caller-owned as for msa_decode; the scratch is a fixed device array of
  * MSA_STATIC_WORKSPACE_BYTES inside the library, and nothing is allocated or
  * freed by this call.
- *   - Returns MSA_ERR_WORKSPACE when msa_workspace_size(seqs) is larger than
+ *   - Returns MSA_ERR_WORKSPACE when the step's workspace without the
+ *     decode-once rows (see msa_workspace_size) is larger than
  *     MSA_STATIC_WORKSPACE_BYTES (the batch needs a caller workspace and
- *     msa_decode), MSA_ERR_INVALID_ARG / MSA_ERR_CUDA as msa_decode.
+ *     msa_decode), MSA_ERR_INVALID_ARG / MSA_ERR_CUDA as msa_decode; the
+ *     decode-once rows are used when they fit as well.
  *   - The first call on a device looks up the array's device address for
  *     that device (cudaGetSymbolAddress, with the device current); make that
  *     first call before any stream capture on the device.  The address is

@@ -65,6 +65,21 @@ def test_workspace_size_layout(lib):
         assert lib.msa_workspace_size(ctypes.byref(bad)) == 0
 
 
+def test_workspace_size_adds_the_decode_once_rows(lib):
+    # T x 16 >= 4 x max_pages (every block of a group selected several times
+    # over, as in prefill): the size holds 32 KB of E4M3 K and V rows per
+    # (sequence, block, KV head); a decode-shaped batch does not
+    al = lambda x: (x + 255) // 256 * 256
+    dkv = 2 * 71 * 4 * 2 * 128 * 128
+    n_pre = lib.msa_workspace_size(ctypes.byref(_seqs(batch=2, T=64, max_pages=71)))
+    rows = 2 * 64 * 4
+    base = al(8) + al(rows * 71 * 4) + al(rows * 16 * 4) + al(rows * 4)
+    assert n_pre >= base + dkv
+    n_dec = lib.msa_workspace_size(ctypes.byref(_seqs(batch=2, T=8, max_pages=1024)))
+    rows = 2 * 8 * 4
+    assert n_dec < al(8) + al(rows * 1024 * 4) + al(rows * 16 * 4) + al(rows * 4) + 2 * 1024 * 4 * 2 * 128 * 128
+
+
 def _decode(lib, cache, seqs, ws=FAKE, ws_bytes=1 << 40, s_qi=1.0, s_q=1.0, scale=0.1,
             qi=FAKE, q=FAKE, out=FAKE, sel=None):
     return lib.msa_decode(ctypes.byref(cache) if cache is not None else None,
