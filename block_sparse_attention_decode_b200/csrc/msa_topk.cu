@@ -67,16 +67,17 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_le
   const int n = nb - 1;                      // candidates 0 .. nb-2
   const bool cached = n <= kTopkCache;
   unsigned kmin = 0xFFFFFFFFu, kmax = 0u;
-  // 16 loads in flight per lane (the scores come from L2 or HBM)
-  for (int base = 0; base < n; base += 16 * 32) {
-    float v[16];
+  // 32 loads in flight per lane (the scores come from L2 or HBM): a row of
+  // up to 1,024 candidates is read in one round trip
+  for (int base = 0; base < n; base += 32 * 32) {
+    float v[32];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < 32; ++j) {
       const int i = base + 32 * j + lane;
       v[j] = i < n ? __ldcg(S + i) : 0.f;
     }
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < 32; ++j) {
       const int i = base + 32 * j + lane;
       if (i < n) {
         const unsigned k = score_key(v[j]);
@@ -113,39 +114,42 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_le
     }
     __syncwarp();
     if (count <= kTopkCand) {
-      // rank of candidate j = how many candidates precede it in (key desc, id asc)
-      int sel_mask_lo = 0, sel_mask_hi = 0;   // lane holds candidates lane and lane + 32
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j = lane + 32 * h;
-        if (j < count) {
-          const unsigned kj = ck[j];
-          const int ij = cid[j];
-          int r = 0;
-          for (int m = 0; m < count; ++m) {
-            const unsigned km = ck[m];
-            r += (km > kj) || (km == kj && cid[m] < ij);
-          }
-          if (r < kTopk - 1) { if (h) sel_mask_hi = 1; else sel_mask_lo = 1; }
-        }
+      // lane holds candidates lane and lane + 32 in registers; the others'
+      // come by shuffle.  Rank of candidate j = how many candidates precede it
+      // in (key desc, id asc); the 15 of rank < 15 are selected.
+      const bool v0 = lane < count, v1 = lane + 32 < count;
+      const unsigned k0 = v0 ? ck[lane] : 0u, k1 = v1 ? ck[lane + 32] : 0u;
+      const int i0 = v0 ? cid[lane] : 0x7FFFFFFF, i1 = v1 ? cid[lane + 32] : 0x7FFFFFFF;
+      int r0 = 0, r1 = 0;
+      const int c0 = min(count, 32), c1 = count - c0;
+      for (int m = 0; m < c0; ++m) {
+        const unsigned km = __shfl_sync(0xffffffffu, k0, m);
+        const int im = __shfl_sync(0xffffffffu, i0, m);
+        r0 += (km > k0) || (km == k0 && im < i0);
+        r1 += (km > k1) || (km == k1 && im < i1);
       }
-      __syncwarp();
+      for (int m = 0; m < c1; ++m) {
+        const unsigned km = __shfl_sync(0xffffffffu, k1, m);
+        const int im = __shfl_sync(0xffffffffu, i1, m);
+        r0 += (km > k0) || (km == k0 && im < i0);
+        r1 += (km > k1) || (km == k1 && im < i1);
+      }
+      const bool s0 = v0 && r0 < kTopk - 1, s1 = v1 && r1 < kTopk - 1;
       // the 15 selected ids in ascending order: position = selected ids below
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j = lane + 32 * h;
-        const bool mine = h ? sel_mask_hi : sel_mask_lo;
-        const unsigned b0 = __ballot_sync(0xffffffffu, sel_mask_lo), b1 = __ballot_sync(0xffffffffu, sel_mask_hi);
-        if (mine) {
-          const int ij = cid[j];
-          int posn = 0;
-          for (int m = 0; m < 32; ++m) {
-            if ((b0 >> m) & 1u) posn += cid[m] < ij;
-            if ((b1 >> m) & 1u) posn += cid[m + 32] < ij;
-          }
-          out[posn] = ij;
-        }
+      const unsigned b0 = __ballot_sync(0xffffffffu, s0), b1 = __ballot_sync(0xffffffffu, s1);
+      int p0 = 0, p1 = 0;
+      for (unsigned bb = b0; bb; bb &= bb - 1u) {
+        const int im = __shfl_sync(0xffffffffu, i0, __ffs(bb) - 1);
+        p0 += im < i0;
+        p1 += im < i1;
       }
+      for (unsigned bb = b1; bb; bb &= bb - 1u) {
+        const int im = __shfl_sync(0xffffffffu, i1, __ffs(bb) - 1);
+        p0 += im < i0;
+        p1 += im < i1;
+      }
+      if (s0) out[p0] = i0;
+      if (s1) out[p1] = i1;
       if (lane == 0) out[kTopk - 1] = nb - 1;
       return;
     }
