@@ -89,7 +89,7 @@ __host__ __device__ inline AttLayout att_layout() {
   L.red = off;   off += 2 * 4 * kHpg * 4;                  // block maxima [parity][quarter][16]
   L.bc = off;    off += kAttSoft * 2 * kHh * 4;            // per softmax warp: offsets, alphas
   L.lsum = off;  off += 2 * 4 * kHpg * 4;                  // row sums [parity][quarter][16]
-  L.bars = off;  off += (2 * kAttStages + 19) * 8;
+  L.bars = off;  off += (2 * kAttStages + 2 * kVB + 14) * 8;
   L.meta = off;  off += kAttStages * kInfo * 4;
   L.binfo = off; off += 4 * kInfo * 4;
   L.tslot = off; off += 16;
@@ -164,8 +164,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   uint64_t* q_empty = q_full + 2;                // [2] MMA -> producer
   uint64_t* kv_full = q_empty + 2;               // [2] decoders -> MMA
   uint64_t* s_full = kv_full + 2;                // [2] MMA -> softmax
-  uint64_t* p_full = s_full + 2;                 // [2] softmax -> MMA
-  uint64_t* pv_done = p_full + 2;                // [kVB] MMA -> decoders, softmax
+  uint64_t* p_full = s_full + 2;                 // [kVB] softmax -> MMA
+  uint64_t* pv_done = p_full + kVB;              // [kVB] MMA -> decoders, softmax
   uint64_t* o_free = pv_done + kVB;              // [2] softmax -> MMA
   uint64_t* red_full = o_free + 2;               // [1] softmax rendezvous
   uint64_t* misc_bar = red_full + 1;             // [1] softmax rendezvous (item end)
@@ -190,10 +190,12 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       mbar_init(&q_empty[x], 1);
       mbar_init(&kv_full[x], kAttDecoders);
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], kAttSoft);
       mbar_init(&o_free[x], kAttSoft);
     }
-    for (int x = 0; x < kVB; ++x) mbar_init(&pv_done[x], 1);
+    for (int x = 0; x < kVB; ++x) {
+      mbar_init(&p_full[x], kAttSoft);
+      mbar_init(&pv_done[x], 1);
+    }
     mbar_init(red_full, kAttSoft);
     mbar_init(misc_bar, kAttSoft);
     for (int x = 0; x < 2; ++x) mbar_init(&s_free[x], kAttSoft);
@@ -423,8 +425,10 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           }
         }
         if (ko < ks && (s_end < 0 || ko < s_end)) {
-          const int x = ko & 1;
-          if (mbar_test(&p_full[x], (ko >> 1) & 1)) {
+          // P of block ko: p_full[ko % kVB].  Its previous phase (block
+          // ko-kVB) was taken here before the softmax, which waits for that
+          // block's O update, could start block ko: phases never alias
+          if (mbar_test(&p_full[ko % kVB], (ko / kVB) & 1)) {
             tc_fence_after();
             const int* bi = binfo + (ko & 3) * kInfo;
             const int kind = bi[0], first = bi[2], ki = bi[4];
@@ -565,15 +569,16 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[x]);
+      if (lane == 0) mbar_arrive(&p_full[vb]);
       if (!last) continue;
 
       // ---------------------------------------------------- end of the item
-      // row sums: this warp's 32 keys, then the four quarters
-      if (kind == kBlkLoad) {
-        if (!mbar_wait(&pv_done[vb], (k / kVB) & 1)) { report(a.flags, 5, 30); break; }
-        tc_fence_after();
-      }
+      // The item's last O update (for an empty item: the O stream's pass over
+      // its block, which takes o_free's phase of item ki-2) before o_free's
+      // phase of this item; then the row sums: this warp's 32 keys, then the
+      // four quarters
+      if (!mbar_wait(&pv_done[vb], (k / kVB) & 1)) { report(a.flags, 5, 30); break; }
+      tc_fence_after();
 #pragma unroll
       for (int h = 0; h < kHh; ++h) {
         float v = lt[h];

@@ -308,6 +308,26 @@ def test_repeat_calls_reuse_workspace():
     assert ws[64:80].view(torch.int32).tolist() == [0, 0, 0, 0]
 
 
+def test_split_k_with_empty_slices_repeated():
+    """Few rows (8 sequences x 1 token x 4 groups): the attention splits each
+    row's 16 selected blocks into 16 one-block slices merged through fp32
+    partials, and a slice past a short sequence's last visible block is an
+    empty item, which passes through the pipeline without a load or an MMA.
+    Twenty calls on one workspace give the same bits (the row counters go
+    back to 0 and no item's hand-offs race ahead of another's), and the first
+    matches the oracle."""
+    lens = [300, 700, 1025, 130, 5000, 2000, 900, 64]
+    w = dev_workload("empty_slices", len(lens), lens, 1, paged=True, seed=54)
+    seqs = msa.seqs_of(w)
+    ws = msa.alloc_workspace(seqs)
+    o1, s1 = run_decode(w, ws)
+    for _ in range(19):
+        o2, s2 = run_decode(w, ws)
+        assert torch.equal(s1, s2)
+        assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    compare_decode(w, what="split-K with empty slices")
+
+
 # ---------------------------------------------------------- boundaries -----
 def test_bad_page_id_sets_device_flag_and_context_survives():
     w = dev_workload("badpage", 2, [5000, 3000], 1, paged=True, seed=61)
