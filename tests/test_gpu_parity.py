@@ -328,6 +328,31 @@ def test_split_k_with_empty_slices_repeated():
     compare_decode(w, what="split-K with empty slices")
 
 
+# batches whose (sequence, token, group) rows take 8, 4 and 2 slices each (rows x
+# slices >= 4 x 148), short sequences among long ones: empty and partial slices
+SPLIT_CASES = [(8, 19), (4, 37), (2, 74)]
+
+
+@pytest.mark.parametrize("splits,batch", SPLIT_CASES, ids=["splits%d" % s for s, _ in SPLIT_CASES])
+def test_split_counts_with_empty_slices(splits, batch):
+    """Each split count of the attention's split-K on one token per sequence:
+    the rows' outputs against the oracle over the GPU's own selection (on
+    every fourth sequence, all lengths represented), and two calls on one
+    workspace bit-identical."""
+    rows = batch * 4
+    assert rows * splits >= 4 * 148 and (splits == 16 or rows * splits // 2 < 4 * 148)
+    cycle = [300, 700, 1025, 130, 5000, 2000, 900, 64, 9000, 16000, 2049]
+    lens = [cycle[i % len(cycle)] for i in range(batch)]
+    w = dev_workload("splits%d" % splits, batch, lens, 1, paged=True, seed=55 + splits)
+    seqs = msa.seqs_of(w)
+    ws = msa.alloc_workspace(seqs)
+    o1, s1 = run_decode(w, ws)
+    o2, s2 = run_decode(w, ws)
+    assert torch.equal(s1, s2)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    compare_decode(w, seq_ids=list(range(0, batch, 4)), what="split-K x%d" % splits)
+
+
 # ---------------------------------------------------------- boundaries -----
 def test_bad_page_id_sets_device_flag_and_context_survives():
     w = dev_workload("badpage", 2, [5000, 3000], 1, paged=True, seed=61)
