@@ -15,7 +15,7 @@
 //     tiled TMA loads of the K and V codes (64-byte swizzle) and two bulk
 //     copies of their scales into a ring of shared-memory stages;
 //   warps 0-3 (decoders): thread = key row, warp w decoding rows
-//     32w..32w+31.  K is decoded signed (dq8) straight into tensor memory
+//     32w..32w+31 (kKVSplit below: K here and V on warps 4-7).  K is decoded signed (dq8) straight into tensor memory
 //     (dq8; one A operand: 4 MMAs per block rather than 8 for a split by sign --
 //     the MMA-issuing thread is the scarcer resource here); V is decoded
 //     signed into shared memory as E4M3 rows of 128
@@ -48,11 +48,18 @@
 
 namespace msa {
 
+// kKVSplit: K and V decoded by separate warps (K: 0-3, V: 4-7), so that a
+// block's two decodes run side by side, the softmax then on four warps of 16
+// heads (8-11).  Correct, but slower (0.211 against 0.202 ms at 64 x 128K,
+// T = 8): off.
+constexpr bool kKVSplit = false;
 constexpr int kAttDecoders = 4;             // warps 0-3, one per TMEM lane quarter
-constexpr int kAttSoftWarp0 = 4;            // softmax warps 4-11: two per lane quarter
-constexpr int kAttSoft = 8;
-constexpr int kHh = kHpg / 2;               // heads per softmax warp
-static_assert(kHh == 8, "softmax warps hold eight heads (two float4 of block maxima)");
+constexpr int kAttVWarp0 = 4;               // V decoders (with the split): warps 4-7
+constexpr int kAttSoft = kKVSplit ? 4 : 8;  // softmax warps: one or two per lane quarter
+constexpr int kAttSoftWarp0 = kKVSplit ? 8 : 4;
+constexpr int kHh = kHpg * 4 / kAttSoft;    // heads per softmax warp
+static_assert(kHh % 8 == 0, "softmax warps hold whole groups of eight heads");
+constexpr int kRing = 8;                    // block info slots (decoders -> MMA, softmax)
 constexpr int kAttProducerWarp = 12;
 constexpr int kAttMmaWarp = 13;
 constexpr int kAttRawStride = 2 * (kPageCodes + kPageScales);   // 18432 = 18 x 1024
@@ -65,7 +72,7 @@ constexpr int kVB = 3;                      // V and P buffers (blocks between d
 enum : int { kBlkLoad = 0, kBlkEmpty = 1, kBlkEnd = 2 };
 
 // Block info (producer -> decoders via the stage meta, decoders -> MMA and
-// softmax via a ring of 4): kind, block id, first, last, item sequence
+// softmax via a ring of kRing): kind, block id, first, last, item sequence
 // number, row, split, query position.
 constexpr int kInfo = 8;
 
@@ -89,9 +96,9 @@ __host__ __device__ inline AttLayout att_layout() {
   L.red = off;   off += 2 * 4 * kHpg * 4;                  // block maxima [parity][quarter][16]
   L.bc = off;    off += kAttSoft * 2 * kHh * 4;            // per softmax warp: offsets, alphas
   L.lsum = off;  off += 2 * 4 * kHpg * 4;                  // row sums [parity][quarter][16]
-  L.bars = off;  off += (2 * kAttStages + 2 * kVB + 14) * 8;
+  L.bars = off;  off += (2 * kAttStages + 3 * kVB + 14) * 8;
   L.meta = off;  off += kAttStages * kInfo * 4;
-  L.binfo = off; off += 4 * kInfo * 4;
+  L.binfo = off; off += kRing * kInfo * 4;
   L.tslot = off; off += 16;
   L.misc = off;  off += 16;
   L.total = off + 1024;                                    // alignment slack
@@ -170,6 +177,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   uint64_t* red_full = o_free + 2;               // [1] softmax rendezvous
   uint64_t* misc_bar = red_full + 1;             // [1] softmax rendezvous (item end)
   uint64_t* s_free = misc_bar + 1;               // [2] softmax -> MMA: S buffer read
+  uint64_t* v_full = s_free + 2;                 // [kVB] V decoders -> MMA (with the split)
   int* meta = reinterpret_cast<int*>(smem + Ly.meta);
   int* binfo = reinterpret_cast<int*>(smem + Ly.binfo);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly.tslot);
@@ -183,7 +191,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
   if (tid == 0) {
     for (int s = 0; s < kAttStages; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], PRE ? 1 : kAttDecoders);   // decode-once: released by the S MMA
+      // decode-once: released by the S MMA; else by the K (and V) decoders
+      mbar_init(&raw_empty[s], PRE ? 1 : kKVSplit ? 2 * kAttDecoders : kAttDecoders);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&q_full[x], 1);
@@ -195,6 +204,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     for (int x = 0; x < kVB; ++x) {
       mbar_init(&p_full[x], kAttSoft);
       mbar_init(&pv_done[x], 1);
+      mbar_init(&v_full[x], kAttDecoders);
     }
     mbar_init(red_full, kAttSoft);
     mbar_init(misc_bar, kAttSoft);
@@ -228,13 +238,13 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 20);
           good = false;
         } else if (PRE && k >= kVB && !mbar_wait(&pv_done[k % kVB], ((k / kVB) - 1) & 1)) {
-          // decode-once: V buffer k % kVB and block info slot k % 4 are free
+          // decode-once: V buffer k % kVB and block info slot k % 8 are free
           // once block k-kVB's O update is done
           report(a.flags, 5 /*MSA_ERR_TIMEOUT*/, 23);
           good = false;
         } else if (PRE) {
           const int s = k % kAttStages;
-          int* bi = binfo + (k & 3) * kInfo;
+          int* bi = binfo + (k & (kRing - 1)) * kInfo;
           bi[0] = kind; bi[1] = blk; bi[2] = first; bi[3] = last;
           bi[4] = ki; bi[5] = (int)row; bi[6] = sp; bi[7] = pos;
           if (kind == kBlkLoad) {
@@ -398,7 +408,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
                               : mbar_test(&kv_full[x], (ks >> 1) & 1);
           if (in && (ks < 2 || mbar_test(&s_free[x], ((ks >> 1) - 1) & 1))) {
             tc_fence_after();
-            const int* bi = binfo + (ks & 3) * kInfo;
+            const int* bi = binfo + (ks & (kRing - 1)) * kInfo;
             const int kind = bi[0], first = bi[2], last = bi[3], ki = bi[4];
             if (kind != kBlkLoad || !first || mbar_test(&q_full[ki & 1], (ki >> 1) & 1)) {
               if (kind == kBlkLoad) {
@@ -428,9 +438,10 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           // P of block ko: p_full[ko % kVB].  Its previous phase (block
           // ko-kVB) was taken here before the softmax, which waits for that
           // block's O update, could start block ko: phases never alias
-          if (mbar_test(&p_full[ko % kVB], (ko / kVB) & 1)) {
+          if (mbar_test(&p_full[ko % kVB], (ko / kVB) & 1) &&
+              (PRE || !kKVSplit || mbar_test(&v_full[ko % kVB], (ko / kVB) & 1))) {
             tc_fence_after();
-            const int* bi = binfo + (ko & 3) * kInfo;
+            const int* bi = binfo + (ko & (kRing - 1)) * kInfo;
             const int kind = bi[0], first = bi[2], ki = bi[4];
             const int ob = ki & 1;
             if (!(first && ki >= 2) || mbar_test(&o_free[ob], ((ki >> 1) - 1) & 1)) {
@@ -464,7 +475,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     }
   } else if (warp >= kAttSoftWarp0) {
     // ------------------------------------------------------------ softmax
-    // warp 4 + 4*hh + q: keys (TMEM lanes) 32q..32q+31, heads 8hh..8hh+7
+    // warp kAttSoftWarp0 + 4*hh + q: keys (TMEM lanes) 32q..32q+31, heads kHh*hh..kHh*hh+kHh-1
     const int q = warp & 3, hh = (warp - kAttSoftWarp0) >> 2, h0 = kHh * hh;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     const float c = a.logit_scale_log2;               // softmax_scale * s_q * s_k * log2(e)
@@ -472,13 +483,13 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     float lt[kHh];                                    // this key lane's share of the row sums
 #pragma unroll
     for (int h = 0; h < kHh; ++h) lt[h] = 0.f;
-    float m_used = -INFINITY;                         // lanes 0-7: running max of head h0+lane
+    float m_used = -INFINITY;                         // lanes < kHh: running max of head h0+lane
     int nred = 0, nmisc = 0, nitem = 0;
     for (int k = 0;; ++k) {
       const int x = k & 1;
       if (!mbar_wait(&s_full[x], (k >> 1) & 1)) { report(a.flags, 5, 26); break; }
       tc_fence_after();
-      const int* bi = binfo + (k & 3) * kInfo;
+      const int* bi = binfo + (k & (kRing - 1)) * kInfo;
       const int kind = bi[0], blk = bi[1], first = bi[2], last = bi[3], ki = bi[4];
       const long long row = bi[5];
       const int sp = bi[6], pos = bi[7];
@@ -488,7 +499,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       if (k >= kVB && !mbar_wait(&pv_done[vb], ((k / kVB) - 1) & 1)) { report(a.flags, 5, 27); break; }
       float s[kHh];
       if (kind == kBlkLoad) {
-        tmem_ld8(lane_base + kColS + kHpg * x + h0, s);
+#pragma unroll
+        for (int j = 0; j < kHh / 8; ++j)
+          tmem_ld8(lane_base + kColS + kHpg * x + h0 + 8 * j, *reinterpret_cast<float(*)[8]>(s + 8 * j));
         tmem_wait_ld();
       }
       tc_fence_before();
@@ -505,8 +518,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
 #pragma unroll
         for (int h = 0; h < kHh; ++h) mh[h] = warp_max(s[h]);
         if (lane == 0) {
-          reinterpret_cast<float4*>(rq)[0] = make_float4(mh[0], mh[1], mh[2], mh[3]);
-          reinterpret_cast<float4*>(rq)[1] = make_float4(mh[4], mh[5], mh[6], mh[7]);
+#pragma unroll
+          for (int j = 0; j < kHh / 4; ++j)
+            reinterpret_cast<float4*>(rq)[j] = make_float4(mh[4 * j], mh[4 * j + 1], mh[4 * j + 2], mh[4 * j + 3]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(red_full);
@@ -537,19 +551,20 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           tc_fence_after();
           const uint32_t oa = lane_base + kColO + 2 * kHpg * ob + h0;
 #pragma unroll 1
-          for (int j = 0; j < 2; ++j) {   // the hi and the lo columns of heads h0..h0+7
+          for (int j = 0; j < 2 * (kHh / 8); ++j) {   // hi, lo columns of heads h0.., eight at a time
+            const int hg = 8 * (j % (kHh / 8)), col = kHpg * (j / (kHh / 8)) + hg;
             float o8[8];
-            tmem_ld8(oa + kHpg * j, o8);
+            tmem_ld8(oa + col, o8);
             tmem_wait_ld();
             uint32_t w8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(o8[i] * al[i]);
-            tmem_st8(oa + kHpg * j, w8);
+            for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(o8[i] * al[hg + i]);
+            tmem_st8(oa + col, w8);
           }
           tmem_wait_st();
         }
-        // P = 2^(s c - m c + 4) as hi + lo E4M3: bytes h0..h0+7 of the key's rows
-        uint32_t ph[2], pl[2];
+        // P = 2^(s c - m c + 4) as hi + lo E4M3: bytes h0..h0+kHh-1 of the key's rows
+        uint32_t ph[kHh / 4], pl[kHh / 4];
 #pragma unroll
         for (int h2 = 0; h2 < kHh / 2; ++h2) {
           const float2 mo = *reinterpret_cast<const float2*>(mybc + 2 * h2);   // exponent offsets
@@ -563,8 +578,13 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
           else { ph[h2 >> 1] = hw; pl[h2 >> 1] = lw; }
         }
         uint8_t* pb = pbuf + vb * 2 * kBlock * kHpg + (32 * q + lane) * kHpg + h0;
-        *reinterpret_cast<uint2*>(pb) = make_uint2(ph[0], ph[1]);
-        *reinterpret_cast<uint2*>(pb + kBlock * kHpg) = make_uint2(pl[0], pl[1]);
+        if constexpr (kHh == 16) {
+          *reinterpret_cast<uint4*>(pb) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+          *reinterpret_cast<uint4*>(pb + kBlock * kHpg) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        } else {
+          *reinterpret_cast<uint2*>(pb) = make_uint2(ph[0], ph[1]);
+          *reinterpret_cast<uint2*>(pb + kBlock * kHpg) = make_uint2(pl[0], pl[1]);
+        }
         fence_async_smem();
       }
       tc_fence_before();
@@ -594,34 +614,35 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
       if (lane == 0) mbar_arrive(misc_bar);
       if (!mbar_wait(misc_bar, (nmisc++) & 1)) { report(a.flags, 5, 31); break; }
       const float* ls = lsum + (nitem & 1) * 4 * kHpg + h0;   // [quarter][16] row sums
-      const float mc = m_used * c;                     // lanes 0-7: m of head h0+lane, log2 units
+      const float mc = m_used * c;                     // lanes < kHh: m of head h0+lane, log2 units
       const int d = 32 * q + lane;                     // this thread's dimension
       const int b = (int)(row / (kG * a.T));
       const int t = (int)((row / kG) % a.T);
       const int g = (int)(row % kG);
-      // O = O_hi + O_lo of heads h0..h0+7, then release O^T
+      // O = O_hi + O_lo of heads h0..h0+kHh-1, then release O^T
       float o[kHh];
-      {
+#pragma unroll
+      for (int j = 0; j < kHh / 8; ++j) {
         float hi8[8], lo8[8];
         if (kind == kBlkLoad) {
-          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + h0, hi8);
-          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + kHpg + h0, lo8);
+          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + h0 + 8 * j, hi8);
+          tmem_ld8(lane_base + kColO + 2 * kHpg * ob + kHpg + h0 + 8 * j, lo8);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) hi8[i] = lo8[i] = 0.f;
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = hi8[i] + lo8[i];
+        for (int i = 0; i < 8; ++i) o[8 * j + i] = hi8[i] + lo8[i];
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[ob]);
-      // lanes 0-7: the row sum of head h0+lane over the four quarters
+      // lanes < kHh: the row sum of head h0+lane over the four quarters
       const float lrow = lane < kHh ? ls[lane] + ls[kHpg + lane] + ls[2 * kHpg + lane] + ls[3 * kHpg + lane]
                                     : 0.f;
       if (a.splits == 1) {
-        const float f = lrow > 0.f ? a.out_scale / lrow : 0.f;   // lanes 0-7
+        const float f = lrow > 0.f ? a.out_scale / lrow : 0.f;   // lanes < kHh
         uint16_t* dst = a.out + (((long long)b * a.T + t) * kHq + kHpg * g + h0) * kDim + d;
 #pragma unroll
         for (int h = 0; h < kHh; ++h) {
@@ -651,33 +672,36 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         if (!mbar_wait(misc_bar, (nmisc++) & 1)) { report(a.flags, 5, 35); break; }
         if (misc[nitem & 1]) {
           __threadfence();
-          // 256 threads: head hr = tq/16, 8 dims from (tq%16)*8
-          const int tq = (warp - kAttSoftWarp0) * 32 + lane, hr = tq >> 4, d0 = (tq & 15) * 8;
+          // kAttSoft x 32 threads: head hr, kDpt dims from d0
+          constexpr int kDpt = kHpg * kDim / (kAttSoft * 32), kTph = kDim / kDpt;   // dims / thread, threads / head
+          const int tq = (warp - kAttSoftWarp0) * 32 + lane, hr = tq / kTph, d0 = (tq % kTph) * kDpt;
           const float* base = a.partials + row * a.splits * kPartialFloats;
           float Mx = -INFINITY;
           for (int s2 = 0; s2 < a.splits; ++s2)
             Mx = fmaxf(Mx, __ldcg(base + s2 * kPartialFloats + kHpg * kDim + hr));
           const float Mu = (Mx == -INFINITY) ? 0.f : Mx;
-          float tot[8];
+          float tot[kDpt];
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) tot[cc] = 0.f;
+          for (int cc = 0; cc < kDpt; ++cc) tot[cc] = 0.f;
           float Lt = 0.f;
           for (int s2 = 0; s2 < a.splits; ++s2) {
             const float* ps2 = base + s2 * kPartialFloats;
             const float f = exp2f(__ldcg(ps2 + kHpg * kDim + hr) - Mu);
             Lt += __ldcg(ps2 + kHpg * kDim + kHpg + hr) * f;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) tot[cc] += __ldcg(ps2 + hr * kDim + d0 + cc) * f;
+            for (int cc = 0; cc < kDpt; ++cc) tot[cc] += __ldcg(ps2 + hr * kDim + d0 + cc) * f;
           }
           const float inv = Lt > 0.f ? a.out_scale / Lt : 0.f;
-          uint32_t packed[4];
+          uint32_t packed[kDpt / 2];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < kDpt / 2; ++cc) {
             const __nv_bfloat162 v = __floats2bfloat162_rn(tot[2 * cc] * inv, tot[2 * cc + 1] * inv);
             packed[cc] = *reinterpret_cast<const uint32_t*>(&v);
           }
-          *reinterpret_cast<uint4*>(a.out + (((long long)b * a.T + t) * kHq + kHpg * g + hr) * kDim + d0) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          uint4* op = reinterpret_cast<uint4*>(a.out + (((long long)b * a.T + t) * kHq + kHpg * g + hr) * kDim + d0);
+#pragma unroll
+          for (int cc = 0; cc < kDpt / 8; ++cc)
+            op[cc] = make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2], packed[4 * cc + 3]);
           if (tq == 0) a.counters[row] = 0;   // ready for the next call
         }
       }
@@ -686,15 +710,22 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
     }
   } else if (!PRE) {
     // ------------------------------------------------------------ decoders
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-    const int row = 32 * warp + lane;                // key row of this thread
+    // warps 0-3 decode K (and, without the split, V); warps 4-7 decode V
+    const bool vdec = kKVSplit && warp >= kAttVWarp0;
+    const bool kdec = !vdec;
+    const int qd = warp & 3;                         // row block = TMEM lane quarter
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * qd) << 16);
+    const int row = 32 * qd + lane;                  // key row of this thread
     const int sw = (row >> 1) & 3;                   // 64-byte swizzle of the code rows
     for (int k = 0;; ++k) {
       const int s = k % kAttStages, x = k & 1;
       if (!mbar_wait(&raw_full[s], (k / kAttStages) & 1)) { report(a.flags, 5, 33); break; }
       // A[x] was last read by block k-2's S; V buffer k % kVB by block k-kVB's O
-      if (k >= 2 && !mbar_wait(&s_full[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 34); break; }
-      if (k >= kVB && !mbar_wait(&pv_done[k % kVB], ((k / kVB) - 1) & 1)) { report(a.flags, 5, 36); break; }
+      if (kdec && k >= 2 && !mbar_wait(&s_full[x], ((k >> 1) - 1) & 1)) { report(a.flags, 5, 34); break; }
+      if ((vdec || !kKVSplit) && k >= kVB && !mbar_wait(&pv_done[k % kVB], ((k / kVB) - 1) & 1)) {
+        report(a.flags, 5, 36);
+        break;
+      }
       tc_fence_after();
       const int* m = meta + s * kInfo;
       const int kind = m[0];
@@ -704,55 +735,64 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const __grid_const
         const uint8_t* vc = rs + kPageCodes;
         const uint8_t* ks = rs + 2 * kPageCodes;
         const uint8_t* vs = ks + kPageScales;
-        // K signed, as E4M3 into A[x] (row = TMEM lane, 32 columns)
-        const uint32_t abase = lane_base + kColA + 32 * x;
-        const uint2 ksc = *reinterpret_cast<const uint2*>(ks + row * kRowScales);
+        if (kdec) {
+          // K signed, as E4M3 into A[x] (row = TMEM lane, 32 columns)
+          const uint32_t abase = lane_base + kColA + 32 * x;
+          const uint2 ksc = *reinterpret_cast<const uint2*>(ks + row * kRowScales);
 #pragma unroll
-        for (int cix = 0; cix < 4; ++cix) {
-          const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
-          const uint32_t sb = (cix < 2 ? ksc.x : ksc.y) >> (16 * (cix & 1));
-          const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
-          uint32_t o[8];
-          dq8(w4.x, r0, o[0], o[1]);
-          dq8(w4.y, r0, o[2], o[3]);
-          dq8(w4.z, r1, o[4], o[5]);
-          dq8(w4.w, r1, o[6], o[7]);
-          tmem_st8(abase + 8 * cix, o);
+          for (int cix = 0; cix < 4; ++cix) {
+            const uint4 w4 = lds128(kc + row * kRowCodes + ((cix ^ sw) << 4));
+            const uint32_t sb = (cix < 2 ? ksc.x : ksc.y) >> (16 * (cix & 1));
+            const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+            uint32_t o[8];
+            dq8(w4.x, r0, o[0], o[1]);
+            dq8(w4.y, r0, o[2], o[3]);
+            dq8(w4.z, r1, o[4], o[5]);
+            dq8(w4.w, r1, o[6], o[7]);
+            tmem_st8(abase + 8 * cix, o);
+          }
+          tmem_wait_st();
         }
-        // V signed, as E4M3 into the 128-byte V row of this key (16-byte
-        // chunk j at chunk position j ^ (key % 8))
-        const uint2 vsc = *reinterpret_cast<const uint2*>(vs + row * kRowScales);
-        uint8_t* vrow = vbuf + (k % kVB) * kBlock * kDim + row * kDim;
+        if (vdec || !kKVSplit) {
+          // V signed, as E4M3 into the 128-byte V row of this key (16-byte
+          // chunk j at chunk position j ^ (key % 8))
+          const uint2 vsc = *reinterpret_cast<const uint2*>(vs + row * kRowScales);
+          uint8_t* vrow = vbuf + (k % kVB) * kBlock * kDim + row * kDim;
 #pragma unroll
-        for (int cix = 0; cix < 4; ++cix) {
-          const uint4 w4 = lds128(vc + row * kRowCodes + ((cix ^ sw) << 4));
-          const uint32_t sb = (cix < 2 ? vsc.x : vsc.y) >> (16 * (cix & 1));
-          const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
-          uint32_t o[8];
-          dq8(w4.x, r0, o[0], o[1]);
-          dq8(w4.y, r0, o[2], o[3]);
-          dq8(w4.z, r1, o[4], o[5]);
-          dq8(w4.w, r1, o[6], o[7]);
-          // code chunk cix = dims 32cix..32cix+31 = V chunks 2cix, 2cix+1
-          *reinterpret_cast<uint4*>(vrow + (((2 * cix) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(vrow + (((2 * cix + 1) ^ (row & 7)) << 4)) =
-              make_uint4(o[4], o[5], o[6], o[7]);
+          for (int cix = 0; cix < 4; ++cix) {
+            const uint4 w4 = lds128(vc + row * kRowCodes + ((cix ^ sw) << 4));
+            const uint32_t sb = (cix < 2 ? vsc.x : vsc.y) >> (16 * (cix & 1));
+            const uint2 r0 = lut[sb & 0xFFu], r1 = lut[(sb >> 8) & 0xFFu];
+            uint32_t o[8];
+            dq8(w4.x, r0, o[0], o[1]);
+            dq8(w4.y, r0, o[2], o[3]);
+            dq8(w4.z, r1, o[4], o[5]);
+            dq8(w4.w, r1, o[6], o[7]);
+            // code chunk cix = dims 32cix..32cix+31 = V chunks 2cix, 2cix+1
+            *reinterpret_cast<uint4*>(vrow + (((2 * cix) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(vrow + (((2 * cix + 1) ^ (row & 7)) << 4)) =
+                make_uint4(o[4], o[5], o[6], o[7]);
+          }
+          fence_async_smem();
         }
-        tmem_wait_st();
-        fence_async_smem();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         // the block info leaves the stage before the stage is released (the
-        // producer rewrites it for block k + kAttStages right after)
+        // producer rewrites it for block k + kAttStages right after); the
+        // ring of kRing slots outlives every reader: slot k is rewritten at
+        // block k + kRing, after block k + kRing - 2's S, hence after the
+        // softmax of block k + kRing - 4 began, which waited for block
+        // k + kRing - 4 - kVB's O update (and the O stream runs in order)
         if (warp == 0) {
-          int* bi = binfo + (k & 3) * kInfo;
+          int* bi = binfo + (k & (kRing - 1)) * kInfo;
 #pragma unroll
           for (int i = 0; i < kInfo; ++i) bi[i] = m[i];
         }
         mbar_arrive(&raw_empty[s]);
-        mbar_arrive(&kv_full[x]);
+        if (vdec) mbar_arrive(&v_full[k % kVB]);
+        else mbar_arrive(&kv_full[x]);
       }
       if (kind == kBlkEnd) break;
     }
