@@ -669,16 +669,18 @@ def main():
             return 0
         w = cpu_sample_workload(args.workload)
         threads = host_threads()
-        # K steps of one query each (token k % T of the sampled sequence: full
-        # index scan, top-16, attention), evaluated together on all host cores;
-        # the W warm-up queries likewise.
-        oracle_step(w, [(0, k % w.q_tokens) for k in range(args.warmup)], threads)
-        t = oracle_step(w, [(0, k % w.q_tokens) for k in range(args.steps)], threads)
-        qps = args.steps / t
-        sample = ("per step: one query token of 1 sequence of %d tokens (shapes of %s): full "
-                  "index scan, top-16 and attention in the float64 C oracle; the %d steps run "
-                  "together on %d host threads" % (int(w.seq_lens[0]), args.workload, args.steps,
-                                                   threads))
+        # K steps of T queries each (every query token of the sampled sequence:
+        # full index scan, top-16, attention), evaluated together on all host
+        # cores, so that even a few steps give every core rows; the W warm-up
+        # steps likewise.
+        T = w.q_tokens
+        oracle_step(w, [(0, k % T) for k in range(args.warmup * T)], threads)
+        t = oracle_step(w, [(0, k % T) for k in range(args.steps * T)], threads)
+        qps = args.steps * T / t
+        sample = ("per step: the %d query tokens of 1 sequence of %d tokens (shapes of %s): "
+                  "full index scan, top-16 and attention in the float64 C oracle; the %d steps "
+                  "run together on %d host threads" % (T, int(w.seq_lens[0]), args.workload,
+                                                       args.steps, threads))
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
